@@ -1,0 +1,285 @@
+"""Pins for the fp64 oracle: facts fixed by the method and by mathematics.
+
+Each ``pin_*`` takes an implementation object exposing the oracle's interface
+(``quadratic``, ``recurrent``, ``blocked``, ``state``, ``decode_step``) and
+raises AssertionError when that implementation disagrees with a fact that
+does not come from the implementation itself:
+
+* a hand-worked example (``tests/golden/hand_example.json``);
+* closed forms on special inputs (one token; one-hot queries and keys, whose
+  result is a count-and-select; all-ones scores, whose result is a cumulative
+  sum);
+* exact rational brute force on tiny integer inputs;
+* invariants: three associations of the sum agree for every block size B,
+  linearity in Q, K and V, causality, per-sequence independence of packed
+  sequences, additivity of the state, prefill/decode continuity and resume
+  from a carried-in state.
+
+The method is causal linear attention as described on the page "MiniMax-01
+Lightning Attention", section "Lightning Attention 设计": left product inside a
+block, right product across blocks through a d x d KV state, and an O(d^2)
+recurrent update at inference.
+"""
+from __future__ import annotations
+
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_example.json")
+
+
+def _rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    scale = max(np.abs(b).max(initial=0.0), 1e-300)
+    return float(np.abs(a - b).max(initial=0.0) / scale)
+
+
+def _close(a, b, tol, what):
+    r = _rel(a, b)
+    assert r <= tol, f"{what}: relative max error {r:.3e} > {tol:.1e}"
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# --------------------------------------------------------------------------- golden
+def pin_golden(impl):
+    g = json.load(open(GOLDEN))
+    q, k, v = (np.array(g[x], dtype=np.float64) for x in ("q", "k", "v"))
+    o = np.array(g["o"], dtype=np.float64)
+    assert np.array_equal(impl.quadratic(q, k, v), o), "quadratic != hand example"
+    assert np.array_equal(impl.recurrent(q, k, v), o), "recurrent != hand example"
+    for B in (1, 2, 3):
+        assert np.array_equal(impl.blocked(q, k, v, B), o), f"blocked(B={B}) != hand example"
+    st = np.array(g["state"], dtype=np.float64)
+    assert np.array_equal(impl.state(k, v), st), "state != hand example"
+    dq, dk, dv = (np.array(g["decode"][x], dtype=np.float64) for x in ("q", "k", "v"))
+    do, ds = impl.decode_step(dq, dk, dv, st)
+    assert np.array_equal(do, np.array(g["decode"]["o"], dtype=np.float64)), "decode o != hand example"
+    assert np.array_equal(ds, np.array(g["decode"]["state"], dtype=np.float64)), "decode state != hand example"
+
+
+# --------------------------------------------------------------------------- closed forms
+def pin_single_token(impl):
+    """n = 1: O_1 = (q_1 . k_1) v_1; with a carried-in state add q_1 S0."""
+    r = _rng(11)
+    H, d = 3, 5
+    q, k, v = (r.integers(-4, 5, size=(1, H, d)).astype(np.float64) for _ in range(3))
+    want = np.zeros((1, H, d))
+    for h in range(H):
+        score = sum(q[0, h, i] * k[0, h, i] for i in range(d))
+        want[0, h] = score * v[0, h]
+    for f in (impl.quadratic, impl.recurrent):
+        assert np.array_equal(f(q, k, v), want), "single token closed form"
+    assert np.array_equal(impl.blocked(q, k, v, 4), want), "single token closed form (blocked)"
+    S0 = r.integers(-3, 4, size=(1, H, d, d)).astype(np.float64)
+    want0 = want.copy()
+    for h in range(H):
+        for j in range(d):
+            want0[0, h, j] += sum(q[0, h, i] * S0[0, h, i, j] for i in range(d))
+    for f in (impl.quadratic, impl.recurrent):
+        assert np.array_equal(f(q, k, v, init=S0), want0), "single token with init state"
+    assert np.array_equal(impl.blocked(q, k, v, 2, init=S0), want0), "single token with init (blocked)"
+    # the state of one token is the outer product k^T v (row index from k)
+    st = impl.state(k, v)
+    for h in range(H):
+        for i in range(d):
+            for j in range(d):
+                assert st[0, h, i, j] == k[0, h, i] * v[0, h, j], "state orientation k_i v_j"
+
+
+def pin_onehot(impl):
+    """q_t = e_{a_t}, k_s = e_{c_s}: O_t = sum of v_s over s <= t with c_s == a_t."""
+    r = _rng(12)
+    T, H, d = 41, 2, 6
+    a = r.integers(0, d, size=(T, H))
+    c = r.integers(0, d, size=(T, H))
+    q = np.zeros((T, H, d)); k = np.zeros((T, H, d))
+    for t in range(T):
+        for h in range(H):
+            q[t, h, a[t, h]] = 1.0
+            k[t, h, c[t, h]] = 1.0
+    v = r.integers(-9, 10, size=(T, H, d)).astype(np.float64)
+    cu = [0, 17, 17, 41]
+    want = np.zeros((T, H, d))
+    for si in range(len(cu) - 1):
+        for h in range(H):
+            for t in range(cu[si], cu[si + 1]):
+                for s in range(cu[si], t + 1):
+                    if c[s, h] == a[t, h]:
+                        want[t, h] += v[s, h]
+    assert np.array_equal(impl.quadratic(q, k, v, cu), want), "one-hot count (quadratic)"
+    assert np.array_equal(impl.recurrent(q, k, v, cu), want), "one-hot count (recurrent)"
+    for B in (1, 3, 16, 64):
+        assert np.array_equal(impl.blocked(q, k, v, B, cu), want), f"one-hot count (blocked B={B})"
+
+
+def pin_cumsum(impl):
+    """All scores equal to one (q = k = e_0): O is the per-sequence cumulative sum of V."""
+    r = _rng(13)
+    T, H, d = 30, 2, 4
+    q = np.zeros((T, H, d)); q[:, :, 0] = 1.0
+    k = q.copy()
+    v = r.integers(-5, 6, size=(T, H, d)).astype(np.float64)
+    cu = [0, 7, 30]
+    want = np.concatenate([np.cumsum(v[cu[i]:cu[i + 1]], axis=0) for i in range(2)])
+    for f in (impl.quadratic, impl.recurrent):
+        assert np.array_equal(f(q, k, v, cu), want), "cumsum closed form"
+    assert np.array_equal(impl.blocked(q, k, v, 4, cu), want), "cumsum closed form (blocked)"
+
+
+def pin_bruteforce_exact(impl):
+    """Exact rational arithmetic over every (t, s) pair on tiny integer inputs."""
+    r = _rng(14)
+    T, H, d = 7, 2, 3
+    q, k, v = (r.integers(-3, 4, size=(T, H, d)) for _ in range(3))
+    cu = [0, 3, 7]
+    want = np.zeros((T, H, d))
+    for si in range(2):
+        for h in range(H):
+            for t in range(cu[si], cu[si + 1]):
+                acc = [Fraction(0)] * d
+                for s in range(cu[si], t + 1):
+                    score = Fraction(0)
+                    for i in range(d):
+                        score += Fraction(int(q[t, h, i])) * Fraction(int(k[s, h, i]))
+                    for j in range(d):
+                        acc[j] += score * Fraction(int(v[s, h, j]))
+                want[t, h] = [float(x) for x in acc]
+    qf, kf, vf = (x.astype(np.float64) for x in (q, k, v))
+    assert np.array_equal(impl.quadratic(qf, kf, vf, cu), want), "brute force (quadratic)"
+    assert np.array_equal(impl.recurrent(qf, kf, vf, cu), want), "brute force (recurrent)"
+    for B in (1, 2, 3, 5, 8):
+        assert np.array_equal(impl.blocked(qf, kf, vf, B, cu), want), f"brute force (blocked B={B})"
+
+
+# --------------------------------------------------------------------------- invariants
+def pin_forms_agree(impl):
+    """quadratic == recurrent == blocked(B) for every B in 1..n (fp64, 1e-10 relative)."""
+    r = _rng(15)
+    T, H, d = 67, 2, 5
+    q, k, v = (r.standard_normal((T, H, d)) for _ in range(3))
+    ref = impl.quadratic(q, k, v)
+    _close(impl.recurrent(q, k, v), ref, 1e-10, "recurrent vs quadratic")
+    for B in range(1, T + 1):
+        _close(impl.blocked(q, k, v, B), ref, 1e-10, f"blocked(B={B}) vs quadratic")
+    # long sequence: recurrent vs quadratic
+    T2 = 1500
+    q, k, v = (r.standard_normal((T2, 1, 8)) / np.sqrt(8) for _ in range(3))
+    _close(impl.recurrent(q, k, v), impl.quadratic(q, k, v), 1e-10, "recurrent vs quadratic (n=1500)")
+    _close(impl.blocked(q, k, v, 256), impl.quadratic(q, k, v), 1e-10, "blocked(256) vs quadratic (n=1500)")
+
+
+def pin_linearity(impl):
+    """O is linear in each of Q, K and V separately."""
+    r = _rng(16)
+    T, H, d = 23, 2, 4
+    q, k, v, x = (r.standard_normal((T, H, d)) for _ in range(4))
+    alpha = 1.75
+    o = impl.recurrent(q, k, v)
+    _close(impl.recurrent(q, k, alpha * v + x), alpha * o + impl.recurrent(q, k, x), 1e-10, "linear in V")
+    _close(impl.recurrent(alpha * q + x, k, v), alpha * o + impl.recurrent(x, k, v), 1e-10, "linear in Q")
+    _close(impl.blocked(q, alpha * k + x, v, 5), alpha * o + impl.blocked(q, x, v, 5), 1e-10, "linear in K")
+
+
+def pin_causality(impl):
+    """Changing tokens after t0 leaves O_t (t <= t0) untouched; changing token t0 moves O_t0."""
+    r = _rng(17)
+    T, H, d, t0 = 20, 2, 4, 9
+    q, k, v = (r.standard_normal((T, H, d)) for _ in range(3))
+    base = {n: f(q, k, v) for n, f in (("q", impl.quadratic), ("r", impl.recurrent))}
+    base["b"] = impl.blocked(q, k, v, 4)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[t0 + 1:] += 3.0; k2[t0 + 1:] -= 2.0; v2[t0 + 1:] *= -5.0
+    for n, f in (("q", impl.quadratic), ("r", impl.recurrent)):
+        assert np.array_equal(f(q2, k2, v2)[: t0 + 1], base[n][: t0 + 1]), "future tokens leak into the past"
+    assert np.array_equal(impl.blocked(q2, k2, v2, 4)[: t0 + 1], base["b"][: t0 + 1]), "future leak (blocked)"
+    # the diagonal is part of the sum: token t0's own key/value moves O_t0
+    k3, v3 = k.copy(), v.copy()
+    k3[t0] += 1.0; v3[t0] += 1.0
+    for f in (impl.quadratic, impl.recurrent):
+        assert not np.allclose(f(q, k3, v3)[t0], base["r"][t0]), "diagonal term missing"
+    # and an earlier token moves every later output of its sequence
+    v4 = v.copy(); v4[0] += 1.0
+    assert not np.allclose(impl.recurrent(q, k, v4)[T - 1], base["r"][T - 1]), "earliest token ignored"
+
+
+def pin_varlen(impl):
+    """Packed sequences are independent: packing equals running each sequence alone."""
+    r = _rng(18)
+    lens = [5, 0, 13, 1, 9]
+    H, d = 2, 3
+    seqs = [tuple(r.standard_normal((n, H, d)) for _ in range(3)) for n in lens]
+    q = np.concatenate([s[0] for s in seqs]); k = np.concatenate([s[1] for s in seqs])
+    v = np.concatenate([s[2] for s in seqs])
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    packed = {"q": impl.quadratic(q, k, v, cu), "r": impl.recurrent(q, k, v, cu),
+              "b": impl.blocked(q, k, v, 4, cu)}
+    st = impl.state(k, v, cu)
+    for i, n in enumerate(lens):
+        sl = slice(int(cu[i]), int(cu[i + 1]))
+        if n == 0:
+            assert np.array_equal(st[i], np.zeros((H, d, d))), "empty sequence state"
+            continue
+        sq, sk, sv = seqs[i]
+        _close(packed["q"][sl], impl.quadratic(sq, sk, sv), 1e-12, "varlen (quadratic)")
+        _close(packed["r"][sl], impl.recurrent(sq, sk, sv), 1e-12, "varlen (recurrent)")
+        _close(packed["b"][sl], impl.blocked(sq, sk, sv, 4), 1e-12, "varlen (blocked)")
+        _close(st[i], impl.state(sk, sv)[0], 1e-12, "varlen state")
+
+
+def pin_state(impl):
+    """state(a || b) = state(a) + state(b); it equals the recurrent and blocked final states."""
+    r = _rng(19)
+    H, d = 2, 4
+    ka, va = (r.standard_normal((11, H, d)) for _ in range(2))
+    kb, vb = (r.standard_normal((6, H, d)) for _ in range(2))
+    k = np.concatenate([ka, kb]); v = np.concatenate([va, vb])
+    sab = impl.state(k, v)
+    _close(sab, impl.state(ka, va) + impl.state(kb, vb), 1e-12, "state additivity")
+    q = r.standard_normal(k.shape)
+    _, s_rec = impl.recurrent(q, k, v, return_state=True)
+    _, s_blk = impl.blocked(q, k, v, 4, return_state=True)
+    _close(s_rec, sab, 1e-12, "recurrent final state")
+    _close(s_blk, sab, 1e-12, "blocked final state")
+    S0 = r.standard_normal((1, H, d, d))
+    _close(impl.state(k, v, init=S0), sab + S0, 1e-12, "state with init")
+
+
+def pin_decode_continuity(impl):
+    """Prefill of the first m tokens, then decode steps, reproduces the full prefill rows."""
+    r = _rng(20)
+    T, m, H, d = 19, 12, 2, 4
+    q, k, v = (r.standard_normal((T, H, d)) for _ in range(3))
+    full = impl.quadratic(q, k, v)
+    st = impl.state(k[:m], v[:m])
+    for t in range(m, T):
+        o, st = impl.decode_step(q[t:t + 1], k[t:t + 1], v[t:t + 1], st)
+        _close(o[0], full[t], 1e-10, f"decode step at t={t}")
+    _close(st, impl.state(k, v), 1e-12, "decode final state")
+    # one step from a zero state is (q . k) v
+    o1, _ = impl.decode_step(q[:1], k[:1], v[:1], np.zeros((1, H, d, d)))
+    _close(o1, impl.quadratic(q[:1], k[:1], v[:1]), 1e-14, "decode from zero state")
+
+
+def pin_resume(impl):
+    """Prefill of b with init = state(a) equals the b rows of prefill over a || b."""
+    r = _rng(21)
+    H, d = 2, 4
+    q, k, v = (r.standard_normal((25, H, d)) for _ in range(3))
+    full = impl.recurrent(q, k, v)
+    S0 = impl.state(k[:10], v[:10])
+    for name, o in (("quadratic", impl.quadratic(q[10:], k[10:], v[10:], init=S0)),
+                    ("recurrent", impl.recurrent(q[10:], k[10:], v[10:], init=S0)),
+                    ("blocked", impl.blocked(q[10:], k[10:], v[10:], 4, init=S0))):
+        _close(o, full[10:], 1e-10, f"resume from carried state ({name})")
+
+
+ALL_PINS = [pin_golden, pin_single_token, pin_onehot, pin_cumsum, pin_bruteforce_exact,
+            pin_forms_agree, pin_linearity, pin_causality, pin_varlen, pin_state,
+            pin_decode_continuity, pin_resume]

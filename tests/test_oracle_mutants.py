@@ -1,0 +1,154 @@
+"""The pins are sharp: each plausible mistake, planted in a small numpy twin of
+the oracle on the CPU, fails at least one pin, while the twin without a
+mistake passes them all."""
+import numpy as np
+import pytest
+
+import pins
+
+
+class Twin:
+    """numpy restatement of the oracle's five functions with an optional planted bug."""
+
+    def __init__(self, bug=None):
+        self.bug = bug
+
+    # helpers ---------------------------------------------------------------
+    @staticmethod
+    def _cu(T, cu):
+        return [0, T] if cu is None else [int(x) for x in cu]
+
+    def _outer(self, kv, vv):
+        return np.outer(vv, kv) if self.bug == "transpose_state" else np.outer(kv, vv)
+
+    def _mask(self, n):
+        if self.bug == "exclusive_mask":
+            return np.tril(np.ones((n, n)), -1)
+        if self.bug == "anticausal":
+            return np.triu(np.ones((n, n)))
+        return np.tril(np.ones((n, n)))
+
+    def _scores(self, Q, K):
+        return K @ Q.T if self.bug == "swap_qk" else Q @ K.T
+
+    def _post(self, o, d):
+        return o / np.sqrt(d) if self.bug == "scaled" else o
+
+    def _init(self, init, s, h, d):
+        if init is None or self.bug == "drop_init":
+            return np.zeros((d, d))
+        return np.array(init[s, h], dtype=np.float64)
+
+    # interface ---------------------------------------------------------------
+    def quadratic(self, q, k, v, cu_seqlens=None, init=None):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        o = np.zeros_like(q)
+        for s in range(len(cu) - 1):
+            a, b = cu[s], cu[s + 1]
+            for h in range(H):
+                Q, K, V = q[a:b, h], k[a:b, h], v[a:b, h]
+                o[a:b, h] = (self._scores(Q, K) * self._mask(b - a)) @ V + Q @ self._init(init, s, h, d)
+        return self._post(o, d)
+
+    def recurrent(self, q, k, v, cu_seqlens=None, init=None, return_state=False):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        o = np.zeros_like(q)
+        st = np.zeros((len(cu) - 1, H, d, d))
+        carry = [np.zeros((d, d)) for _ in range(H)]
+        for s in range(len(cu) - 1):
+            for h in range(H):
+                S = carry[h] if self.bug == "no_reset" else self._init(init, s, h, d)
+                for t in range(cu[s], cu[s + 1]):
+                    if self.bug == "output_before_update":
+                        o[t, h] = q[t, h] @ S
+                        S = S + self._outer(k[t, h], v[t, h])
+                    else:
+                        S = S + self._outer(k[t, h], v[t, h])
+                        o[t, h] = q[t, h] @ S
+                st[s, h] = S
+                carry[h] = S
+        o = self._post(o, d)
+        return (o, st) if return_state else o
+
+    def blocked(self, q, k, v, B, cu_seqlens=None, init=None, return_state=False):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        o = np.zeros_like(q)
+        st = np.zeros((len(cu) - 1, H, d, d))
+        for s in range(len(cu) - 1):
+            a, e = cu[s], cu[s + 1]
+            for h in range(H):
+                KV = self._init(init, s, h, d)
+                starts = list(range(a, e, B))
+                for i, b0 in enumerate(starts):
+                    b1 = starts[i + 1] if i + 1 < len(starts) else e
+                    Q, K, V = q[b0:b1, h], k[b0:b1, h], v[b0:b1, h]
+                    upd = sum((self._outer(K[u], V[u]) for u in range(b1 - b0)), np.zeros((d, d)))
+                    if self.bug == "prefix_inclusive":
+                        KV = KV + upd
+                    mask = np.ones((b1 - b0, b1 - b0)) if self.bug == "block_nomask" else self._mask(b1 - b0)
+                    o[b0:b1, h] = (self._scores(Q, K) * mask) @ V
+                    if self.bug != "no_inter":
+                        o[b0:b1, h] += Q @ KV
+                    if self.bug != "prefix_inclusive":
+                        KV = KV + upd
+                st[s, h] = KV
+        o = self._post(o, d)
+        return (o, st) if return_state else o
+
+    def state(self, k, v, cu_seqlens=None, init=None):
+        k, v = (np.asarray(x, dtype=np.float64) for x in (k, v))
+        T, H, d = k.shape
+        cu = self._cu(T, cu_seqlens)
+        st = np.zeros((len(cu) - 1, H, d, d))
+        for s in range(len(cu) - 1):
+            for h in range(H):
+                S = self._init(init, s, h, d)
+                for t in range(cu[s], cu[s + 1]):
+                    S = S + self._outer(k[t, h], v[t, h])
+                st[s, h] = S
+        return st
+
+    def decode_step(self, q, k, v, state_in):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        Bt, H, d = q.shape
+        st = np.array(state_in, dtype=np.float64, copy=True)
+        o = np.zeros_like(q)
+        for b in range(Bt):
+            for h in range(H):
+                if self.bug == "output_before_update":
+                    o[b, h] = q[b, h] @ st[b, h]
+                    st[b, h] += self._outer(k[b, h], v[b, h])
+                else:
+                    st[b, h] += self._outer(k[b, h], v[b, h])
+                    o[b, h] = q[b, h] @ st[b, h]
+        return self._post(o, d), st
+
+
+BUGS = ["exclusive_mask", "anticausal", "transpose_state", "drop_init", "output_before_update",
+        "no_inter", "prefix_inclusive", "no_reset", "swap_qk", "scaled", "block_nomask"]
+
+
+def _failing_pins(impl):
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+def test_clean_twin_passes_every_pin():
+    assert _failing_pins(Twin()) == []
+
+
+@pytest.mark.parametrize("bug", BUGS)
+def test_planted_bug_is_caught(bug):
+    failed = _failing_pins(Twin(bug))
+    assert failed, f"no pin catches the planted bug {bug!r}"
