@@ -1,0 +1,250 @@
+"""B200 (sm_100a) Lightning Attention: block-tiled causal linear attention.
+
+Thin Python binding over the C ABI of ``liblightning_attention.so`` (declared
+in ``include/lightning_attention.h``). Every step of the computation runs in
+the library's CUDA kernels; this module only marshals torch tensors into
+pointers and sizes. There is no fallback: if the library has not been built
+(``python -m causal_linear_attention_02_b200.build``), every call raises.
+
+The ``la_*`` functions mirror the C entry points one to one and return the
+integer status. ``prefill``, ``state_from_prefill`` and ``decode_step`` are
+conveniences that size and allocate outputs/workspace with torch, call the
+``la_*`` function and raise ``LightningError`` on a non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "LightningError", "LA_BF16", "LA_FP32", "STATUS", "library_path", "load_library",
+    "la_prefill_workspace_size", "la_prefill", "la_state_workspace_size", "la_state_from_prefill",
+    "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_status_string", "la_version",
+    "prefill", "state_from_prefill", "decode_step", "device_status", "uses_tensor_cores",
+]
+
+LA_BF16 = 0
+LA_FP32 = 1
+STATUS = {
+    0: "LA_OK", 1: "LA_ERR_INVALID_ARGUMENT", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_MISALIGNED",
+    4: "LA_ERR_WORKSPACE_TOO_SMALL", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT", 7: "LA_ERR_BAD_SEQLENS",
+}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liblightning_attention.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class LightningError(RuntimeError):
+    """A library call returned a non-zero status, or the library is missing."""
+
+    def __init__(self, msg, status=None):
+        super().__init__(msg)
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load the CUDA library (raises LightningError if it was never built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise LightningError(
+                f"{_LIB_PATH} is missing: build it with `python -m causal_linear_attention_02_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64
+        lib.la_prefill_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+        lib.la_prefill_workspace_size.restype = sz
+        lib.la_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp, sz, vp]
+        lib.la_prefill.restype = i32
+        lib.la_state_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+        lib.la_state_workspace_size.restype = sz
+        lib.la_state_from_prefill.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, sz, vp]
+        lib.la_state_from_prefill.restype = i32
+        lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        lib.la_decode_step.restype = i32
+        lib.la_get_device_status.argtypes = [vp]
+        lib.la_get_device_status.restype = i32
+        lib.la_status_string.argtypes = [i32]
+        lib.la_status_string.restype = ctypes.c_char_p
+        lib.la_set_kernel_timer.argtypes = [vp, vp]
+        lib.la_set_kernel_timer.restype = i32
+        lib.la_version.argtypes = []
+        lib.la_version.restype = i32
+        _lib = lib
+        return lib
+
+
+# ---------------------------------------------------------------- C ABI mirrors
+def la_prefill_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) -> int:
+    return int(load_library().la_prefill_workspace_size(total_tokens, num_seqs, heads, d, B, dtype))
+
+
+def la_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state,
+               workspace, workspace_bytes, stream) -> int:
+    return int(load_library().la_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype,
+                                         init_state, workspace, workspace_bytes, stream))
+
+
+def la_state_workspace_size(total_tokens, num_seqs, heads, d, dtype) -> int:
+    return int(load_library().la_state_workspace_size(total_tokens, num_seqs, heads, d, dtype))
+
+
+def la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype, init_state, state_out,
+                          workspace, workspace_bytes, stream) -> int:
+    return int(load_library().la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype,
+                                                    init_state, state_out, workspace, workspace_bytes, stream))
+
+
+def la_decode_step(q, k, v, state, o, batch, heads, d, dtype, stream) -> int:
+    return int(load_library().la_decode_step(q, k, v, state, o, batch, heads, d, dtype, stream))
+
+
+def la_get_device_status(stream) -> int:
+    return int(load_library().la_get_device_status(stream))
+
+
+def la_status_string(status: int) -> str:
+    return load_library().la_status_string(int(status)).decode()
+
+
+def la_set_kernel_timer(start_event, stop_event) -> int:
+    return int(load_library().la_set_kernel_timer(start_event, stop_event))
+
+
+def la_version() -> int:
+    return int(load_library().la_version())
+
+
+# ---------------------------------------------------------------- marshalling helpers
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return LA_BF16
+    if t == torch.float32:
+        return LA_FP32
+    raise LightningError(f"unsupported dtype {t} (bf16 or fp32)", 2)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, device=None):
+    if not t.is_cuda:
+        raise LightningError(f"{name} must be a CUDA tensor", 1)
+    if not t.is_contiguous():
+        raise LightningError(f"{name} must be contiguous", 1)
+    if device is not None and t.device != device:
+        raise LightningError(f"{name} is on {t.device}, expected {device}", 1)
+
+
+def _raise(status: int, what: str):
+    if status != 0:
+        raise LightningError(f"{what}: {STATUS.get(status, status)} ({la_status_string(status)})", status)
+
+
+def uses_tensor_cores(dtype: torch.dtype, d: int, B: int) -> bool:
+    """True when la_prefill runs this shape on the tcgen05 path (bf16, d=128, B in {128, 256})."""
+    return dtype == torch.bfloat16 and d == 128 and B in (128, 256)
+
+
+# ---------------------------------------------------------------- conveniences
+def prefill(q, k, v, cu_seqlens=None, B: int = 256, init_state=None, out=None, workspace=None, stream=None):
+    """O = causal linear attention of packed [T, H, d] q, k, v (see la_prefill)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise LightningError("q, k, v must share one [T, H, d] shape and dtype", 1)
+    T, H, d = q.shape
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", q.device)
+        if cu_seqlens.dtype != torch.int32:
+            raise LightningError("cu_seqlens must be int32", 1)
+        nseq = cu_seqlens.numel() - 1
+    else:
+        nseq = 1
+    if init_state is not None:
+        _need(init_state, "init_state", q.device)
+        if init_state.dtype != torch.float32 or tuple(init_state.shape) != (nseq, H, d, d):
+            raise LightningError("init_state must be fp32 [num_seqs, H, d, d]", 1)
+    code = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.device)
+    ws_bytes = la_prefill_workspace_size(T, nseq, H, d, B, code)
+    if ws_bytes == 0:
+        raise LightningError(f"unsupported prefill shape T={T} H={H} d={d} B={B}", 2)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    status = la_prefill(_p(q), _p(k), _p(v), _p(out), _p(cu_seqlens), nseq, T, H, d, B, code, _p(init_state),
+                        _p(workspace), workspace.numel() * workspace.element_size(),
+                        _stream_handle(stream, q.device))
+    _raise(status, "la_prefill")
+    return out
+
+
+def state_from_prefill(k, v, cu_seqlens=None, init_state=None, out=None, workspace=None, stream=None):
+    """fp32 [num_seqs, H, d, d] state S0 + sum_t k_t^T v_t per sequence (see la_state_from_prefill)."""
+    _need(k, "k"); _need(v, "v", k.device)
+    if k.dim() != 3 or v.shape != k.shape or v.dtype != k.dtype:
+        raise LightningError("k, v must share one [T, H, d] shape and dtype", 1)
+    T, H, d = k.shape
+    nseq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", k.device)
+    if out is None:
+        out = torch.empty((nseq, H, d, d), dtype=torch.float32, device=k.device)
+    _need(out, "out", k.device)
+    if init_state is not None:
+        _need(init_state, "init_state", k.device)
+    code = _dtype_code(k.dtype)
+    ws_bytes = la_state_workspace_size(T, nseq, H, d, code)
+    if ws_bytes == 0:
+        raise LightningError(f"unsupported state shape T={T} H={H} d={d}", 2)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device)
+    status = la_state_from_prefill(_p(k), _p(v), _p(cu_seqlens), nseq, T, H, d, code, _p(init_state), _p(out),
+                                   _p(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream_handle(stream, k.device))
+    _raise(status, "la_state_from_prefill")
+    return out
+
+
+def decode_step(q, k, v, state, out=None, stream=None):
+    """One step S <- S + k^T v, o = q S on [batch, H, d] inputs; state updated in place."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("state", state)):
+        _need(t, n, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise LightningError("q, k, v must share one [batch, H, d] shape", 1)
+    batch, H, d = q.shape
+    if state.dtype != torch.float32 or tuple(state.shape) != (batch, H, d, d):
+        raise LightningError("state must be fp32 [batch, H, d, d]", 1)
+    code = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    status = la_decode_step(_p(q), _p(k), _p(v), _p(state), _p(out), batch, H, d, code,
+                            _stream_handle(stream, q.device))
+    _raise(status, "la_decode_step")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    return la_get_device_status(_stream_handle(stream, dev))

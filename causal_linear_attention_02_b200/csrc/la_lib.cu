@@ -1,0 +1,413 @@
+// C ABI of the Lightning Attention library (declared in include/lightning_attention.h).
+// Host side: argument validation, workspace layout, TMA tensor-map encoding and
+// the launch sequence of each entry point. The whole library is this one
+// translation unit (kernels come in through the .cuh files), so the per-device
+// status word is a single __device__ symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <mutex>
+#include <stdint.h>
+#include <string.h>
+
+#include "lightning_attention.h"
+#include "common.cuh"
+#include "prep.cuh"
+#include "simt.cuh"
+#include "decode.cuh"
+#include "tc.cuh"
+
+namespace {
+
+using la::BlockEntry;
+using la::Control;
+
+constexpr uint64_t kWaitNs = 4000000000ull;   // bound on any single device-side wait (4 s)
+constexpr int kStateBlock = 2048;             // tokens per partial state in la_state_from_prefill
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t esize(la_dtype t) { return t == LA_BF16 ? 2 : 4; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+bool supported_d(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
+bool supported_B(int B) { return B == 64 || B == 128 || B == 256; }
+bool use_tensor_cores(la_dtype dt, int d, int B) { return dt == LA_BF16 && d == 128 && (B == 128 || B == 256); }
+
+// ------------------------------------------------------------------ workspace layouts
+struct Layout {
+    int64_t max_blocks = 0;
+    size_t off_seq_blk = 0, off_table = 0, off_U = 0, off_prefix = 0, total = 0;
+};
+
+Layout prefill_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt) {
+    Layout L;
+    L.max_blocks = (T + B - 1) / B + nseq;
+    size_t off = sizeof(Control);
+    L.off_seq_blk = off; off = align_up(off + sizeof(int32_t) * (size_t)(nseq + 1), 256);
+    L.off_table = off;   off = align_up(off + sizeof(BlockEntry) * (size_t)L.max_blocks, 256);
+    const size_t dd = (size_t)d * d;
+    L.off_U = off;       off = align_up(off + 4 * dd * (size_t)H * (size_t)L.max_blocks, 256);
+    const size_t pre_es = use_tensor_cores(dt, d, B) ? 2 : 4;
+    L.off_prefix = off;  off = align_up(off + pre_es * dd * (size_t)H * (size_t)L.max_blocks, 256);
+    L.total = off;
+    return L;
+}
+
+Layout state_layout(int64_t T, int nseq, int H, int d) {
+    Layout L;
+    L.max_blocks = (T + kStateBlock - 1) / kStateBlock + nseq;
+    size_t off = sizeof(Control);
+    L.off_seq_blk = off; off = align_up(off + sizeof(int32_t) * (size_t)(nseq + 1), 256);
+    L.off_table = off;   off = align_up(off + sizeof(BlockEntry) * (size_t)L.max_blocks, 256);
+    L.off_U = off;       off = align_up(off + 4 * (size_t)d * d * (size_t)H * (size_t)L.max_blocks, 256);
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------------ TMA tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [T][H][d] bf16 viewed as 3D {d, H, T}; box {64, 1, rows}, 128-byte swizzle.
+bool map_tokens(CUtensorMap* m, const void* base, int64_t T, int H, int d, int rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)rows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [rows][d] viewed as 2D {d, rows}; box {64, 128}, 128-byte swizzle.
+bool map_matrix(CUtensorMap* m, const void* base, int64_t rows, int d) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+la_status cuda_check() { return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+// One-shot per-thread timer around the main kernel of the next call (la_set_kernel_timer).
+thread_local cudaEvent_t t_timer_start = nullptr, t_timer_stop = nullptr;
+
+struct MainKernelTimer {
+    cudaStream_t st;
+    cudaEvent_t a, b;
+    explicit MainKernelTimer(cudaStream_t s) : st(s), a(t_timer_start), b(t_timer_stop) {
+        t_timer_start = t_timer_stop = nullptr;
+        if (a) cudaEventRecord(a, st);
+    }
+    ~MainKernelTimer() {
+        if (b) cudaEventRecord(b, st);
+    }
+};
+
+// ------------------------------------------------------------------ launch helpers
+la_status launch_block_table(const int32_t* cu, int nseq, int64_t T, int B, const Layout& L, uint8_t* ws,
+                             cudaStream_t st) {
+    Control* ctrl = reinterpret_cast<Control*>(ws);
+    int32_t* seq_blk = reinterpret_cast<int32_t*>(ws + L.off_seq_blk);
+    BlockEntry* table = reinterpret_cast<BlockEntry*>(ws + L.off_table);
+    la::seq_blocks_kernel<<<1, 1024, 0, st>>>(cu, nseq, T, B, seq_blk, ctrl);
+    const int64_t nb = (L.max_blocks + 255) / 256;
+    la::fill_block_table_kernel<<<(unsigned)nb, 256, 0, st>>>(cu, nseq, T, B, seq_blk, ctrl, table, L.max_blocks);
+    return cuda_check();
+}
+
+template <typename Tin, int D>
+la_status prefill_simt_main(const void* q, const void* k, const void* v, void* o, int H, int B,
+                            const Layout& L, uint8_t* ws, cudaStream_t st) {
+    const Control* ctrl = reinterpret_cast<const Control*>(ws);
+    const BlockEntry* table = reinterpret_cast<const BlockEntry*>(ws + L.off_table);
+    const float* prefix = reinterpret_cast<const float*>(ws + L.off_prefix);
+    constexpr size_t smem = la::simt::prefill_simt_smem<D>();
+    if (cudaFuncSetAttribute(la::simt::prefill_simt<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return LA_ERR_CUDA;
+    const int64_t grid = L.max_blocks * H * (B / 64);
+    la::simt::prefill_simt<Tin, D><<<(unsigned)grid, la::simt::THREADS, smem, st>>>(
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, prefix, table, ctrl, H, B);
+    return cuda_check();
+}
+
+template <typename Tin, int D>
+la_status state_simt_launch(const void* k, const void* v, int H, const Layout& L, uint8_t* ws, cudaStream_t st) {
+    const Control* ctrl = reinterpret_cast<const Control*>(ws);
+    const BlockEntry* table = reinterpret_cast<const BlockEntry*>(ws + L.off_table);
+    float* U = reinterpret_cast<float*>(ws + L.off_U);
+    la::simt::block_state_simt<Tin, D><<<(unsigned)(L.max_blocks * H), la::simt::THREADS, 0, st>>>(
+        (const Tin*)k, (const Tin*)v, table, ctrl, H, U);
+    return cuda_check();
+}
+
+#define LA_DISPATCH_D(d, FN, ...)                          \
+    switch (d) {                                           \
+        case 16: return FN<16>(__VA_ARGS__);               \
+        case 32: return FN<32>(__VA_ARGS__);               \
+        case 48: return FN<48>(__VA_ARGS__);               \
+        case 64: return FN<64>(__VA_ARGS__);               \
+        case 80: return FN<80>(__VA_ARGS__);               \
+        case 96: return FN<96>(__VA_ARGS__);               \
+        case 112: return FN<112>(__VA_ARGS__);             \
+        case 128: return FN<128>(__VA_ARGS__);             \
+        default: return LA_ERR_UNSUPPORTED;                \
+    }
+
+template <int D>
+la_status simt_states(la_dtype dt, const void* k, const void* v, int H, const Layout& L, uint8_t* ws,
+                      cudaStream_t st) {
+    return dt == LA_BF16 ? state_simt_launch<__nv_bfloat16, D>(k, v, H, L, ws, st)
+                         : state_simt_launch<float, D>(k, v, H, L, ws, st);
+}
+
+template <int D>
+la_status simt_prefill(la_dtype dt, const void* q, const void* k, const void* v, void* o, int H, int B,
+                       const Layout& L, uint8_t* ws, cudaStream_t st) {
+    return dt == LA_BF16 ? prefill_simt_main<__nv_bfloat16, D>(q, k, v, o, H, B, L, ws, st)
+                         : prefill_simt_main<float, D>(q, k, v, o, H, B, L, ws, st);
+}
+
+template <int D>
+la_status decode_launch(la_dtype dt, const void* q, const void* k, const void* v, float* state, void* o,
+                        int64_t pairs, cudaStream_t st) {
+    constexpr int nt = (D / 4) * la::decode_row_groups(D);
+    if (dt == LA_BF16)
+        la::decode_step_kernel<__nv_bfloat16, D><<<(unsigned)pairs, nt, 0, st>>>(
+            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, state, (__nv_bfloat16*)o);
+    else
+        la::decode_step_kernel<float, D><<<(unsigned)pairs, nt, 0, st>>>(
+            (const float*)q, (const float*)k, (const float*)v, state, (float*)o);
+    return cuda_check();
+}
+
+la_status simt_states_d(int d, la_dtype dt, const void* k, const void* v, int H, const Layout& L, uint8_t* ws,
+                        cudaStream_t st) {
+    LA_DISPATCH_D(d, simt_states, dt, k, v, H, L, ws, st);
+}
+la_status simt_prefill_d(int d, la_dtype dt, const void* q, const void* k, const void* v, void* o, int H, int B,
+                         const Layout& L, uint8_t* ws, cudaStream_t st) {
+    LA_DISPATCH_D(d, simt_prefill, dt, q, k, v, o, H, B, L, ws, st);
+}
+la_status decode_d(int d, la_dtype dt, const void* q, const void* k, const void* v, float* state, void* o,
+                   int64_t pairs, cudaStream_t st) {
+    LA_DISPATCH_D(d, decode_launch, dt, q, k, v, state, o, pairs, st);
+}
+
+// Common argument checks of the token-major entry points.
+la_status check_tokens(int64_t T, int nseq, int H, int d, la_dtype dt, const int32_t* cu) {
+    if (T < 0 || H < 1 || nseq < 1) return LA_ERR_INVALID_ARGUMENT;
+    if (cu == nullptr && nseq != 1) return LA_ERR_INVALID_ARGUMENT;
+    if (dt != LA_BF16 && dt != LA_FP32) return LA_ERR_UNSUPPORTED;
+    if (!supported_d(d)) return LA_ERR_UNSUPPORTED;
+    if (T >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;    // int32 cu_seqlens
+    if (cu && !aligned(cu, 4)) return LA_ERR_MISALIGNED;
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_prefill_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B, la_dtype dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || heads < 1 || !supported_d(d) || !supported_B(B) ||
+        (dtype != LA_BF16 && dtype != LA_FP32))
+        return 0;
+    return prefill_layout(total_tokens, num_seqs, heads, d, B, dtype).total;
+}
+
+size_t la_state_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, la_dtype dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || heads < 1 || !supported_d(d) || (dtype != LA_BF16 && dtype != LA_FP32))
+        return 0;
+    return state_layout(total_tokens, num_seqs, heads, d).total;
+}
+
+la_status la_prefill(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                     int num_seqs, int64_t total_tokens, int heads, int d, int B, la_dtype dtype,
+                     const float* init_state, void* workspace, size_t workspace_bytes, void* stream) {
+    la_status s = check_tokens(total_tokens, num_seqs, heads, d, dtype, cu_seqlens);
+    if (s != LA_OK) return s;
+    if (!supported_B(B)) return LA_ERR_UNSUPPORTED;
+    const size_t tensor_bytes = (size_t)total_tokens * heads * d * esize(dtype);
+    if (total_tokens > 0 && (!q || !k || !v || !o)) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return LA_ERR_MISALIGNED;
+    if (init_state && !aligned(init_state, 16)) return LA_ERR_MISALIGNED;
+    if (overlaps(o, tensor_bytes, q, tensor_bytes) || overlaps(o, tensor_bytes, k, tensor_bytes) ||
+        overlaps(o, tensor_bytes, v, tensor_bytes))
+        return LA_ERR_INVALID_ARGUMENT;
+    if (total_tokens == 0) return LA_OK;
+    const Layout L = prefill_layout(total_tokens, num_seqs, heads, d, B, dtype);
+    if (!workspace) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
+    if (overlaps(workspace, L.total, o, tensor_bytes)) return LA_ERR_INVALID_ARGUMENT;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const Control* ctrl = reinterpret_cast<const Control*>(ws);
+    const int32_t* seq_blk = reinterpret_cast<const int32_t*>(ws + L.off_seq_blk);
+    const BlockEntry* table = reinterpret_cast<const BlockEntry*>(ws + L.off_table);
+    float* U = reinterpret_cast<float*>(ws + L.off_U);
+    const int dd = d * d;
+
+    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, B, L, ws, st)) != LA_OK) return s;
+
+    if (use_tensor_cores(dtype, d, B)) {
+        CUtensorMap tq, tk, tv, tp;
+        __nv_bfloat16* prefix = reinterpret_cast<__nv_bfloat16*>(ws + L.off_prefix);
+        if (!map_tokens(&tq, q, total_tokens, heads, d, 128) || !map_tokens(&tk, k, total_tokens, heads, d, 64) ||
+            !map_tokens(&tv, v, total_tokens, heads, d, 64) ||
+            !map_matrix(&tp, prefix, L.max_blocks * heads * (int64_t)d, d))
+            return LA_ERR_CUDA;
+        // 1) block states U_b = K_b^T V_b on the tensor cores
+        const size_t smem_state = (size_t)2 * B * d * 2 + 1024 + 256;
+        if (cudaFuncSetAttribute(la::tc::block_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)la::tc::SMEM_STATE_MAX) != cudaSuccess)
+            return LA_ERR_CUDA;
+        la::tc::block_state_tc_kernel<<<(unsigned)(L.max_blocks * heads), 128, smem_state, st>>>(
+            tk, tv, U, table, ctrl, heads, B, kWaitNs);
+        if ((s = cuda_check()) != LA_OK) return s;
+        // 2) exclusive prefix over the blocks of every (sequence, head), rounded to bf16
+        dim3 sg((dd + 1023) / 1024, num_seqs * heads);
+        la::chain_scan_kernel<__nv_bfloat16><<<sg, 256, 0, st>>>(U, prefix, init_state, nullptr, seq_blk, ctrl,
+                                                                 num_seqs, heads, dd, true);
+        if ((s = cuda_check()) != LA_OK) return s;
+        // 3) intra-block left product + inter-block right product, fused in TMEM
+        if (cudaFuncSetAttribute(la::tc::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)la::tc::SMEM_PREFILL) != cudaSuccess)
+            return LA_ERR_CUDA;
+        const int64_t units = L.max_blocks * (B / 128) * heads;
+        const int sms = num_sms();
+        if (sms <= 0) return LA_ERR_CUDA;
+        const unsigned grid = (unsigned)(units < sms ? units : sms);
+        MainKernelTimer timer(st);
+        la::tc::prefill_tc_kernel<<<grid, 192, la::tc::SMEM_PREFILL, st>>>(
+            tq, tk, tv, tp, static_cast<__nv_bfloat16*>(o), table, ctrl, heads, B / 128, kWaitNs);
+        return cuda_check();
+    }
+
+    // CUDA-core path
+    if ((s = simt_states_d(d, dtype, k, v, heads, L, ws, st)) != LA_OK) return s;
+    dim3 sg((dd + 1023) / 1024, num_seqs * heads);
+    la::chain_scan_kernel<float><<<sg, 256, 0, st>>>(U, reinterpret_cast<float*>(ws + L.off_prefix), init_state,
+                                                     nullptr, seq_blk, ctrl, num_seqs, heads, dd, true);
+    if ((s = cuda_check()) != LA_OK) return s;
+    MainKernelTimer timer(st);
+    return simt_prefill_d(d, dtype, q, k, v, o, heads, B, L, ws, st);
+}
+
+la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_seqlens, int num_seqs,
+                                int64_t total_tokens, int heads, int d, la_dtype dtype, const float* init_state,
+                                float* state_out, void* workspace, size_t workspace_bytes, void* stream) {
+    la_status s = check_tokens(total_tokens, num_seqs, heads, d, dtype, cu_seqlens);
+    if (s != LA_OK) return s;
+    if (!state_out || (total_tokens > 0 && (!k || !v))) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(state_out, 16)) return LA_ERR_MISALIGNED;
+    if (init_state && !aligned(init_state, 16)) return LA_ERR_MISALIGNED;
+    const size_t state_bytes = (size_t)num_seqs * heads * d * d * 4;
+    if (init_state && init_state != state_out && overlaps(init_state, state_bytes, state_out, state_bytes))
+        return LA_ERR_INVALID_ARGUMENT;
+    const Layout L = state_layout(total_tokens, num_seqs, heads, d);
+    if (!workspace) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, kStateBlock, L, ws, st)) != LA_OK) return s;
+    if (total_tokens > 0 && (s = simt_states_d(d, dtype, k, v, heads, L, ws, st)) != LA_OK) return s;
+    const int dd = d * d;
+    dim3 sg((dd + 1023) / 1024, num_seqs * heads);
+    la::chain_scan_kernel<float><<<sg, 256, 0, st>>>(
+        reinterpret_cast<const float*>(ws + L.off_U), static_cast<float*>(nullptr), init_state, state_out,
+        reinterpret_cast<const int32_t*>(ws + L.off_seq_blk), reinterpret_cast<const Control*>(ws), num_seqs,
+        heads, dd, false);
+    return cuda_check();
+}
+
+la_status la_decode_step(const void* q, const void* k, const void* v, float* state, void* o, int batch, int heads,
+                         int d, la_dtype dtype, void* stream) {
+    if (batch < 0 || heads < 1) return LA_ERR_INVALID_ARGUMENT;
+    if (dtype != LA_BF16 && dtype != LA_FP32) return LA_ERR_UNSUPPORTED;
+    if (!supported_d(d)) return LA_ERR_UNSUPPORTED;
+    if (batch == 0) return LA_OK;
+    if (!q || !k || !v || !state || !o) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(state, 16))
+        return LA_ERR_MISALIGNED;
+    const int64_t pairs = (int64_t)batch * heads;
+    const size_t vec = (size_t)pairs * d * esize(dtype);
+    const size_t sbytes = (size_t)pairs * d * d * 4;
+    if (overlaps(o, vec, q, vec) || overlaps(o, vec, k, vec) || overlaps(o, vec, v, vec) ||
+        overlaps(o, vec, state, sbytes) || overlaps(state, sbytes, q, vec) || overlaps(state, sbytes, k, vec) ||
+        overlaps(state, sbytes, v, vec))
+        return LA_ERR_INVALID_ARGUMENT;
+    if (pairs >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;
+    MainKernelTimer timer(reinterpret_cast<cudaStream_t>(stream));
+    return decode_d(d, dtype, q, k, v, state, o, pairs, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return LA_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, la::g_status, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(la::g_status, &zero, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+    return static_cast<la_status>(v);
+}
+
+la_status la_set_kernel_timer(void* start_event, void* stop_event) {
+    if ((start_event == nullptr) != (stop_event == nullptr)) return LA_ERR_INVALID_ARGUMENT;
+    t_timer_start = reinterpret_cast<cudaEvent_t>(start_event);
+    t_timer_stop = reinterpret_cast<cudaEvent_t>(stop_event);
+    return LA_OK;
+}
+
+const char* la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "ok";
+        case LA_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case LA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case LA_ERR_MISALIGNED: return "pointer not 16-byte aligned (workspace: 256-byte)";
+        case LA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case LA_ERR_CUDA: return "CUDA error";
+        case LA_ERR_TIMEOUT: return "device-side wait timed out";
+        case LA_ERR_BAD_SEQLENS: return "cu_seqlens inconsistent with total_tokens";
+    }
+    return "unknown status";
+}
+
+int la_version(void) { return 100; }
+
+}  // extern "C"

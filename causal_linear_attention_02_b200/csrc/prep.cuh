@@ -1,0 +1,152 @@
+// Block table and block-state prefix scan.
+//
+// The method cuts every sequence into blocks of B tokens (page "首个线性注意力
+// 架构的大模型来了…", section "4.1 创新的线性注意力": 序列划分) and carries a
+// compact d x d prefix state from block to block (双阶段计算, 区块间处理). Packed
+// varlen sequences are independent ("data packing", page "MiniMax-01 Lightning
+// Attention", section "计算优化"), so blocks restart at every sequence start.
+#pragma once
+
+#include "common.cuh"
+
+namespace la {
+
+// Validates cu_seqlens and writes per-sequence block offsets:
+//   seq_blk[s] = sum_{s' < s} ceil(len_s' / B),  seq_blk[nseq] = total blocks.
+// One CTA of 1024 threads. cu == nullptr means one sequence of T tokens.
+__global__ void __launch_bounds__(1024) seq_blocks_kernel(const int32_t* __restrict__ cu, int nseq,
+                                                          int64_t T, int B, int32_t* __restrict__ seq_blk,
+                                                          Control* __restrict__ ctrl) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry;
+    __shared__ int bad;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) { carry = 0; bad = 0; }
+    __syncthreads();
+    // validation: cu[0] = 0, non-decreasing, cu[nseq] = T
+    if (cu != nullptr) {
+        for (int s = tid; s < nseq; s += blockDim.x) {
+            if (cu[s + 1] < cu[s]) bad = 1;
+        }
+        if (tid == 0 && (cu[0] != 0 || (int64_t)cu[nseq] != T)) bad = 1;
+    }
+    __syncthreads();
+    if (bad) {
+        if (tid == 0) {
+            ctrl->nblocks = 0;
+            ctrl->ok = 0;
+            ctrl->ticket = 0;
+            record_status(LA_ERR_BAD_SEQLENS);
+        }
+        return;
+    }
+    for (int base = 0; base < nseq; base += blockDim.x) {
+        const int s = base + tid;
+        int32_t nb = 0;
+        if (s < nseq) {
+            const int64_t len = cu ? (int64_t)(cu[s + 1] - cu[s]) : T;
+            nb = (int32_t)((len + B - 1) / B);
+        }
+        // block-wide exclusive scan of nb
+        int32_t x = nb;
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            int32_t w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+            for (int o = 1; o < 32; o <<= 1) {
+                int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[lane] = w;   // inclusive over warps
+        }
+        __syncthreads();
+        const int32_t excl = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + x - nb;
+        if (s < nseq) seq_blk[s] = excl;
+        __syncthreads();
+        if (tid == 0) carry += warp_sums[(blockDim.x >> 5) - 1];
+        __syncthreads();
+    }
+    if (tid == 0) {
+        seq_blk[nseq] = carry;
+        ctrl->nblocks = carry;
+        ctrl->ok = 1;
+        ctrl->ticket = 0;
+    }
+}
+
+// One thread per possible block: finds its sequence by binary search over
+// seq_blk and writes the BlockEntry.
+__global__ void fill_block_table_kernel(const int32_t* __restrict__ cu, int nseq, int64_t T, int B,
+                                        const int32_t* __restrict__ seq_blk,
+                                        const Control* __restrict__ ctrl,
+                                        BlockEntry* __restrict__ table, int64_t max_blocks) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= max_blocks || g >= ctrl->nblocks) return;
+    int lo = 0, hi = nseq - 1;          // last s with seq_blk[s] <= g
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (seq_blk[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int s = lo;
+    const int32_t b = (int32_t)(g - seq_blk[s]);
+    const int64_t start = cu ? (int64_t)cu[s] : 0;
+    const int64_t len = cu ? (int64_t)(cu[s + 1] - cu[s]) : T;
+    BlockEntry e;
+    e.seq = s;
+    e.blk = b;
+    e.tok0 = (int32_t)(start + (int64_t)b * B);
+    const int64_t rest = len - (int64_t)b * B;
+    e.len = (int32_t)(rest < B ? rest : B);
+    table[g] = e;
+}
+
+// Exclusive prefix over the blocks of every (sequence, head) chain:
+//   prefix[g] = S0 + sum_{blocks c of the same sequence before g} U[c]
+// and, optionally, the chain total S0 + sum_all U into state_out.
+// U, prefix: [block][H][d*d]; init, state_out: [nseq][H][d*d].
+// grid = (ceil(d*d / 1024), nseq * H), 256 threads, 4 consecutive elements per thread.
+template <typename OutT>
+__global__ void __launch_bounds__(256) chain_scan_kernel(const float* __restrict__ U,
+                                                         OutT* __restrict__ prefix,
+                                                         const float* init, float* state_out,
+                                                         const int32_t* __restrict__ seq_blk,
+                                                         const Control* __restrict__ ctrl,
+                                                         int nseq, int H, int dd, bool skip_last) {
+    if (!ctrl->ok) return;
+    const int chain = blockIdx.y;
+    const int s = chain / H, h = chain % H;
+    const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
+    if (e >= dd) return;
+    const int64_t g0 = seq_blk[s], g1 = seq_blk[s + 1];
+    float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (init) run = *reinterpret_cast<const float4*>(init + ((int64_t)s * H + h) * dd + e);
+    const int64_t gend = skip_last ? g1 - 1 : g1;   // the last block's U is not needed by a prefill
+    float4 nxt = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (g0 < gend) nxt = __ldcs(reinterpret_cast<const float4*>(U + ((int64_t)g0 * H + h) * dd + e));
+    for (int64_t g = g0; g < g1; ++g) {
+        if (prefix) {
+            OutT* p = prefix + ((int64_t)g * H + h) * dd + e;
+            if constexpr (sizeof(OutT) == 4) {
+                *reinterpret_cast<float4*>(p) = run;
+            } else {
+                uint2 w;
+                w.x = pack_bf16x2(run.x, run.y);
+                w.y = pack_bf16x2(run.z, run.w);
+                *reinterpret_cast<uint2*>(p) = w;
+            }
+        }
+        if (g < gend) {
+            const float4 u = nxt;
+            if (g + 1 < gend)
+                nxt = __ldcs(reinterpret_cast<const float4*>(U + ((int64_t)(g + 1) * H + h) * dd + e));
+            run.x += u.x; run.y += u.y; run.z += u.z; run.w += u.w;
+        }
+    }
+    if (state_out) *reinterpret_cast<float4*>(state_out + ((int64_t)s * H + h) * dd + e) = run;
+}
+
+}  // namespace la

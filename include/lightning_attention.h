@@ -1,0 +1,151 @@
+/*
+ * lightning_attention.h - C ABI of the B200 (sm_100a) Lightning Attention library.
+ *
+ * Causal linear attention with no decay, no feature map and no normaliser:
+ *
+ *     O_t = q_t . S0 + sum_{s in seq(t), s <= t} (q_t . k_s) v_s
+ *
+ * computed the Lightning way (page "MiniMax-01 Lightning Attention", section
+ * "Lightning Attention 设计"; page "首个线性注意力架构的大模型来了…", section
+ * "4.1 创新的线性注意力"): tokens are cut into blocks of B; inside a block the
+ * left product (Q_b K_b^T masked causally) V_b, across blocks the right product
+ * Q_b . KV with the d x d prefix state KV = S0 + sum_{c<b} K_c^T V_c. The
+ * decode step is the recurrent form S <- S + k^T v, o = q S, O(d^2) per token
+ * (same page, same section, and section "与标准 Softmax Attention 的区别").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    allocates no memory and performs no host synchronisation, except
+ *    la_get_device_status, which synchronises the given stream.
+ *  - q, k, v, o are packed token-major [total_tokens][heads][d], d fastest,
+ *    element type given by `dtype` (bf16 or fp32). Sequences of a varlen pack
+ *    are concatenated; cu_seqlens (device, int32 [num_seqs + 1]) holds their
+ *    offsets: cu_seqlens[0] = 0, non-decreasing, cu_seqlens[num_seqs] =
+ *    total_tokens. cu_seqlens = NULL means one sequence (num_seqs must be 1).
+ *    No state crosses a sequence boundary.
+ *  - States are fp32 [num_seqs or batch][heads][d][d], row-major, with
+ *    element [i][j] = sum_t k_t[i] * v_t[j] (row index from k, column from v).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every launch is enqueued on it; nothing else is touched.
+ *  - Arithmetic: fp32 accumulation throughout. For bf16 inputs the intra-block
+ *    scores are rounded to bf16 (RNE) before the P.V product and the prefix
+ *    state is rounded to bf16 (RNE) before the Q.KV product; O is rounded to
+ *    bf16 (RNE) once at the end. fp32 inputs are computed in fp32 end to end.
+ *
+ * Errors
+ * ------
+ *  Host-checkable argument errors are returned before anything is enqueued.
+ *  Launch errors return LA_ERR_CUDA. Conditions only visible on the device
+ *  (cu_seqlens inconsistent with total_tokens, a bounded wait that ran out)
+ *  set a per-device status word that la_get_device_status reports; the
+ *  affected launch then writes no output rows.
+ */
+#ifndef LIGHTNING_ATTENTION_H
+#define LIGHTNING_ATTENTION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARGUMENT = 1,    /* null pointer, negative size, aliasing, bad num_seqs   */
+    LA_ERR_UNSUPPORTED = 2,         /* shape or dtype outside the supported set               */
+    LA_ERR_MISALIGNED = 3,          /* a tensor pointer is not 16-byte aligned                */
+    LA_ERR_WORKSPACE_TOO_SMALL = 4, /* workspace_bytes below the *_workspace_size() result     */
+    LA_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed                   */
+    LA_ERR_TIMEOUT = 6,             /* device: a bounded wait ran out (reported by status)    */
+    LA_ERR_BAD_SEQLENS = 7          /* device: cu_seqlens not 0..total_tokens non-decreasing  */
+} la_status;
+
+typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
+
+/*
+ * Supported shapes: heads >= 1, d a multiple of 16 with 16 <= d <= 128,
+ * B in {64, 128, 256}, total_tokens >= 0, num_seqs >= 1.
+ * bf16 with d = 128 and B in {128, 256} runs on the tcgen05 tensor-core path;
+ * every other supported combination runs on the CUDA-core (SIMT) path.
+ */
+
+/* Bytes of device workspace la_prefill needs for these sizes (0 if unsupported). */
+size_t la_prefill_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                 la_dtype dtype);
+
+/*
+ * Block-tiled causal linear attention prefill.
+ *   q, k, v     in   [total_tokens][heads][d] (dtype)
+ *   o           out  [total_tokens][heads][d] (dtype); must not overlap q, k or v
+ *   cu_seqlens  in   device int32 [num_seqs + 1] or NULL (one sequence)
+ *   init_state  in   device fp32 [num_seqs][heads][d][d] carried-in state S0, or NULL (zero)
+ *   workspace   scratch, >= la_prefill_workspace_size(...) bytes, 256-byte aligned;
+ *               its contents on entry do not matter and are undefined on exit
+ * The result does not depend on B except through rounding.
+ */
+la_status la_prefill(const void* q, const void* k, const void* v, void* o,
+                     const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens,
+                     int heads, int d, int B, la_dtype dtype,
+                     const float* init_state, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/* Bytes of device workspace la_state_from_prefill needs (0 if unsupported). */
+size_t la_state_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, la_dtype dtype);
+
+/*
+ * Final recurrent state of each sequence after its prefill:
+ *   state_out[s][h] = S0[s][h] + sum_{t in seq s} k_t^T v_t    (fp32, [num_seqs][heads][d][d])
+ * This is the state the decode step continues from (the d x d KV state the
+ * right product carries, page "MiniMax-01 Lightning Attention", section
+ * "Lightning Attention 设计"). init_state may be NULL (zero) or equal to
+ * state_out (in-place accumulate); it must not partially overlap it.
+ */
+la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_seqlens,
+                                int num_seqs, int64_t total_tokens, int heads, int d,
+                                la_dtype dtype, const float* init_state, float* state_out,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One recurrent decode step for `batch` independent sequences:
+ *   S <- S + k^T v ;  o = q S      (o sees the updated state: s <= t)
+ *   q, k, v  in      [batch][heads][d] (dtype)
+ *   state    in/out  fp32 [batch][heads][d][d], updated in place
+ *   o        out     [batch][heads][d] (dtype); must not overlap q, k, v or state
+ * O(d^2) work per (sequence, head), independent of how many tokens came before
+ * (page "MiniMax-01 Lightning Attention", section "与标准 Softmax Attention 的区别").
+ */
+la_status la_decode_step(const void* q, const void* k, const void* v, float* state, void* o,
+                         int batch, int heads, int d, la_dtype dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the status word of the
+ * current device: LA_OK, LA_ERR_BAD_SEQLENS or LA_ERR_TIMEOUT (the first
+ * condition recorded since the last call), or LA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+la_status la_get_device_status(void* stream);
+
+/*
+ * Instrumentation (no counterpart on the pages). Arms a one-shot timer for the
+ * calling host thread: the next la_prefill or la_decode_step call made by this
+ * thread records `start_event` on its stream immediately before enqueuing its
+ * main kernel (the fused intra/inter-block kernel, or the decode kernel) and
+ * `stop_event` immediately after, then disarms. Both are cudaEvent_t passed as
+ * void*, owned by the caller; NULL, NULL disarms. Lets a caller time the
+ * dominant kernel alone with cudaEventElapsedTime.
+ */
+la_status la_set_kernel_timer(void* start_event, void* stop_event);
+
+/* Static, human-readable name of a status code. */
+const char* la_status_string(la_status s);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_ATTENTION_H */

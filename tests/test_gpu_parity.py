@@ -1,0 +1,228 @@
+"""GPU parity: every entry point through the C ABI against the fp64 oracle.
+
+Tolerances (bound on the whole output, relative to its largest magnitude):
+  bf16 inputs, fp32 accumulation:  max|O - O_ref| <= 1e-2 * max|O_ref|
+  fp32 inputs:                     max|O - O_ref| <= 1e-4 * max|O_ref|
+Integer-valued inputs are exact in every intermediate, so there the bf16
+output must equal the oracle result rounded to bf16, bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import causal_linear_attention_02_b200 as la
+import oracle
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+TOL = {torch.bfloat16: 1e-2, torch.float32: 1e-4}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    from causal_linear_attention_02_b200 import build
+    build.build()
+    la.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.set_device(DEV)
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy() if t.dtype == torch.bfloat16 else \
+        t.detach().cpu().double().numpy()
+
+
+def rel_err(out, ref):
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.abs(out - ref).max(initial=0.0) / max(np.abs(ref).max(initial=0.0), 1e-30))
+
+
+def assert_close(out, ref, tol, what=""):
+    r = rel_err(out, ref)
+    assert r <= tol, f"{what}: max|O-O_ref|/max|O_ref| = {r:.3e} > {tol:.0e}"
+    return r
+
+
+def inputs(T, H, d, dtype, seed):
+    return wl.qkv(T, H, d, dtype, seed, device=DEV)
+
+
+def status_ok():
+    s = la.device_status()
+    assert s == 0, f"device status {la.STATUS.get(s, s)}"
+
+
+def cu_of(lengths):
+    return wl.cu_seqlens(lengths, device=DEV)
+
+
+# ------------------------------------------------------------------ decode
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize("d", [16, 48, 64, 128])
+def test_decode_steps(dtype, d):
+    batch, H, steps = 5, 3, 3
+    st = wl.state_init(batch, H, d, seed=d, device=DEV)
+    ref_state = st.cpu().double().numpy()
+    q, k, v = wl.decode_inputs(batch, H, d, steps, dtype, seed=7 + d, device=DEV)
+    for t in range(steps):
+        o = la.decode_step(q[t], k[t], v[t], st)
+        ref_o, ref_state = oracle.decode_step(f64(q[t]), f64(k[t]), f64(v[t]), ref_state)
+        assert_close(f64(o), ref_o, TOL[dtype], f"decode o step {t}")
+    assert_close(st.cpu().double().numpy(), ref_state, 1e-5, "decode state")
+    status_ok()
+
+
+# ------------------------------------------------------------------ prefill, fp32 small workload
+def test_prefill_fp32_small_workload():
+    w = wl.FP32_SMALL
+    q, k, v = inputs(w.total_tokens, w.heads, w.d, torch.float32, w.seed)
+    o = la.prefill(q, k, v, B=w.B)
+    status_ok()
+    ref = oracle.quadratic(f64(q), f64(k), f64(v))
+    assert_close(f64(o), ref, 1e-4, "fp32 T=1024 H=2 d=64 B=64")
+
+
+# ------------------------------------------------------------------ prefill, tensor-core path
+@pytest.mark.parametrize("B", [128, 256])
+@pytest.mark.parametrize("T", [1, 37, 128, 255, 256, 257, 1000, 1500])
+def test_prefill_tc_random(B, T):
+    H, d = 3, 128
+    q, k, v = inputs(T, H, d, torch.bfloat16, seed=T * 7 + B)
+    o = la.prefill(q, k, v, B=B)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v))
+    assert_close(f64(o), ref, 1e-2, f"tc T={T} B={B}")
+
+
+@pytest.mark.parametrize("B,T", [(256, 512), (128, 384), (256, 300), (128, 200)])
+def test_prefill_tc_integer_exact(B, T):
+    """{-1,0,1} inputs: scores, P, every prefix entry and O are exact integers in
+    bf16/fp32, so the result must equal the oracle's rounded to bf16 bit for bit."""
+    H, d = 2, 128
+    q, k, v = wl.integer_qkv(T, H, d, torch.bfloat16, seed=B + T, device=DEV)
+    for n in range(B, T, B):   # every prefix state the inter-block product uses
+        assert np.abs(oracle.state(f64(k)[:n], f64(v)[:n])).max() <= 256, "precondition: bf16-exact prefix"
+    o = la.prefill(q, k, v, B=B)
+    status_ok()
+    ref = torch.from_numpy(oracle.recurrent(f64(q), f64(k), f64(v))).to(torch.bfloat16)
+    got = o.cpu()
+    mism = (got.view(torch.int16) != ref.view(torch.int16)).sum().item()
+    assert mism == 0, f"{mism} of {ref.numel()} outputs differ from the exact result"
+
+
+@pytest.mark.parametrize("B", [128, 256])
+def test_prefill_tc_varlen(B):
+    lengths = [1, 255, 256, 0, 257, 700, 64, 513, 128]
+    H, d = 2, 128
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, torch.bfloat16, seed=99 + B)
+    cu = cu_of(lengths)
+    o = la.prefill(q, k, v, cu, B=B)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy())
+    assert_close(f64(o), ref, 1e-2, f"tc varlen B={B}")
+
+
+@pytest.mark.parametrize("dtype,d,B", [(torch.bfloat16, 128, 256), (torch.bfloat16, 128, 128),
+                                       (torch.float32, 64, 64), (torch.bfloat16, 64, 128)])
+def test_prefill_init_state(dtype, d, B):
+    lengths = [300, 1, 520]
+    H = 2
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, dtype, seed=5 + d)
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, d, seed=3, device=DEV, scale=4.0)
+    o = la.prefill(q, k, v, cu, B=B, init_state=init)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy(), init=init.cpu().double().numpy())
+    assert_close(f64(o), ref, TOL[dtype], "prefill with carried-in state")
+
+
+# ------------------------------------------------------------------ prefill, CUDA-core path
+@pytest.mark.parametrize("dtype,d,B", [
+    (torch.float32, 64, 64), (torch.float32, 128, 256), (torch.float32, 48, 128), (torch.float32, 16, 64),
+    (torch.bfloat16, 64, 128), (torch.bfloat16, 16, 64), (torch.bfloat16, 128, 64), (torch.bfloat16, 112, 256),
+])
+def test_prefill_simt_shapes(dtype, d, B):
+    lengths = [70, 1, 0, 333, 64]
+    H = 3
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, dtype, seed=d + B)
+    cu = cu_of(lengths)
+    o = la.prefill(q, k, v, cu, B=B)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy())
+    assert_close(f64(o), ref, TOL[dtype], f"simt {dtype} d={d} B={B}")
+
+
+def test_prefill_b_independence():
+    """The result does not depend on B (up to rounding): B = 128 and 256 agree."""
+    q, k, v = inputs(1200, 2, 128, torch.bfloat16, seed=4242)
+    o1 = la.prefill(q, k, v, B=128)
+    o2 = la.prefill(q, k, v, B=256)
+    o3 = la.prefill(q, k, v, B=64)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v))
+    for o in (o1, o2, o3):
+        assert_close(f64(o), ref, 1e-2, "B independence")
+
+
+# ------------------------------------------------------------------ state and continuity
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64), (torch.bfloat16, 32)])
+def test_state_from_prefill(dtype, d):
+    lengths = [5000, 0, 1, 2049, 300]
+    H = 2
+    T = sum(lengths)
+    _, k, v = inputs(T, H, d, dtype, seed=31 + d)
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, d, seed=4, device=DEV)
+    ref = oracle.state(f64(k), f64(v), cu.cpu().numpy(), init=init.cpu().double().numpy())
+    st = la.state_from_prefill(k, v, cu, init_state=init)
+    assert_close(st.cpu().double().numpy(), ref, 1e-5, "state")
+    st2 = init.clone()
+    la.state_from_prefill(k, v, cu, init_state=st2, out=st2)      # in-place accumulate
+    status_ok()
+    assert_close(st2.cpu().double().numpy(), ref, 1e-5, "state in place")
+
+
+@pytest.mark.parametrize("B", [128, 256])
+def test_prefill_state_decode_continuity(B):
+    """Prefill of m tokens -> state -> decode steps reproduces the rows of one
+    prefill over m + n tokens (ties the three entry points together)."""
+    H, d, m, n = 4, 128, 700, 6
+    q, k, v = inputs(m + n, H, d, torch.bfloat16, seed=77)
+    full = la.prefill(q, k, v, B=B)
+    st = la.state_from_prefill(k[:m].contiguous(), v[:m].contiguous())
+    st = st.view(1, H, d, d).clone()
+    outs = []
+    for t in range(m, m + n):
+        outs.append(la.decode_step(q[t:t + 1].contiguous(), k[t:t + 1].contiguous(), v[t:t + 1].contiguous(), st))
+    status_ok()
+    dec = torch.cat(outs)
+    ref = oracle.recurrent(f64(q), f64(k), f64(v))
+    assert_close(f64(dec), ref[m:], 1e-2, "decode rows vs oracle")
+    assert_close(f64(full)[m:], ref[m:], 1e-2, "prefill rows vs oracle")
+
+
+# ------------------------------------------------------------------ edge cases
+def test_empty_input():
+    q = torch.empty((0, 2, 128), dtype=torch.bfloat16, device=DEV)
+    o = la.prefill(q, q, q.clone(), B=256)
+    assert o.shape == (0, 2, 128)
+    status_ok()
+
+
+def test_bad_seqlens_reported_on_device():
+    T, H, d = 20, 2, 64
+    q, k, v = inputs(T, H, d, torch.float32, seed=1)
+    cu = torch.tensor([0, 10, 5, 20], dtype=torch.int32, device=DEV)   # decreasing
+    o = torch.full_like(q, 7.0)
+    la.prefill(q, k, v, cu, B=64, out=o)
+    assert la.device_status() == 7
+    assert la.device_status() == 0                                    # cleared by the read
+    assert torch.all(o == 7.0), "no output rows are written when cu_seqlens is rejected"
+    cu2 = torch.tensor([0, 10, 19], dtype=torch.int32, device=DEV)    # does not end at T
+    la.prefill(q, k, v, cu2, B=64, out=o)
+    assert la.device_status() == 7
