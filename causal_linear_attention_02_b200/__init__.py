@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "LightningError", "LA_BF16", "LA_FP32", "STATUS", "library_path", "load_library",
     "la_prefill_workspace_size", "la_prefill", "la_state_workspace_size", "la_state_from_prefill",
-    "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_status_string", "la_version",
+    "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_status_string", "la_version",
     "prefill", "state_from_prefill", "decode_step", "device_status", "uses_tensor_cores",
 ]
 
@@ -77,6 +77,10 @@ def load_library():
         lib.la_get_device_status.restype = i32
         lib.la_status_string.argtypes = [i32]
         lib.la_status_string.restype = ctypes.c_char_p
+        lib.la_debug_set_trace.argtypes = [vp, sz]
+        lib.la_debug_set_trace.restype = i32
+        lib.la_debug_set_fault.argtypes = [ctypes.c_longlong, ctypes.c_uint64]
+        lib.la_debug_set_fault.restype = i32
         lib.la_set_kernel_timer.argtypes = [vp, vp]
         lib.la_set_kernel_timer.restype = i32
         lib.la_version.argtypes = []
@@ -116,6 +120,14 @@ def la_get_device_status(stream) -> int:
 
 def la_status_string(status: int) -> str:
     return load_library().la_status_string(int(status)).decode()
+
+
+def la_debug_set_fault(suppress_tile: int, wait_ns: int) -> int:
+    return int(load_library().la_debug_set_fault(suppress_tile, wait_ns))
+
+
+def la_debug_set_trace(device_buffer, nbytes: int) -> int:
+    return int(load_library().la_debug_set_trace(device_buffer, nbytes))
 
 
 def la_set_kernel_timer(start_event, stop_event) -> int:

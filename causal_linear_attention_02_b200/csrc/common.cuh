@@ -24,18 +24,26 @@ __device__ __forceinline__ void record_status(int code) {
 // sequence start; the last block of a sequence may be short). Built on the
 // device from cu_seqlens by build_block_table_kernel.
 struct BlockEntry {
-    int32_t seq;   // sequence index
-    int32_t blk;   // block index within the sequence
-    int32_t tok0;  // first token (global row in the packed [T][H][d] tensors)
-    int32_t len;   // tokens in this block (1..B)
+    int32_t seq;    // sequence index
+    int32_t blk;    // block index within the sequence
+    int32_t tok0;   // first token (global row in the packed [T][H][d] tensors)
+    int32_t len;    // tokens in this block (1..B)
+    int32_t last;   // 1 for the last block of its sequence (its state is never needed)
+    int32_t slot0;  // first published-state slot of this sequence (single-pass prefill)
+    int32_t pad[2];
 };
+static_assert(sizeof(BlockEntry) == 32, "block table entries are 32 bytes");
+
+// Published-state ring slots per (sequence, head) of the single-pass prefill.
+constexpr int kStateSlots = 4;
 
 // Small control area at the start of every prefill / state workspace.
 struct Control {
     int32_t nblocks;     // number of valid BlockEntry rows
     int32_t ok;          // 1 when cu_seqlens passed the device-side checks
-    int32_t ticket;      // work counter for persistent kernels
-    int32_t pad[61];
+    int32_t nslots;      // published-state slots used (single-pass prefill)
+    int32_t abort;       // set by any CTA of the single-pass prefill whose bounded wait expired
+    int32_t pad[60];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 

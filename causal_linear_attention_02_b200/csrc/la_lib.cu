@@ -5,6 +5,7 @@
 // status word is a single __device__ symbol.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <mutex>
 #include <stdint.h>
 #include <string.h>
@@ -14,7 +15,7 @@
 #include "prep.cuh"
 #include "simt.cuh"
 #include "decode.cuh"
-#include "tc.cuh"
+#include "fused.cuh"
 
 namespace {
 
@@ -40,31 +41,46 @@ bool use_tensor_cores(la_dtype dt, int d, int B) { return dt == LA_BF16 && d == 
 
 // ------------------------------------------------------------------ workspace layouts
 struct Layout {
-    int64_t max_blocks = 0;
-    size_t off_seq_blk = 0, off_table = 0, off_U = 0, off_prefix = 0, total = 0;
+    int64_t max_blocks = 0, max_slots = 0;
+    size_t off_seq_blk = 0, off_seq_slot = 0, off_table = 0, off_flags = 0, off_U = 0, off_prefix = 0,
+           off_states = 0, total = 0;
+    int nflag_arrays = 0;
 };
+
+// Control | seq_blk | seq_slot | block table, shared by every layout.
+size_t layout_head(Layout& L, int64_t T, int nseq, int B) {
+    L.max_blocks = (T + B - 1) / B + nseq;
+    size_t off = sizeof(Control);
+    L.off_seq_blk = off;  off = align_up(off + sizeof(int32_t) * (size_t)(nseq + 1), 256);
+    L.off_seq_slot = off; off = align_up(off + sizeof(int32_t) * (size_t)(nseq + 1), 256);
+    L.off_table = off;    off = align_up(off + sizeof(BlockEntry) * (size_t)L.max_blocks, 256);
+    return off;
+}
 
 Layout prefill_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt) {
     Layout L;
-    L.max_blocks = (T + B - 1) / B + nseq;
-    size_t off = sizeof(Control);
-    L.off_seq_blk = off; off = align_up(off + sizeof(int32_t) * (size_t)(nseq + 1), 256);
-    L.off_table = off;   off = align_up(off + sizeof(BlockEntry) * (size_t)L.max_blocks, 256);
+    size_t off = layout_head(L, T, nseq, B);
     const size_t dd = (size_t)d * d;
-    L.off_U = off;       off = align_up(off + 4 * dd * (size_t)H * (size_t)L.max_blocks, 256);
-    const size_t pre_es = use_tensor_cores(dt, d, B) ? 2 : 4;
-    L.off_prefix = off;  off = align_up(off + pre_es * dd * (size_t)H * (size_t)L.max_blocks, 256);
+    if (use_tensor_cores(dt, d, B)) {
+        // single pass: per-block flags (aggregate, inclusive, look-back done) and a
+        // ring of kStateSlots published states per (sequence, head); a sequence with
+        // n blocks uses min(n - 1, kStateSlots) slots.
+        L.nflag_arrays = 3;
+        L.off_flags = off;  off = align_up(off + sizeof(int32_t) * 3 * (size_t)L.max_blocks * H, 256);
+        L.max_slots = std::min<int64_t>((int64_t)nseq * la::kStateSlots, (T + B - 1) / B);
+        L.off_states = off; off = align_up(off + 2 * 4 * dd * (size_t)H * (size_t)L.max_slots, 256);
+    } else {
+        L.off_U = off;      off = align_up(off + 4 * dd * (size_t)H * (size_t)L.max_blocks, 256);
+        L.off_prefix = off; off = align_up(off + 4 * dd * (size_t)H * (size_t)L.max_blocks, 256);
+    }
     L.total = off;
     return L;
 }
 
 Layout state_layout(int64_t T, int nseq, int H, int d) {
     Layout L;
-    L.max_blocks = (T + kStateBlock - 1) / kStateBlock + nseq;
-    size_t off = sizeof(Control);
-    L.off_seq_blk = off; off = align_up(off + sizeof(int32_t) * (size_t)(nseq + 1), 256);
-    L.off_table = off;   off = align_up(off + sizeof(BlockEntry) * (size_t)L.max_blocks, 256);
-    L.off_U = off;       off = align_up(off + 4 * (size_t)d * d * (size_t)H * (size_t)L.max_blocks, 256);
+    size_t off = layout_head(L, T, nseq, kStateBlock);
+    L.off_U = off; off = align_up(off + 4 * (size_t)d * d * (size_t)H * (size_t)L.max_blocks, 256);
     L.total = off;
     return L;
 }
@@ -100,19 +116,6 @@ bool map_tokens(CUtensorMap* m, const void* base, int64_t T, int H, int d, int r
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [rows][d] viewed as 2D {d, rows}; box {64, 128}, 128-byte swizzle.
-bool map_matrix(CUtensorMap* m, const void* base, int64_t rows, int d) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64, 128};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int num_sms() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -121,6 +124,13 @@ int num_sms() {
 }
 
 la_status cuda_check() { return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+// Test hook (la_debug_set_fault): a tile that publishes nothing and a shorter wait limit.
+thread_local long long t_suppress_tile = -1;
+thread_local uint64_t t_wait_ns = 0;
+// Debug trace buffer for the single-pass prefill (la_debug_set_trace).
+thread_local uint64_t* t_trace = nullptr;
+thread_local size_t t_trace_bytes = 0;
 
 // One-shot per-thread timer around the main kernel of the next call (la_set_kernel_timer).
 thread_local cudaEvent_t t_timer_start = nullptr, t_timer_stop = nullptr;
@@ -138,14 +148,17 @@ struct MainKernelTimer {
 };
 
 // ------------------------------------------------------------------ launch helpers
-la_status launch_block_table(const int32_t* cu, int nseq, int64_t T, int B, const Layout& L, uint8_t* ws,
+la_status launch_block_table(const int32_t* cu, int nseq, int64_t T, int B, int H, const Layout& L, uint8_t* ws,
                              cudaStream_t st) {
     Control* ctrl = reinterpret_cast<Control*>(ws);
     int32_t* seq_blk = reinterpret_cast<int32_t*>(ws + L.off_seq_blk);
+    int32_t* seq_slot = reinterpret_cast<int32_t*>(ws + L.off_seq_slot);
     BlockEntry* table = reinterpret_cast<BlockEntry*>(ws + L.off_table);
-    la::seq_blocks_kernel<<<1, 1024, 0, st>>>(cu, nseq, T, B, seq_blk, ctrl);
+    int32_t* flags = L.nflag_arrays ? reinterpret_cast<int32_t*>(ws + L.off_flags) : nullptr;
+    la::seq_blocks_kernel<<<1, 1024, 0, st>>>(cu, nseq, T, B, seq_blk, seq_slot, ctrl);
     const int64_t nb = (L.max_blocks + 255) / 256;
-    la::fill_block_table_kernel<<<(unsigned)nb, 256, 0, st>>>(cu, nseq, T, B, seq_blk, ctrl, table, L.max_blocks);
+    la::fill_block_table_kernel<<<(unsigned)nb, 256, 0, st>>>(cu, nseq, T, B, seq_blk, seq_slot, ctrl, table,
+                                                              L.max_blocks, flags, L.nflag_arrays, H);
     return cuda_check();
 }
 
@@ -284,39 +297,38 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     float* U = reinterpret_cast<float*>(ws + L.off_U);
     const int dd = d * d;
 
-    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, B, L, ws, st)) != LA_OK) return s;
+    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, B, heads, L, ws, st)) != LA_OK) return s;
 
     if (use_tensor_cores(dtype, d, B)) {
-        CUtensorMap tq, tk, tv, tp;
-        __nv_bfloat16* prefix = reinterpret_cast<__nv_bfloat16*>(ws + L.off_prefix);
+        CUtensorMap tq, tk, tv;
         if (!map_tokens(&tq, q, total_tokens, heads, d, 128) || !map_tokens(&tk, k, total_tokens, heads, d, 64) ||
-            !map_tokens(&tv, v, total_tokens, heads, d, 64) ||
-            !map_matrix(&tp, prefix, L.max_blocks * heads * (int64_t)d, d))
+            !map_tokens(&tv, v, total_tokens, heads, d, 64))
             return LA_ERR_CUDA;
-        // 1) block states U_b = K_b^T V_b on the tensor cores
-        const size_t smem_state = (size_t)2 * B * d * 2 + 1024 + 256;
-        if (cudaFuncSetAttribute(la::tc::block_state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)la::tc::SMEM_STATE_MAX) != cudaSuccess)
+        la::fused::Params prm;
+        prm.out = static_cast<__nv_bfloat16*>(o);
+        prm.table = table;
+        prm.ctrl = ctrl;
+        int32_t* flags = reinterpret_cast<int32_t*>(ws + L.off_flags);
+        prm.agg_flag = flags;
+        prm.incl_flag = flags + L.max_blocks * heads;
+        prm.lb_done = flags + 2 * L.max_blocks * heads;
+        prm.states = reinterpret_cast<float*>(ws + L.off_states);
+        prm.init = init_state;
+        prm.H = heads;
+        prm.R = B / 128;
+        prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
+        prm.suppress_tile = t_suppress_tile;
+        const size_t trace_need = (size_t)L.max_blocks * heads * la::fused::kTraceEvents * sizeof(uint64_t);
+        prm.trace = (t_trace && t_trace_bytes >= trace_need) ? t_trace : nullptr;
+        if (cudaFuncSetAttribute(la::fused::prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)la::fused::SMEM_BYTES) != cudaSuccess)
             return LA_ERR_CUDA;
-        la::tc::block_state_tc_kernel<<<(unsigned)(L.max_blocks * heads), 128, smem_state, st>>>(
-            tk, tv, U, table, ctrl, heads, B, kWaitNs);
-        if ((s = cuda_check()) != LA_OK) return s;
-        // 2) exclusive prefix over the blocks of every (sequence, head), rounded to bf16
-        dim3 sg((dd + 1023) / 1024, num_seqs * heads);
-        la::chain_scan_kernel<__nv_bfloat16><<<sg, 256, 0, st>>>(U, prefix, init_state, nullptr, seq_blk, ctrl,
-                                                                 num_seqs, heads, dd, true);
-        if ((s = cuda_check()) != LA_OK) return s;
-        // 3) intra-block left product + inter-block right product, fused in TMEM
-        if (cudaFuncSetAttribute(la::tc::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)la::tc::SMEM_PREFILL) != cudaSuccess)
-            return LA_ERR_CUDA;
-        const int64_t units = L.max_blocks * (B / 128) * heads;
+        const int64_t tiles = L.max_blocks * heads;
         const int sms = num_sms();
         if (sms <= 0) return LA_ERR_CUDA;
-        const unsigned grid = (unsigned)(units < sms ? units : sms);
+        const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
         MainKernelTimer timer(st);
-        la::tc::prefill_tc_kernel<<<grid, 192, la::tc::SMEM_PREFILL, st>>>(
-            tq, tk, tv, tp, static_cast<__nv_bfloat16*>(o), table, ctrl, heads, B / 128, kWaitNs);
+        la::fused::prefill_fused_kernel<<<grid, la::fused::NTHREADS, la::fused::SMEM_BYTES, st>>>(tq, tk, tv, prm);
         return cuda_check();
     }
 
@@ -347,7 +359,7 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
     if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, kStateBlock, L, ws, st)) != LA_OK) return s;
+    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, kStateBlock, heads, L, ws, st)) != LA_OK) return s;
     if (total_tokens > 0 && (s = simt_states_d(d, dtype, k, v, heads, L, ws, st)) != LA_OK) return s;
     const int dd = d * d;
     dim3 sg((dd + 1023) / 1024, num_seqs * heads);
@@ -385,6 +397,21 @@ la_status la_get_device_status(void* stream) {
     if (cudaMemcpyFromSymbol(&v, la::g_status, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
     if (cudaMemcpyToSymbol(la::g_status, &zero, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
     return static_cast<la_status>(v);
+}
+
+la_status la_debug_set_fault(long long suppress_tile, uint64_t wait_ns) {
+    if (suppress_tile < -1) return LA_ERR_INVALID_ARGUMENT;
+    t_suppress_tile = suppress_tile;
+    t_wait_ns = wait_ns;
+    return LA_OK;
+}
+
+la_status la_debug_set_trace(void* device_buffer, size_t bytes) {
+    if ((device_buffer == nullptr) != (bytes == 0)) return LA_ERR_INVALID_ARGUMENT;
+    if (device_buffer && !aligned(device_buffer, 8)) return LA_ERR_MISALIGNED;
+    t_trace = static_cast<uint64_t*>(device_buffer);
+    t_trace_bytes = bytes;
+    return LA_OK;
 }
 
 la_status la_set_kernel_timer(void* start_event, void* stop_event) {

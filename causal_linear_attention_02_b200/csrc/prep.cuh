@@ -11,23 +11,52 @@
 
 namespace la {
 
-// Validates cu_seqlens and writes per-sequence block offsets:
-//   seq_blk[s] = sum_{s' < s} ceil(len_s' / B),  seq_blk[nseq] = total blocks.
-// One CTA of 1024 threads. cu == nullptr means one sequence of T tokens.
+// Block-wide exclusive scan over a 1024-thread CTA; returns the exclusive
+// prefix of `x` and adds the CTA total to `carry` (shared, read by all).
+__device__ __forceinline__ int32_t cta_exclusive_scan(int32_t x, int32_t* warp_sums, int32_t* carry) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int32_t incl = x;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int32_t w = lane < nw ? warp_sums[lane] : 0;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_sums[lane] = w;
+    }
+    __syncthreads();
+    const int32_t excl = *carry + (wid > 0 ? warp_sums[wid - 1] : 0) + incl - x;
+    __syncthreads();
+    if (threadIdx.x == 0) *carry += warp_sums[nw - 1];
+    __syncthreads();
+    return excl;
+}
+
+// Validates cu_seqlens and writes, per sequence s,
+//   seq_blk[s]  = sum_{s' < s} ceil(len_s' / B)            (first global block)
+//   seq_slot[s] = sum_{s' < s} min(nblocks_s' - 1, W)      (first published-state slot)
+// and the totals at index nseq. One CTA of 1024 threads. cu == nullptr means
+// one sequence of T tokens.
 __global__ void __launch_bounds__(1024) seq_blocks_kernel(const int32_t* __restrict__ cu, int nseq,
                                                           int64_t T, int B, int32_t* __restrict__ seq_blk,
+                                                          int32_t* __restrict__ seq_slot,
                                                           Control* __restrict__ ctrl) {
     __shared__ int32_t warp_sums[32];
-    __shared__ int32_t carry;
+    __shared__ int32_t carry_b, carry_s;
     __shared__ int bad;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    if (tid == 0) { carry = 0; bad = 0; }
+    const int tid = threadIdx.x;
+    if (tid == 0) { carry_b = 0; carry_s = 0; bad = 0; }
     __syncthreads();
     // validation: cu[0] = 0, non-decreasing, cu[nseq] = T
     if (cu != nullptr) {
-        for (int s = tid; s < nseq; s += blockDim.x) {
+        for (int s = tid; s < nseq; s += blockDim.x)
             if (cu[s + 1] < cu[s]) bad = 1;
-        }
         if (tid == 0 && (cu[0] != 0 || (int64_t)cu[nseq] != T)) bad = 1;
     }
     __syncthreads();
@@ -35,7 +64,8 @@ __global__ void __launch_bounds__(1024) seq_blocks_kernel(const int32_t* __restr
         if (tid == 0) {
             ctrl->nblocks = 0;
             ctrl->ok = 0;
-            ctrl->ticket = 0;
+            ctrl->nslots = 0;
+            ctrl->abort = 0;
             record_status(LA_ERR_BAD_SEQLENS);
         }
         return;
@@ -47,43 +77,33 @@ __global__ void __launch_bounds__(1024) seq_blocks_kernel(const int32_t* __restr
             const int64_t len = cu ? (int64_t)(cu[s + 1] - cu[s]) : T;
             nb = (int32_t)((len + B - 1) / B);
         }
-        // block-wide exclusive scan of nb
-        int32_t x = nb;
-        for (int o = 1; o < 32; o <<= 1) {
-            int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+        const int32_t ns = nb > 1 ? min(nb - 1, kStateSlots) : 0;
+        const int32_t eb = cta_exclusive_scan(nb, warp_sums, &carry_b);
+        const int32_t es = cta_exclusive_scan(ns, warp_sums, &carry_s);
+        if (s < nseq) {
+            seq_blk[s] = eb;
+            seq_slot[s] = es;
         }
-        if (lane == 31) warp_sums[wid] = x;
-        __syncthreads();
-        if (wid == 0) {
-            int32_t w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
-            for (int o = 1; o < 32; o <<= 1) {
-                int32_t y = __shfl_up_sync(0xffffffffu, w, o);
-                if (lane >= o) w += y;
-            }
-            warp_sums[lane] = w;   // inclusive over warps
-        }
-        __syncthreads();
-        const int32_t excl = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + x - nb;
-        if (s < nseq) seq_blk[s] = excl;
-        __syncthreads();
-        if (tid == 0) carry += warp_sums[(blockDim.x >> 5) - 1];
-        __syncthreads();
     }
     if (tid == 0) {
-        seq_blk[nseq] = carry;
-        ctrl->nblocks = carry;
+        seq_blk[nseq] = carry_b;
+        seq_slot[nseq] = carry_s;
+        ctrl->nblocks = carry_b;
         ctrl->ok = 1;
-        ctrl->ticket = 0;
+        ctrl->nslots = carry_s;
+        ctrl->abort = 0;
     }
 }
 
 // One thread per possible block: finds its sequence by binary search over
-// seq_blk and writes the BlockEntry.
+// seq_blk, writes the BlockEntry and clears the block's `nflags` per-head
+// flag words (flags: [nflag_arrays][max_blocks][H] int32, may be null).
 __global__ void fill_block_table_kernel(const int32_t* __restrict__ cu, int nseq, int64_t T, int B,
                                         const int32_t* __restrict__ seq_blk,
+                                        const int32_t* __restrict__ seq_slot,
                                         const Control* __restrict__ ctrl,
-                                        BlockEntry* __restrict__ table, int64_t max_blocks) {
+                                        BlockEntry* __restrict__ table, int64_t max_blocks,
+                                        int32_t* __restrict__ flags, int nflag_arrays, int H) {
     const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= max_blocks || g >= ctrl->nblocks) return;
     int lo = 0, hi = nseq - 1;          // last s with seq_blk[s] <= g
@@ -101,7 +121,12 @@ __global__ void fill_block_table_kernel(const int32_t* __restrict__ cu, int nseq
     e.tok0 = (int32_t)(start + (int64_t)b * B);
     const int64_t rest = len - (int64_t)b * B;
     e.len = (int32_t)(rest < B ? rest : B);
+    e.last = (g + 1 == seq_blk[s + 1]) ? 1 : 0;
+    e.slot0 = seq_slot ? seq_slot[s] : 0;
+    e.pad[0] = e.pad[1] = 0;
     table[g] = e;
+    for (int a = 0; a < nflag_arrays; ++a)
+        for (int h = 0; h < H; ++h) flags[((int64_t)a * max_blocks + g) * H + h] = 0;
 }
 
 // Exclusive prefix over the blocks of every (sequence, head) chain:

@@ -138,6 +138,31 @@ la_status la_get_device_status(void* stream);
  */
 la_status la_set_kernel_timer(void* start_event, void* stop_event);
 
+/*
+ * Test hook (no counterpart on the pages). For the following la_prefill calls
+ * made by this host thread on the tensor-core path: tile `suppress_tile` (index
+ * block * heads + head over the blocks of all sequences, -1 = none) publishes
+ * no state, and every device-side wait gives up after `wait_ns` nanoseconds
+ * (0 = the default of 4 s). A suppressed tile makes its successors' bounded
+ * waits expire: the launch then ends by itself, la_get_device_status reports
+ * LA_ERR_TIMEOUT and the CUDA context stays usable. Call with (-1, 0) to reset.
+ */
+la_status la_debug_set_fault(long long suppress_tile, uint64_t wait_ns);
+
+/*
+ * Tracing (no counterpart on the pages). While a buffer is set, every
+ * la_prefill call made by this host thread on the tensor-core path records,
+ * for each tile (block * heads + head over the blocks of all sequences), 16
+ * uint64 globaltimer stamps (ns) of its phases into `device_buffer`: [0] first
+ * Q tile ready, [1] chunk MMAs issued, [2] prefix available, [3]/[4] look-back
+ * start/end, [5] prefix written, [6] inclusive state published, [7] output
+ * stored, [8] aggregate published, [9] last P written; unused slots are left
+ * as they were. The buffer must hold max_tiles * 128 bytes, max_tiles =
+ * (ceil(total_tokens / B) + num_seqs) * heads, or the call records nothing.
+ * NULL, 0 stops tracing.
+ */
+la_status la_debug_set_trace(void* device_buffer, size_t bytes);
+
 /* Static, human-readable name of a status code. */
 const char* la_status_string(la_status s);
 

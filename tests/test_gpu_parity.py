@@ -6,6 +6,8 @@ Tolerances (bound on the whole output, relative to its largest magnitude):
 Integer-valued inputs are exact in every intermediate, so there the bf16
 output must equal the oracle result rounded to bf16, bit for bit.
 """
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -226,3 +228,56 @@ def test_bad_seqlens_reported_on_device():
     cu2 = torch.tensor([0, 10, 19], dtype=torch.int32, device=DEV)    # does not end at T
     la.prefill(q, k, v, cu2, B=64, out=o)
     assert la.device_status() == 7
+
+
+# ------------------------------------------------------------------ single-pass scheduling corners
+@pytest.mark.parametrize("T,H,B", [
+    (8192, 2, 256),      # 32 blocks per chain, few tiles: look-backs run deep and wait for inclusives
+    (65536, 1, 256),     # one chain longer than the grid: predecessors on every other CTA
+    (4096, 148, 128),    # one tile per SM per block: a tile's predecessor runs on its own CTA
+    (20001, 7, 128),     # ragged tail, odd head count
+    (3000, 64, 256),     # the 64-head shape, short
+])
+def test_prefill_single_pass_chains(T, H, B):
+    q, k, v = inputs(T, H, 128, torch.bfloat16, seed=T + H + B)
+    o = la.prefill(q, k, v, B=B)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v))
+    assert_close(f64(o), ref, 1e-2, f"single pass T={T} H={H} B={B}")
+
+
+def test_prefill_many_sequences_share_slots():
+    """Many packed sequences (some shorter than one block, some spanning many
+    slot-ring generations) in one launch."""
+    lengths = wl.varlen_lengths(40, 1, 3000, seed=8)
+    H = 3
+    T = sum(lengths)
+    q, k, v = inputs(T, H, 128, torch.bfloat16, seed=88)
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, 128, seed=9, device=DEV)
+    o = la.prefill(q, k, v, cu, B=256, init_state=init)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy(), init=init.cpu().double().numpy())
+    assert_close(f64(o), ref, 1e-2, "40 packed sequences")
+
+
+def test_lost_publication_ends_in_timeout_not_hang():
+    """A tile that never publishes its state makes its successors' bounded
+    waits expire: the launch ends by itself, the status word says TIMEOUT and
+    the context stays usable for a correct run right after."""
+    T, H, B = 4096, 4, 256
+    q, k, v = inputs(T, H, 128, torch.bfloat16, seed=5150)
+    suppress = 5 * H + 1                      # block 5 of head 1
+    assert la.la_debug_set_fault(suppress, 200_000_000) == 0
+    try:
+        t0 = time.time()
+        la.prefill(q, k, v, B=B)
+        st = la.device_status()
+        elapsed = time.time() - t0
+    finally:
+        la.la_debug_set_fault(-1, 0)
+    assert st == 6, f"expected LA_ERR_TIMEOUT, got {la.STATUS.get(st, st)}"
+    assert elapsed < 30, f"timed-out launch took {elapsed:.1f}s"
+    o = la.prefill(q, k, v, B=B)
+    status_ok()
+    assert_close(f64(o), oracle.recurrent(f64(q), f64(k), f64(v)), 1e-2, "run after a timeout")
