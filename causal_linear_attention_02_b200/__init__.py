@@ -22,7 +22,8 @@ import torch
 
 __all__ = [
     "LightningError", "LA_BF16", "LA_FP32", "STATUS", "library_path", "load_library",
-    "la_prefill_workspace_size", "la_prefill", "la_state_workspace_size", "la_state_from_prefill",
+    "la_prefill_workspace_size", "la_prefill", "la_prefill_noalloc", "LA_NOALLOC_SCRATCH_BYTES",
+    "la_state_workspace_size", "la_state_from_prefill",
     "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_status_string", "la_version",
     "prefill", "state_from_prefill", "decode_step", "device_status", "uses_tensor_cores",
 ]
@@ -67,6 +68,8 @@ def load_library():
         lib.la_prefill_workspace_size.restype = sz
         lib.la_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp, sz, vp]
         lib.la_prefill.restype = i32
+        lib.la_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp]
+        lib.la_prefill_noalloc.restype = i32
         lib.la_state_workspace_size.argtypes = [i64, i32, i32, i32, i32]
         lib.la_state_workspace_size.restype = sz
         lib.la_state_from_prefill.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, sz, vp]
@@ -98,6 +101,16 @@ def la_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtyp
                workspace, workspace_bytes, stream) -> int:
     return int(load_library().la_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype,
                                          init_state, workspace, workspace_bytes, stream))
+
+
+# Size of the static scratch of la_prefill_noalloc (LA_NOALLOC_SCRATCH_BYTES).
+LA_NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def la_prefill_noalloc(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state,
+                       stream) -> int:
+    return int(load_library().la_prefill_noalloc(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B,
+                                                 dtype, init_state, stream))
 
 
 def la_state_workspace_size(total_tokens, num_seqs, heads, d, dtype) -> int:

@@ -2,8 +2,9 @@
 
     python -m causal_linear_attention_02_b200.build [--force]
 
-nvcc compiles the single translation unit ``csrc/la_lib.cu`` (which pulls in
-every kernel header) into a shared library next to this file. The CUDA
+nvcc compiles ``csrc/la_lib.cu`` (the C ABI, which pulls in every kernel
+header) and ``csrc/la_noalloc.cu`` (the workspace-free prefill entry point)
+into a shared library next to this file. The CUDA
 runtime is linked statically; the driver entry point for TMA descriptors is
 looked up at run time, so no libcuda stub is needed at link time.
 """
@@ -46,7 +47,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "la_lib.cu"), "-o", tmp]
+           os.path.join(CSRC, "la_lib.cu"), os.path.join(CSRC, "la_noalloc.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)

@@ -91,6 +91,26 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o,
                      const float* init_state, void* workspace, size_t workspace_bytes,
                      void* stream);
 
+/*
+ * la_prefill without a workspace argument (no counterpart on the pages), for
+ * callers that cannot allocate device memory: allocator-free runtimes, fixed
+ * memory budgets, hooks that run inside another library's memory manager. Its
+ * scratch is one static device array of LA_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading the library holds until the process exits. Arguments and
+ * results are those of la_prefill. Problems whose la_prefill_workspace_size
+ * exceeds LA_NOALLOC_SCRATCH_BYTES are rejected with
+ * LA_ERR_WORKSPACE_TOO_SMALL before anything is enqueued. It allocates
+ * nothing: the first call on each device (with that device current) looks up
+ * the array's device address once, so make that first call before any stream
+ * capture. All calls on a device share the array; calls that overlap on the
+ * GPU race and give undefined results.
+ */
+#define LA_NOALLOC_SCRATCH_BYTES (64u << 20)
+la_status la_prefill_noalloc(const void* q, const void* k, const void* v, void* o,
+                             const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens,
+                             int heads, int d, int B, la_dtype dtype,
+                             const float* init_state, void* stream);
+
 /* Bytes of device workspace la_state_from_prefill needs (0 if unsupported). */
 size_t la_state_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, la_dtype dtype);
 
