@@ -35,7 +35,7 @@ struct BlockEntry {
 static_assert(sizeof(BlockEntry) == 32, "block table entries are 32 bytes");
 
 // Published-state ring slots per (sequence, head) of the single-pass prefill.
-constexpr int kStateSlots = 4;
+constexpr int kStateSlots = 6;
 
 // Small control area at the start of every prefill / state workspace.
 struct Control {

@@ -16,16 +16,16 @@
 // round-robin (t = blockIdx.x, blockIdx.x + gridDim.x, ...). A tile is B
 // query rows processed as R = B/128 sub-units of 128 rows, last sub-unit
 // first (it streams every key chunk of the block and so computes U_b on the
-// way). Roles (320 threads):
-//   warp 0     TMA producer: Q sub-unit tiles and 64-token K/V chunks
-//   warp 1     tcgen05 issuer: S = Q K^T, O += P V, U += K^T V, O += Q prefix
-//   warps 2-5  scores -> P (mask, bf16, written back into TMEM); publish U_b
-//   warps 6-9  look-back -> bf16 prefix in shared memory; store the inclusive
-//              prefix; O epilogue (TMEM -> bf16 -> global)
-//   warp 10    publisher: one lane per flag kind makes the stored states visible
-//              (gpu-scope fence after the group's mbarrier arrive) and raises
-//              the flags, so no worker group stalls on a memory fence
-//   warp 11    idle (keeps three warps per sub-partition for the register budget)
+// way). Roles (512 threads, 128 registers each):
+//   warp 0       TMA producer: Q sub-unit tiles and 64-token K/V chunks
+//   warp 1       tcgen05 issuer: U += K^T V, S = Q K^T, O += P V, O += Q prefix
+//   warp 2       publisher: makes stored states visible at gpu scope and raises
+//                their flags; grants ring slots (no worker group waits on a fence)
+//   warp 3       spare
+//   warps 4-7    scores -> P (mask, bf16, written back into TMEM); store U_b
+//   warps 8-11   columns 0..63 and warps 12-15 columns 64..127 of: look-back ->
+//                bf16 prefix in shared memory; inclusive prefix = exclusive +
+//                U_b (read back from the stored aggregate); O epilogue (TMA store)
 // Published states live in a small ring of W slots per (sequence, head) so
 // they stay resident in L2; a slot is reused only after every tile that may
 // read it has finished its look-back (look-back depth is bounded by L = W - 2).
@@ -47,8 +47,8 @@ constexpr int KC = 64;                     // keys per chunk
 constexpr int NQ = 3;                      // Q sub-unit stages
 constexpr int NKV = 3;                     // K/V chunk stages
 constexpr int W = kStateSlots;             // published-state ring slots per chain
-constexpr int L = W - 2;                   // look-back depth: blocks b-1 .. b-L may be read
-static_assert(L == 2, "the look-back below reads at most incl(b-1), or agg(b-1) + incl(b-2)");
+constexpr int L = 3;                       // look-back depth: blocks b-1 .. b-L may be read
+static_assert(W >= L + 2, "slot reuse must not wait on the look-back of the block just before");
 
 constexpr uint32_t Q_BYTES = UM * D * 2;   // 32 KB
 constexpr uint32_t QH_BYTES = UM * 64 * 2; // 16 KB (one 64-column half)
@@ -70,16 +70,21 @@ constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, false, true);
 constexpr uint32_t IDESC_QP = idesc_bf16(128, 128, false, true);
 constexpr uint32_t IDESC_KV = idesc_bf16(128, 128, true, true);
 
-constexpr int NTHREADS = 384;
+constexpr int NTHREADS = 512;
 
 struct Bars {
     uint64_t q_full[NQ], q_empty[NQ];
     uint64_t kv_full[NKV], kv_empty[NKV];
     uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
     uint64_t pre_full, pre_empty, u_full, u_empty, drain;
-    uint64_t grp_a, grp_b;     // bounded 128-thread group barriers of warps 2-5 and 6-9
-    uint64_t lbd_st, agg_st, incl_st;     // worker group -> publisher: look-back reads done / state stored
-    uint64_t lbd_pub, agg_pub, incl_pub;  // publisher -> worker group: flag released
+    uint64_t grp_a;            // bounded 128-thread barrier of the P / epilogue group
+    uint64_t stage_done;       // P group -> column groups: O stores have read the staging buffer
+    uint64_t lbd_st, incl_st;             // worker group -> publisher: look-back reads done / incl stored
+    uint64_t agg_st[2];                   // P group -> publisher and column groups: aggregate stored
+                                          // (two, used alternately: the P group runs one tile ahead)
+    uint64_t lbd_pub;                     // publisher -> look-back group: previous look-back flag released
+    uint64_t incl_pub;                    // publisher -> column groups: previous inclusive flag released
+    uint64_t slot_ok;                     // publisher -> P group: this tile's ring slot may be written
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -99,6 +104,7 @@ struct Params {
     uint64_t wait_ns;
     long long suppress_tile;   // test hook: this tile publishes nothing (-1: none)
     uint64_t* trace;           // optional [tile][kTraceEvents] globaltimer stamps, or nullptr
+    uint64_t grace_ns;         // look-back: how long to wait for incl(b-1) before reading agg(b-1) + incl(b-2)
 };
 
 // Phase stamps of the optional per-tile trace (la_debug_set_trace).
@@ -119,7 +125,20 @@ enum TraceEvent {
     TR_P0 = 13,           // issuer: P of the first chunk ready
     TR_PLAST = 14,        // issuer: P of the first sub-unit's last chunk ready
     TR_LOAD0 = 15,        // producer: first load of the tile issued
-    kTraceEvents = 16
+    TR_B_INCL_ST = 16,    // column group 0: inclusive prefix stored, handed to the publisher
+    TR_B_LBD_ST = 17,     // column group 0: look-back reads done, handed to the publisher
+    TR_A_AGG_ST = 18,     // P group: aggregate stored, handed to the publisher
+    TR_PUB_INCL = 19,     // publisher: inclusive hand-off seen (before its release store)
+    TR_B_LB_DECIDED = 20, // column group 0: look-back sources decided
+    TR_A_EPI1_FULL = 21,  // P group: first epilogue sub-unit accumulator complete
+    TR_A_EPI1_FREE = 22,  // P group: first epilogue sub-unit accumulator released
+    TR_A_U_FULL = 23,     // P group: next tile's block state complete in TMEM
+    TR_A_SLOT_OK = 24,    // P group: next tile's ring slot granted
+    TR_A_EPI0_FULL = 25,  // P group: second epilogue sub-unit accumulator complete
+    TR_A_EPI0_FREE = 26,  // P group: second epilogue sub-unit accumulator released
+    TR_A_S0 = 27,         // P group: scores of the tile's first chunk seen
+    TR_PUB_AGG = 28,      // publisher: aggregate hand-off seen (before its release store)
+    kTraceEvents = 32
 };
 #define LA_TRACE(t, ev)                                                         \
     do {                                                                       \
@@ -207,6 +226,16 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
     }
 }
 
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1,
+                                             int32_t c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t c0, int32_t c1, int32_t c2) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];"
                  :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2) : "memory");
@@ -226,29 +255,10 @@ __device__ __forceinline__ bool spin_flag(const int* flag, const Abort& ab) {
     }
 }
 
-// A slot is rewritten only after every tile that may still read its previous
-// occupant (block b - W, read by the look-backs of blocks b-W+1 .. b-W+L) has
-// finished its look-back. With W = L + 2 the newest of those is two blocks
-// back, so publishing never waits on the look-back of the block just before.
-// Called by one thread; the caller shares the outcome through a group barrier.
-__device__ __forceinline__ bool wait_reclaim(const Params& p, const Tile& x, const Abort& ab) {
-    const int blk = x.e.blk;
-    for (int c = max(0, blk - W + 1); c <= blk - W + L; ++c) {
-        const int gc = x.g - (blk - c);
-        if (!spin_flag(p.lb_done + (int64_t)gc * p.H + x.h, ab)) return false;
-    }
-    return true;
-}
-// Early, non-blocking probe of the same condition (relaxed loads issued at the
-// start of a tile, consumed much later). A true result still needs an acquire
-// fence before the slot is written; a false result falls back to wait_reclaim.
-__device__ __forceinline__ bool probe_reclaim(const Params& p, const Tile& x) {
-    const int blk = x.e.blk;
-    int all = 1;
-    for (int c = max(0, blk - W + 1); c <= blk - W + L; ++c)
-        all &= ld_relaxed(p.lb_done + (int64_t)(x.g - (blk - c)) * p.H + x.h);
-    return all != 0;
-}
+// Ring-slot reuse: block b writes slot b % W, last used by block b - W, which
+// the look-backs of blocks b-W+1 .. b-W+L may read. With W = L + 2 the newest
+// of those is two blocks back, so the check (made by the publisher lane) never
+// waits on the look-back of the block just before.
 
 // Bounded barrier of one 128-thread group built on an mbarrier (arrive, then
 // wait for the phase). Unlike bar.sync it cannot hang if a member has left
@@ -262,7 +272,8 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, const
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const Params p) {
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -276,19 +287,20 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_init(&bars->s_full[i], 1);  mbar_init(&bars->p_full[i], 128);
             mbar_init(&bars->o_full[i], 1);  mbar_init(&bars->o_empty[i], 128);
         }
-        mbar_init(&bars->pre_full, 128);
+        mbar_init(&bars->pre_full, 256);
         mbar_init(&bars->pre_empty, 1);
         mbar_init(&bars->u_full, 1);
-        mbar_init(&bars->u_empty, 256);
+        mbar_init(&bars->u_empty, 128);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->grp_a, 128);
-        mbar_init(&bars->grp_b, 128);
-        mbar_init(&bars->lbd_st, 128);
-        mbar_init(&bars->agg_st, 128);
-        mbar_init(&bars->incl_st, 128);
+        mbar_init(&bars->stage_done, 1);
+        mbar_init(&bars->lbd_st, 256);
+        mbar_init(&bars->agg_st[0], 128);
+        mbar_init(&bars->agg_st[1], 128);
+        mbar_init(&bars->incl_st, 256);
         mbar_init(&bars->lbd_pub, 1);
-        mbar_init(&bars->agg_pub, 1);
         mbar_init(&bars->incl_pub, 1);
+        mbar_init(&bars->slot_ok, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -308,32 +320,55 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 
     if (warp == 0) {
         // ================================================================ TMA producer
+        // Per tile: first the whole K and V of this CTA's NEXT tile (its block state
+        // U is computed one tile ahead, see the issuer), then Q and the K/V chunks
+        // of this tile's sub-units. The lookahead load brings the next tile's K/V
+        // into L2, where its own pass finds it a tile later.
         if (lane == 0) {
             const uint64_t pol = policy_evict_first();
             uint32_t q_it = 0, kv_it = 0;
             bool ok = true;
+            auto load_chunk = [&](const Tile& y, int j, uint64_t hint) -> bool {
+                const uint32_t st = kv_it % NKV;
+                if (!wait_bar(&bars->kv_empty[st], ((kv_it / NKV) & 1) ^ 1, ab)) return false;
+                uint8_t* kd = smem + OFF_KV + st * 2 * KV_BYTES;
+                uint8_t* vd = kd + KV_BYTES;
+                const int tk = y.e.tok0 + KC * j;
+                mbar_expect_tx(&bars->kv_full[st], 2 * KV_BYTES);
+                if (hint) {
+                    tma_load_3d_hint(kd, &tmK, &bars->kv_full[st], 0, y.h, tk, hint);
+                    tma_load_3d_hint(kd + KVH_BYTES, &tmK, &bars->kv_full[st], 64, y.h, tk, hint);
+                    tma_load_3d_hint(vd, &tmV, &bars->kv_full[st], 0, y.h, tk, hint);
+                    tma_load_3d_hint(vd + KVH_BYTES, &tmV, &bars->kv_full[st], 64, y.h, tk, hint);
+                } else {
+                    tma_load_3d(kd, &tmK, &bars->kv_full[st], 0, y.h, tk);
+                    tma_load_3d(kd + KVH_BYTES, &tmK, &bars->kv_full[st], 64, y.h, tk);
+                    tma_load_3d(vd, &tmV, &bars->kv_full[st], 0, y.h, tk);
+                    tma_load_3d(vd + KVH_BYTES, &tmV, &bars->kv_full[st], 64, y.h, tk);
+                }
+                ++kv_it;
+                return true;
+            };
+            auto load_lookahead = [&](int64_t tt) -> bool {
+                if (tt >= ntiles) return true;
+                const Tile y = tile_of(tt, p);
+                if (!owns_state(y)) return true;
+                for (int j = 0; j < R * (UM / KC); ++j)
+                    if (!load_chunk(y, j, 0)) return false;
+                return true;
+            };
+            if (!load_lookahead(blockIdx.x)) ok = false;
             for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
                 const Tile x = tile_of(t, p);
-                // stage the next tile of this CTA in L2 a whole tile ahead, so that the
-                // shared-memory loads below (and the next tile's) hit L2
-                if (t + gridDim.x < ntiles) {
+                if (t + gridDim.x < ntiles) {          // the next tile's Q into L2 a tile ahead
                     const Tile y = tile_of(t + gridDim.x, p);
                     for (int r = R - 1; r >= 0; --r) {
                         if (sub_rows(y, r) <= 0) continue;
                         tma_prefetch_l2_3d(&tmQ, 0, y.h, y.e.tok0 + UM * r);
                         tma_prefetch_l2_3d(&tmQ, 64, y.h, y.e.tok0 + UM * r);
                     }
-                    int rf = R - 1;                       // first sub-unit streamed (most chunks)
-                    while (rf > 0 && sub_rows(y, rf) <= 0) --rf;
-                    const int nk = sub_chunks(y, rf);
-                    for (int j = 0; j < nk; ++j) {
-                        const int tk = y.e.tok0 + KC * j;
-                        tma_prefetch_l2_3d(&tmK, 0, y.h, tk);
-                        tma_prefetch_l2_3d(&tmK, 64, y.h, tk);
-                        tma_prefetch_l2_3d(&tmV, 0, y.h, tk);
-                        tma_prefetch_l2_3d(&tmV, 64, y.h, tk);
-                    }
                 }
+                if (!load_lookahead(t + gridDim.x)) { ok = false; break; }
                 for (int r = R - 1; ok && r >= 0; --r) {
                     if (sub_rows(x, r) <= 0) continue;
                     const uint32_t qs = q_it % NQ;
@@ -347,26 +382,9 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     ++q_it;
                     const int nkc = sub_chunks(x, r);
                     for (int j = 0; j < nkc; ++j) {
-                        const uint32_t st = kv_it % NKV;
-                        if (!wait_bar(&bars->kv_empty[st], ((kv_it / NKV) & 1) ^ 1, ab)) { ok = false; break; }
-                        uint8_t* kd = smem + OFF_KV + st * 2 * KV_BYTES;
-                        uint8_t* vd = kd + KV_BYTES;
-                        const int tk = x.e.tok0 + KC * j;
                         // chunks re-streamed by a later sub-unit of the same block stay in L2
-                        const uint64_t pk = (r == R - 1 && R > 1 && j < (R - 1) * (UM / KC)) ? 0 : pol;
-                        mbar_expect_tx(&bars->kv_full[st], 2 * KV_BYTES);
-                        if (pk) {
-                            tma_load_3d_hint(kd, &tmK, &bars->kv_full[st], 0, x.h, tk, pk);
-                            tma_load_3d_hint(kd + KVH_BYTES, &tmK, &bars->kv_full[st], 64, x.h, tk, pk);
-                            tma_load_3d_hint(vd, &tmV, &bars->kv_full[st], 0, x.h, tk, pk);
-                            tma_load_3d_hint(vd + KVH_BYTES, &tmV, &bars->kv_full[st], 64, x.h, tk, pk);
-                        } else {
-                            tma_load_3d(kd, &tmK, &bars->kv_full[st], 0, x.h, tk);
-                            tma_load_3d(kd + KVH_BYTES, &tmK, &bars->kv_full[st], 64, x.h, tk);
-                            tma_load_3d(vd, &tmV, &bars->kv_full[st], 0, x.h, tk);
-                            tma_load_3d(vd + KVH_BYTES, &tmV, &bars->kv_full[st], 64, x.h, tk);
-                        }
-                        ++kv_it;
+                        const bool again = r == R - 1 && R > 1 && j < (R - 1) * (UM / KC);
+                        if (!load_chunk(x, j, again ? 0 : pol)) { ok = false; break; }
                     }
                 }
             }
@@ -393,15 +411,37 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint32_t kv_base = smem_u32(smem + OFF_KV);
             const uint32_t pre_base = smem_u32(smem + OFF_PRE);
             bool ok = true;
+            // Block state of tile tt, one tile ahead: U = sum over its chunks of K^T V,
+            // accumulated in TMEM as the chunks land; u_full fires when it is complete.
+            auto lookahead_state = [&](int64_t tt) -> bool {
+                if (tt >= ntiles) return true;
+                const Tile y = tile_of(tt, p);
+                if (!owns_state(y)) return true;
+                if (!wait_bar(&bars->u_empty, (u_it & 1) ^ 1, ab)) return false;  // previous U drained
+                for (int j = 0; j < R * (UM / KC); ++j, ++kv_it) {
+                    const uint32_t st = kv_it % NKV;
+                    if (!wait_bar(&bars->kv_full[st], (kv_it / NKV) & 1, ab)) return false;
+                    tc_fence_after();
+                    const uint32_t kb = kv_base + st * 2 * KV_BYTES, vb = kb + KV_BYTES;
+#pragma unroll
+                    for (int s = 0; s < KC / 16; ++s)
+                        mma_ss(tmem + TM_U, sdesc_sw128(kb + s * 2048, KVH_BYTES, 1024),
+                               sdesc_sw128(vb + s * 2048, KVH_BYTES, 1024), IDESC_KV, (j > 0 || s > 0));
+                    tc_commit(&bars->kv_empty[st]);
+                }
+                tc_commit(&bars->u_full);
+                ++u_it;
+                return true;
+            };
+            if (!lookahead_state(blockIdx.x)) ok = false;
             for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
                 const Tile x = tile_of(t, p);
-                const bool own = owns_state(x);
+                if (!lookahead_state(t + gridDim.x)) { ok = false; break; }
                 uint32_t sub_q[2], sub_o[2];
                 int nsub = 0;
                 for (int r = R - 1; ok && r >= 0; --r) {
                     if (sub_rows(x, r) <= 0) continue;
                     const int nkc = sub_chunks(x, r);
-                    const bool with_u = own && r == R - 1;
                     const uint32_t qs = q_it % NQ, ob = o_it & 1;
                     if (!wait_bar(&bars->q_full[qs], (q_it / NQ) & 1, ab)) { ok = false; break; }
                     if (nsub == 0) LA_TRACE(t, TR_MMA_START);
@@ -411,7 +451,6 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     auto issue_scores = [&](int j) -> bool {
                         const uint32_t kvi = kv_it + j, st = kvi % NKV;
                         if (!wait_bar(&bars->kv_full[st], (kvi / NKV) & 1, ab)) return false;
-                        if (nsub == 0 && j == 0) LA_TRACE(t, TR_KV0);
                         tc_fence_after();
                         const uint32_t kb = kv_base + st * 2 * KV_BYTES;
                         const uint32_t d_s = tmem + TM_S + ((s_it + j) & 1) * 64;
@@ -425,7 +464,6 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (!issue_scores(0)) { ok = false; break; }
                     if (!wait_bar(&bars->o_empty[ob], ((o_it >> 1) & 1) ^ 1, ab)) { ok = false; break; }
                     LA_TRACE(t, nsub == 0 ? TR_OEMPTY_A : TR_OEMPTY_B);
-                    if (with_u && !wait_bar(&bars->u_empty, (u_it & 1) ^ 1, ab)) { ok = false; break; }
                     tc_fence_after();
                     for (int j = 0; j < nkc; ++j) {
                         if (j + 1 < nkc && !issue_scores(j + 1)) { ok = false; break; }
@@ -441,16 +479,9 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         for (int s = 0; s < KC / 16; ++s)
                             mma_ts(d_o, a_p + s * 8, sdesc_sw128(vb + s * 2048, KVH_BYTES, 1024), IDESC_PV,
                                    (j > 0 || s > 0));
-                        if (with_u) {
-#pragma unroll
-                            for (int s = 0; s < KC / 16; ++s)
-                                mma_ss(tmem + TM_U, sdesc_sw128(kb + s * 2048, KVH_BYTES, 1024),
-                                       sdesc_sw128(vb + s * 2048, KVH_BYTES, 1024), IDESC_KV, (j > 0 || s > 0));
-                        }
                         tc_commit(&bars->kv_empty[st]);
                     }
                     if (!ok) break;
-                    if (with_u) { tc_commit(&bars->u_full); ++u_it; }
                     kv_it += nkc;
                     s_it += nkc;
                     sub_q[nsub] = qs;
@@ -483,18 +514,49 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&bars->drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
         }
-    } else if (warp < 6) {
-        // ================================================================ scores -> P; publish U_b
+    } else if (warp >= 4 && warp < 8) {
+        // ================================================================ scores -> P; store U of the next tile
         const int quad = warp & 3;
         const int m = quad * 32 + lane;
         const uint32_t lane_base = uint32_t(quad * 32) << 16;
-        const int wt = threadIdx.x - 64;                  // 0..127 within this group
-        uint32_t s_it = 0, u_it = 0, grp_phase = 0;
+        const int wt = threadIdx.x - 128;                 // 0..127 within this group
+        uint32_t s_it = 0, u_it = 0, o_it = 0, tile_it = 0, grp_phase = 0;
         bool ok = true;
+        // Store the block state of tile tt (computed one tile ahead by the issuer) as
+        // the aggregate of its ring slot; the publisher raises its flag.
+        auto store_aggregate = [&](int64_t tt) -> bool {
+            if (tt >= ntiles) return true;
+            const Tile y = tile_of(tt, p);
+            if (!owns_state(y)) return true;
+            if (!warp_all(wait_bar(&bars->u_full, u_it & 1, ab))) return false;
+            if (wt == 0) LA_TRACE(tt, TR_A_U_FULL);
+            tc_fence_after();
+            if (!warp_all(wait_bar(&bars->slot_ok, u_it & 1, ab))) return false;   // ring slot is free
+            if (wt == 0) LA_TRACE(tt, TR_A_SLOT_OK);
+            if (tt != p.suppress_tile) {
+                float* dst = slot_ptr(p, y, y.e.blk, 0);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t u[16];
+                    tmem_ld_x16(tmem + lane_base + TM_U + 16 * c, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        __stcg(reinterpret_cast<float4*>(dst + ((4 * c + w) * D + m) * 4),
+                               make_float4(__uint_as_float(u[4 * w]), __uint_as_float(u[4 * w + 1]),
+                                           __uint_as_float(u[4 * w + 2]), __uint_as_float(u[4 * w + 3])));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->u_empty);
+            mbar_arrive(&bars->agg_st[u_it & 1]);
+            if (wt == 0) LA_TRACE(tt, TR_A_AGG_ST);
+            ++u_it;
+            return true;
+        };
+        if (!store_aggregate(blockIdx.x)) ok = false;
         for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
             const Tile x = tile_of(t, p);
-            const bool own = owns_state(x);
-            const bool slot_free = (own && wt == 0) ? probe_reclaim(p, x) : true;
             for (int r = R - 1; ok && r >= 0; --r) {
                 if (sub_rows(x, r) <= 0) continue;
                 const int nkc = sub_chunks(x, r);
@@ -502,26 +564,27 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 for (int j = 0; j < nkc; ++j, ++s_it) {
                     const uint32_t sb = s_it & 1;
                     if (!warp_all(wait_bar(&bars->s_full[sb], (s_it >> 1) & 1, ab))) { ok = false; break; }
+                    if (wt == 0 && r == R - 1 && j == 0) LA_TRACE(t, TR_A_S0);
                     tc_fence_after();
                     const uint32_t ts = tmem + lane_base + TM_S + sb * 64;
-                    uint32_t a[32], b[32], pk[32];
-                    tmem_ld_x32(ts, a);
-                    tmem_ld_x32(ts + 32, b);
-                    tmem_wait_ld();
                     const int lim = qi - KC * j;          // key column c is kept when c <= lim
-                    if (lim >= KC - 1) {
+                    uint32_t pk[32];
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            pk[c] = pack_bf16x2(__uint_as_float(a[2 * c]), __uint_as_float(a[2 * c + 1]));
-                            pk[16 + c] = pack_bf16x2(__uint_as_float(b[2 * c]), __uint_as_float(b[2 * c + 1]));
-                        }
-                    } else {
+                    for (int hh = 0; hh < 2; ++hh) {      // two 32-column halves keep registers low
+                        uint32_t a[32];
+                        tmem_ld_x32(ts + 32 * hh, a);
+                        tmem_wait_ld();
+                        if (lim >= KC - 1) {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            pk[c] = pack_bf16x2(2 * c <= lim ? __uint_as_float(a[2 * c]) : 0.f,
-                                                2 * c + 1 <= lim ? __uint_as_float(a[2 * c + 1]) : 0.f);
-                            pk[16 + c] = pack_bf16x2(32 + 2 * c <= lim ? __uint_as_float(b[2 * c]) : 0.f,
-                                                     33 + 2 * c <= lim ? __uint_as_float(b[2 * c + 1]) : 0.f);
+                            for (int c = 0; c < 16; ++c)
+                                pk[16 * hh + c] = pack_bf16x2(__uint_as_float(a[2 * c]), __uint_as_float(a[2 * c + 1]));
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 16; ++c) {
+                                const int c0 = 32 * hh + 2 * c;
+                                pk[16 * hh + c] = pack_bf16x2(c0 <= lim ? __uint_as_float(a[2 * c]) : 0.f,
+                                                              c0 + 1 <= lim ? __uint_as_float(a[2 * c + 1]) : 0.f);
+                            }
                         }
                     }
                     tmem_st_x32(ts, pk);
@@ -530,120 +593,161 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     mbar_arrive(&bars->p_full[sb]);
                     if (wt == 0 && r == 0 && j + 1 == nkc) LA_TRACE(t, TR_P_END);
                 }
-                if (!ok) break;
-                if (own && r == R - 1) {
-                    // store the aggregate U_b = K_b^T V_b of this (block, head); the
-                    // publisher lane raises its flag once the stores are visible
-                    if (!wait_bar(&bars->u_full, u_it & 1, ab)) ok = false;
-                    tc_fence_after();
-                    if (ok && wt == 0) {
-                        if (slot_free) fence_acq_rel_gpu();
-                        else if (!wait_reclaim(p, x, ab)) ok = false;
+            }
+            // ---- O epilogue of each sub-unit, in the order the issuer finishes them:
+            // drain the accumulator row (packed to bf16) and free it at once; full
+            // 128-row sub-units go out as TMA tensor stores staged in the prefix buffer
+            // (free once this tile's inter-block MMAs are done), a ragged last sub-unit
+            // of a sequence with masked direct stores. The next tile's block state is
+            // stored right after the first sub-unit, so the issuer can compute the one
+            // after it while the rest of this epilogue runs.
+            bool staged = false;
+            for (int r = R - 1; ok && r >= 0; --r) {
+                const int rows = sub_rows(x, r);
+                if (rows <= 0) continue;
+                const uint32_t ob = o_it & 1;
+                if (!warp_all(wait_bar(&bars->o_full[ob], (o_it >> 1) & 1, ab))) { ok = false; break; }
+                if (wt == 0) LA_TRACE(t, r == R - 1 ? TR_A_EPI1_FULL : TR_A_EPI0_FULL);
+                tc_fence_after();
+                const bool full = rows == UM;
+                uint8_t* stage = smem + OFF_PRE;
+                if (full) {
+                    if (!staged) {            // all inter-block MMAs of this tile have read the prefix
+                        if (!warp_all(wait_bar(&bars->pre_empty, tile_it & 1, ab))) { ok = false; break; }
+                        staged = true;
                     }
-                    if (!group_sync(&bars->grp_a, grp_phase, ab) || ab.raised()) ok = false;
-                    if (ok && !wait_bar(&bars->agg_pub, (u_it & 1) ^ 1, ab)) ok = false;
-                    ok = warp_all(ok);
-                    if (ok && t != p.suppress_tile) {
-                        float* dst = slot_ptr(p, x, x.e.blk, 0);
+                    if (wt == 0) bulk_wait_read0();              // the previous O store has read the buffer
+                    if (!warp_all(group_sync(&bars->grp_a, grp_phase, ab))) { ok = false; break; }
+                }
+                __nv_bfloat16* orow = p.out + ((int64_t)(x.e.tok0 + UM * r + m) * p.H + x.h) * D;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            uint32_t u[16];
-                            tmem_ld_x16(tmem + lane_base + TM_U + 16 * c, u);
-                            tmem_wait_ld();
+                for (int c4 = 0; c4 < 4; ++c4) {      // 32 columns at a time
+                    uint32_t v0[32];
+                    tmem_ld_x32(tmem + lane_base + TM_O + ob * 128 + 32 * c4, v0);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
-                            for (int w = 0; w < 4; ++w)
-                                __stcg(reinterpret_cast<float4*>(dst + ((4 * c + w) * D + m) * 4),
-                                       make_float4(__uint_as_float(u[4 * w]), __uint_as_float(u[4 * w + 1]),
-                                                   __uint_as_float(u[4 * w + 2]), __uint_as_float(u[4 * w + 3])));
-                        }
+                    for (int c = 0; c < 16; ++c)
+                        pk[c] = pack_bf16x2(__uint_as_float(v0[2 * c]), __uint_as_float(v0[2 * c + 1]));
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int g = 4 * c4 + w;     // 16-byte group of the row
+                        const uint4 val = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+                        if (full)
+                            *reinterpret_cast<uint4*>(stage + (g >> 3) * PREH_BYTES + (m >> 3) * 1024 +
+                                                      (m & 7) * 128 + (((g & 7) ^ (m & 7)) << 4)) = val;
+                        else if (m < rows)
+                            __stcs(reinterpret_cast<uint4*>(orow + 8 * g), val);
                     }
-                    tc_fence_before();
-                    mbar_arrive(&bars->u_empty);
-                    mbar_arrive(&bars->agg_st);
-                    ++u_it;
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->o_empty[ob]);               // the accumulator is free again
+                if (wt == 0) LA_TRACE(t, r == R - 1 ? TR_A_EPI1_FREE : TR_A_EPI0_FREE);
+                ++o_it;
+                if (full) {
+                    fence_proxy_async_smem();
+                    if (!warp_all(group_sync(&bars->grp_a, grp_phase, ab))) { ok = false; break; }
+                    if (wt == 0) {
+                        const int tq = x.e.tok0 + UM * r;
+                        tma_store_3d(&tmO, stage, 0, x.h, tq);
+                        tma_store_3d(&tmO, stage + PREH_BYTES, 64, x.h, tq);
+                        bulk_commit();
+                    }
+                }
+                if (r == R - 1 && ok && !store_aggregate(t + gridDim.x)) ok = false;
+            }
+            if (!ok) break;
+            if (sub_rows(x, R - 1) <= 0 && !store_aggregate(t + gridDim.x)) { ok = false; break; }
+            // the staging buffer is free for the next prefix once these stores have read it
+            if (wt == 0) {
+                bulk_wait_read0();
+                mbar_arrive(&bars->stage_done);
+            }
+            if (wt == 0) LA_TRACE(t, TR_EPI_END);
+            ++tile_it;
+        }
+        if (wt == 0) bulk_wait0();            // every O store has landed before the CTA exits
+    } else if (warp >= 8) {
+        // ================================================================ look-back, prefix, inclusive
+        // Two groups, each owning 64 of the 128 state / output columns.
+        const int hb = warp >= 12 ? 1 : 0;
+        const int kb = 16 * hb;                           // first float4 column group of this half
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;                   // state row owned by this thread
+        const int wt = threadIdx.x - (hb ? 384 : 256);
+        uint8_t* half_buf = smem + OFF_PRE + hb * PREH_BYTES;   // prefix half (O staging between tiles)
+        uint32_t tile_it = 0, u_it = 0;
+        bool ok = true;
+        auto add_row = [&](float4 (&acc)[16], const float* src) {
+#pragma unroll
+            for (int k0 = 0; k0 < 16; k0 += 8) {          // 8 loads in flight at a time
+                float4 v[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    v[k] = __ldcg(reinterpret_cast<const float4*>(src + ((kb + k0 + k) * D + m) * 4));
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    acc[k0 + k].x += v[k].x; acc[k0 + k].y += v[k].y;
+                    acc[k0 + k].z += v[k].z; acc[k0 + k].w += v[k].w;
                 }
             }
-        }
-    } else if (warp < 10) {
-        // ================================================================ look-back, prefix, inclusive, epilogue
-        const int quad = warp & 3;
-        const int m = quad * 32 + lane;                   // state row / O row owned by this thread
-        const uint32_t lane_base = uint32_t(quad * 32) << 16;
-        const int wt = threadIdx.x - 192;
-        uint32_t tile_it = 0, o_it = 0, u_it = 0, grp_phase = 0;
-        bool ok = true;
+        };
         for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
             const Tile x = tile_of(t, p);
             const bool own = owns_state(x);
-            float4 acc[32];
+            float4 acc[16];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            // ---- decoupled look-back: excl(b) = S0 + sum_{c<b} U_c
-            if (wt == 0) LA_TRACE(t, TR_LB_START);
-            const bool slot_free = (own && wt == 0) ? probe_reclaim(p, x) : true;
+            for (int k = 0; k < 16; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            // ---- decoupled look-back: excl(b) = S0 + sum_{c<b} U_c (this group's columns)
+            if (wt == 0 && hb == 0) LA_TRACE(t, TR_LB_START);
             {
-                // Depth L = 2: either incl(b-1), or agg(b-1) + incl(b-2); near the
-                // sequence start agg(b-1) (+ S0). Lane 0 of each warp polls the
-                // flags with relaxed loads issued together, decides, and every lane
-                // then takes an acquire fence before reading the chosen states.
+                // Depth up to L: incl(b-1), or agg(b-1) + incl(b-2), or agg(b-1) + agg(b-2)
+                // + incl(b-3), ...; near the sequence start the aggregates down to block 0
+                // plus S0. Lane 0 of each warp polls the flags with relaxed loads, prefers
+                // incl(b-1) during a grace period, decides, takes an acquire fence;
+                // __syncwarp orders it before every lane's reads.
                 const int blk = x.e.blk;
-                int srcs = 0;               // bit 0: incl(b-1), bit 1: agg(b-1), bit 2: incl(b-2), bit 3: S0
+                int srcs = 0;               // bits 0-2: aggregates b-1, b-2, ... to add; bit 3: base is S0
                 if (blk == 0) {
                     srcs = 8;
                 } else if (lane == 0) {
-                    const int64_t f1 = (int64_t)(x.g - 1) * p.H + x.h;
-                    const int64_t f2 = (int64_t)(x.g - 2) * p.H + x.h;
+                    const int64_t fb = (int64_t)x.g * p.H + x.h;      // flag index of block b
                     const uint64_t t0 = globaltimer_ns();
                     for (uint32_t it = 0;; ++it) {
-                        const int i1 = ld_relaxed(p.incl_flag + f1);
-                        const int a1 = ld_relaxed(p.agg_flag + f1);
-                        const int i2 = blk >= 2 ? ld_relaxed(p.incl_flag + f2) : 0;
-                        if (i1) { srcs = 1; break; }
-                        if (a1 && blk == 1) { srcs = 2 | 8; break; }
-                        if (a1 && i2) { srcs = 2 | 4; break; }
+                        if (ld_relaxed(p.incl_flag + fb - p.H)) { srcs = 0; break; }
+                        if (globaltimer_ns() - t0 > p.grace_ns) {
+                            int na = 0;
+                            srcs = -2;
+                            while (na < L - 1 && na < blk && ld_relaxed(p.agg_flag + fb - (int64_t)(na + 1) * p.H)) {
+                                ++na;        // aggregates of blocks b-1 .. b-na are published
+                                if (na == blk) { srcs = na | 8; break; }
+                                if (ld_relaxed(p.incl_flag + fb - (int64_t)(na + 1) * p.H)) { srcs = na; break; }
+                            }
+                            if (srcs >= 0) break;
+                            srcs = 0;
+                        }
                         if ((it & 7u) == 7u) {
                             if (ab.raised()) { *ab.cta = 1; srcs = -1; break; }
                             if (globaltimer_ns() - t0 > ab.limit_ns) { ab.raise(); srcs = -1; break; }
                             __nanosleep(32);
                         }
                     }
-                    // acquire: the flags seen above synchronise with their release stores;
-                    // __syncwarp then orders this before every lane's reads of the states
                     fence_acq_rel_gpu();
                 }
                 __syncwarp();
                 srcs = __shfl_sync(0xffffffffu, srcs, 0);
+                if (wt == 0 && hb == 0) LA_TRACE(t, TR_B_LB_DECIDED);
                 if (srcs < 0) ok = false;
                 if (ok) {
-                    if (srcs & 1) {
-                        const float* src = slot_ptr(p, x, blk - 1, 1);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) {
-                            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (k * D + m) * 4));
-                            acc[k].x += v.x; acc[k].y += v.y; acc[k].z += v.z; acc[k].w += v.w;
-                        }
-                    }
-                    if (srcs & 2) {
-                        const float* src = slot_ptr(p, x, blk - 1, 0);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) {
-                            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (k * D + m) * 4));
-                            acc[k].x += v.x; acc[k].y += v.y; acc[k].z += v.z; acc[k].w += v.w;
-                        }
-                    }
-                    if (srcs & 4) {
-                        const float* src = slot_ptr(p, x, blk - 2, 1);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) {
-                            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (k * D + m) * 4));
-                            acc[k].x += v.x; acc[k].y += v.y; acc[k].z += v.z; acc[k].w += v.w;
-                        }
-                    }
-                    if ((srcs & 8) && p.init) {
+                    const int na = srcs & 7;
+                    for (int c = 1; c <= na; ++c) add_row(acc, slot_ptr(p, x, blk - c, 0));
+                    if (!(srcs & 8)) {
+                        add_row(acc, slot_ptr(p, x, blk - na - 1, 1));
+                    } else if (p.init) {
                         const float4* s0 = reinterpret_cast<const float4*>(
-                            p.init + (((int64_t)x.e.seq * p.H + x.h) * D + m) * D);
+                            p.init + (((int64_t)x.e.seq * p.H + x.h) * D + m) * D) + kb;
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) {
+                        for (int k = 0; k < 16; ++k) {
                             const float4 v = __ldg(s0 + k);
                             acc[k].x += v.x; acc[k].y += v.y; acc[k].z += v.z; acc[k].w += v.w;
                         }
@@ -653,129 +757,112 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 if (ok && !wait_bar(&bars->lbd_pub, (tile_it & 1) ^ 1, ab)) ok = false;
                 ok = warp_all(ok);
                 if (ok) mbar_arrive(&bars->lbd_st);
+                if (wt == 0 && hb == 0) LA_TRACE(t, TR_B_LBD_ST);
             }
             if (!ok) break;
-            // ---- bf16 prefix into shared memory (MN-major, 128-byte swizzle: row m = key index i)
-            if (!warp_all(wait_bar(&bars->pre_empty, (tile_it & 1) ^ 1, ab))) { ok = false; break; }
-            {
-                uint8_t* pre = smem + OFF_PRE;
-#pragma unroll
-                for (int jg = 0; jg < 16; ++jg) {
-                    const float4 lo = acc[2 * jg], hi = acc[2 * jg + 1];
-                    uint4 w;
-                    w.x = pack_bf16x2(lo.x, lo.y); w.y = pack_bf16x2(lo.z, lo.w);
-                    w.z = pack_bf16x2(hi.x, hi.y); w.w = pack_bf16x2(hi.z, hi.w);
-                    const uint32_t off = (jg >> 3) * PREH_BYTES + (m >> 3) * 1024 + (m & 7) * 128 +
-                                         (((jg & 7) ^ (m & 7)) << 4);
-                    *reinterpret_cast<uint4*>(pre + off) = w;
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&bars->pre_full);
-                if (wt == 0) LA_TRACE(t, TR_PREFIX);
-            }
-            // ---- inclusive prefix incl(b) = excl(b) + U_b (the publisher raises its flag)
+            // ---- inclusive prefix incl(b) = excl(b) + U_b first (it is on the chain of the
+            // next block), with U_b read back from the aggregate the P group stored
             if (own) {
-                if (!wait_bar(&bars->u_full, u_it & 1, ab)) ok = false;
-                tc_fence_after();
-                if (ok && wt == 0) {
-                    if (slot_free) fence_acq_rel_gpu();
-                    else if (!wait_reclaim(p, x, ab)) ok = false;
-                }
-                if (!group_sync(&bars->grp_b, grp_phase, ab) || ab.raised()) ok = false;
-                if (ok && !wait_bar(&bars->incl_pub, (u_it & 1) ^ 1, ab)) ok = false;
+                // aggregate stored (CTA scope); the P group waited for the ring slot before
+                // storing it, which also frees the slot's inclusive half
+                if (!wait_bar(&bars->agg_st[u_it & 1], (u_it >> 1) & 1, ab)) ok = false;
                 ok = warp_all(ok);
-                if (ok && t != p.suppress_tile) {
+                if (ok && t != p.suppress_tile) {          // acc keeps excl(b) for the prefix
+                    const float* src = slot_ptr(p, x, x.e.blk, 0);
                     float* dst = slot_ptr(p, x, x.e.blk, 1);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t u[16];
-                        tmem_ld_x16(tmem + lane_base + TM_U + 16 * c, u);
-                        tmem_wait_ld();
+                    for (int k0 = 0; k0 < 16; k0 += 8) {
+                        float4 v[8];
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const float4 a = acc[4 * c + w];
-                            __stcg(reinterpret_cast<float4*>(dst + ((4 * c + w) * D + m) * 4),
-                                   make_float4(a.x + __uint_as_float(u[4 * w]), a.y + __uint_as_float(u[4 * w + 1]),
-                                               a.z + __uint_as_float(u[4 * w + 2]), a.w + __uint_as_float(u[4 * w + 3])));
+                        for (int k = 0; k < 8; ++k)
+                            v[k] = __ldcg(reinterpret_cast<const float4*>(src + ((kb + k0 + k) * D + m) * 4));
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const float4 a4 = acc[k0 + k];
+                            __stcg(reinterpret_cast<float4*>(dst + ((kb + k0 + k) * D + m) * 4),
+                                   make_float4(a4.x + v[k].x, a4.y + v[k].y, a4.z + v[k].z, a4.w + v[k].w));
                         }
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(&bars->u_empty);
+                // the publisher has taken the previous inclusive prefix (one in flight)
+                if (ok && !wait_bar(&bars->incl_pub, (u_it & 1) ^ 1, ab)) ok = false;
+                ok = warp_all(ok);
                 if (ok) mbar_arrive(&bars->incl_st);
+                if (wt == 0 && hb == 0) LA_TRACE(t, TR_B_INCL_ST);
                 ++u_it;
                 if (!ok) break;
             }
-            // ---- O epilogue of each sub-unit, in the order the MMA warp finishes them
-            for (int r = R - 1; ok && r >= 0; --r) {
-                const int rows = sub_rows(x, r);
-                if (rows <= 0) continue;
-                const uint32_t ob = o_it & 1;
-                if (!warp_all(wait_bar(&bars->o_full[ob], (o_it >> 1) & 1, ab))) { ok = false; break; }
-                tc_fence_after();
-                const bool valid = m < rows;
-                __nv_bfloat16* orow = p.out + ((int64_t)(x.e.tok0 + UM * r + m) * p.H + x.h) * D;
-                // drain the whole accumulator row (packed to bf16 on the way) and free
-                // the TMEM buffer at once, so the next sub-unit's P.V can start while
-                // these rows are stored
-                uint32_t pk[64];
+            // ---- bf16 prefix (this group's 64 columns) into its half of the shared
+            // buffer (MN-major, 128-byte swizzle, row m = key index i). The buffer also
+            // stages O for the previous tile's TMA stores: wait until they have read it.
+            if (!warp_all(wait_bar(&bars->pre_empty, (tile_it & 1) ^ 1, ab))) { ok = false; break; }
+            if (!warp_all(wait_bar(&bars->stage_done, (tile_it & 1) ^ 1, ab))) { ok = false; break; }
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t v0[32];
-                    tmem_ld_x32(tmem + lane_base + TM_O + ob * 128 + 32 * c4, v0);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        pk[16 * c4 + c] = pack_bf16x2(__uint_as_float(v0[2 * c]), __uint_as_float(v0[2 * c + 1]));
-                }
-                tc_fence_before();
-                mbar_arrive(&bars->o_empty[ob]);
-                ++o_it;
-                if (valid) {
-#pragma unroll
-                    for (int w = 0; w < 16; ++w)
-                        __stcs(reinterpret_cast<uint4*>(orow + 8 * w),
-                               make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]));
-                }
+            for (int g = 0; g < 8; ++g) {
+                const float4 lo = acc[2 * g], hi = acc[2 * g + 1];
+                uint4 w;
+                w.x = pack_bf16x2(lo.x, lo.y); w.y = pack_bf16x2(lo.z, lo.w);
+                w.z = pack_bf16x2(hi.x, hi.y); w.w = pack_bf16x2(hi.z, hi.w);
+                *reinterpret_cast<uint4*>(half_buf + (m >> 3) * 1024 + (m & 7) * 128 + ((g ^ (m & 7)) << 4)) = w;
             }
-            if (wt == 0) LA_TRACE(t, TR_EPI_END);
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->pre_full);
+            if (wt == 0 && hb == 0) LA_TRACE(t, TR_PREFIX);
             ++tile_it;
         }
-    } else if (warp == 10 && lane == 0) {
+    } else if (warp == 2 && lane == 0) {
         // ================================================================ publisher
-        // Three in-order streams (look-back done, aggregate stored, inclusive stored),
-        // polled round robin without blocking. For each completed item: the worker
-        // group's mbarrier arrive released its stores at CTA scope; the release
-        // store below makes them visible at gpu scope together with the flag.
-        int64_t t_lb = blockIdx.x, t_ag = blockIdx.x, t_in = blockIdx.x;
-        uint32_t n_lb = 0, n_ag = 0, n_in = 0;
+        // Four in-order streams polled round robin without blocking:
+        //   slot: own tile n may write its ring slot once the tiles that may still
+        //         read the slot's previous occupant have finished their look-backs
+        //         (acquire loads of their flags); released to the P group through
+        //         slot_ok, at most one own tile ahead of it (the column groups write
+        //         the slot's inclusive half only after that group's aggregate);
+        //   lb / agg / incl: for each completed item the worker group's mbarrier
+        //         arrive released its accesses at CTA scope; the release store below
+        //         makes them visible at gpu scope together with the flag.
+        int64_t t_lb = blockIdx.x, t_ag = blockIdx.x, t_in = blockIdx.x, t_sl = blockIdx.x;
+        uint32_t n_lb = 0, n_ag = 0, n_in = 0, n_sl = 0;
         auto next_own = [&](int64_t t) {
             while (t < ntiles && !owns_state(tile_of(t, p))) t += gridDim.x;
             return t;
         };
         t_ag = next_own(t_ag);
         t_in = next_own(t_in);
+        t_sl = next_own(t_sl);
         uint64_t t0 = globaltimer_ns();
         while (t_lb < ntiles || t_ag < ntiles || t_in < ntiles) {
             bool any = false;
-            if (t_lb < ntiles && mbar_try_wait(&bars->lbd_st, n_lb & 1)) {
+            if (t_sl < ntiles && n_sl <= n_ag) {
+                const Tile x = tile_of(t_sl, p);
+                const int blk = x.e.blk;
+                int free = 1;
+                for (int c = max(0, blk - W + 1); c <= blk - W + L; ++c)
+                    free &= ld_acquire(p.lb_done + (int64_t)(x.g - (blk - c)) * p.H + x.h);
+                if (free) {
+                    mbar_arrive(&bars->slot_ok);
+                    ++n_sl; t_sl = next_own(t_sl + gridDim.x); any = true;
+                }
+            }
+            if (t_lb < ntiles && mbar_test_wait(&bars->lbd_st, n_lb & 1)) {
                 const Tile x = tile_of(t_lb, p);
                 st_release(p.lb_done + (int64_t)x.g * p.H + x.h, 1);
                 LA_TRACE(t_lb, TR_LB_END);
                 mbar_arrive(&bars->lbd_pub);
                 ++n_lb; t_lb += gridDim.x; any = true;
             }
-            if (t_ag < ntiles && mbar_try_wait(&bars->agg_st, n_ag & 1)) {
+            if (t_ag < ntiles && mbar_test_wait(&bars->agg_st[n_ag & 1], (n_ag >> 1) & 1)) {
                 const Tile x = tile_of(t_ag, p);
+                LA_TRACE(t_ag, TR_PUB_AGG);
                 if (t_ag != p.suppress_tile) {
                     st_release(p.agg_flag + (int64_t)x.g * p.H + x.h, 1);
                     LA_TRACE(t_ag, TR_AGG);
                 }
-                mbar_arrive(&bars->agg_pub);
                 ++n_ag; t_ag = next_own(t_ag + gridDim.x); any = true;
             }
-            if (t_in < ntiles && mbar_try_wait(&bars->incl_st, n_in & 1)) {
+            if (t_in < ntiles && mbar_test_wait(&bars->incl_st, n_in & 1)) {
                 const Tile x = tile_of(t_in, p);
+                LA_TRACE(t_in, TR_PUB_INCL);
                 if (t_in != p.suppress_tile) {
                     st_release(p.incl_flag + (int64_t)x.g * p.H + x.h, 1);
                     LA_TRACE(t_in, TR_INCL);

@@ -300,9 +300,9 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, B, heads, L, ws, st)) != LA_OK) return s;
 
     if (use_tensor_cores(dtype, d, B)) {
-        CUtensorMap tq, tk, tv;
+        CUtensorMap tq, tk, tv, to;
         if (!map_tokens(&tq, q, total_tokens, heads, d, 128) || !map_tokens(&tk, k, total_tokens, heads, d, 64) ||
-            !map_tokens(&tv, v, total_tokens, heads, d, 64))
+            !map_tokens(&tv, v, total_tokens, heads, d, 64) || !map_tokens(&to, o, total_tokens, heads, d, 128))
             return LA_ERR_CUDA;
         la::fused::Params prm;
         prm.out = static_cast<__nv_bfloat16*>(o);
@@ -320,6 +320,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
         prm.suppress_tile = t_suppress_tile;
         const size_t trace_need = (size_t)L.max_blocks * heads * la::fused::kTraceEvents * sizeof(uint64_t);
         prm.trace = (t_trace && t_trace_bytes >= trace_need) ? t_trace : nullptr;
+        prm.grace_ns = 1500;
         if (cudaFuncSetAttribute(la::fused::prefill_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)la::fused::SMEM_BYTES) != cudaSuccess)
             return LA_ERR_CUDA;
@@ -328,7 +329,8 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
         if (sms <= 0) return LA_ERR_CUDA;
         const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
         MainKernelTimer timer(st);
-        la::fused::prefill_fused_kernel<<<grid, la::fused::NTHREADS, la::fused::SMEM_BYTES, st>>>(tq, tk, tv, prm);
+        la::fused::prefill_fused_kernel<<<grid, la::fused::NTHREADS, la::fused::SMEM_BYTES, st>>>(tq, tk, tv, to,
+                                                                                                   prm);
         return cuda_check();
     }
 
