@@ -26,9 +26,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import threading
 import time
 
@@ -55,63 +53,105 @@ def flops_per_token_head(B, d):
     return 4 * B * d + 4 * d * d
 
 
+# DRAM bytes per launch of the main kernels (dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture), stored in profiles/ with the
+# SHA-256 of the kernel's source files at capture time. A figure is reported
+# only while those sources are unchanged; otherwise traffic is null.
+KERNEL_SOURCES = {
+    "prefill_fused_kernel": ("fused.cuh", "sm100.cuh", "common.cuh"),
+    "decode_step_kernel": ("decode.cuh", "common.cuh"),
+}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+
+def kernel_sources_sha(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "causal_linear_attention_02_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(kernel):
+    """Bytes per launch for `kernel` if profiles/ holds a capture of its current sources."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    sha = kernel_sources_sha(kernel)
+    for line in open(TRAFFIC_FILE):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel and parts[1] == sha:
+            return float(parts[2])
+    return None
+
+
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons while the timed region runs."""
+    """SM clock, power and throttle reasons sampled every few milliseconds (NVML)
+    while the timed region runs; read-only queries."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, device, period_s=0.002):
+        self.device = device
+        self.period = period_s
+        self.samples = []
+        self.smax = None
+        self.err = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _handle(self, nv):
+        props = torch.cuda.get_device_properties(self.device)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            devno = getattr(props, "pci_device_id", 0)
+            try:
+                return nv.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{devno:02x}.0".encode())
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+
+    def _run(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), int(get_reasons(h)),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+                return
+            time.sleep(self.period)
 
     def __enter__(self):
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, args=(nv, h), daemon=True)
+            self._thread.start()
+        except Exception as e:  # noqa: BLE001
+            self.err = f"NVML unavailable: {e}"
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons, power = [], None, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for n, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons)}
-        loaded = [x for x in sm if smax and x > 0.5 * smax] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power) if power else None}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.smax, "reasons": [self.err or "no samples"]}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted(n for n, bit in self.REASONS.items() if any(x[1] & bit for x in self.samples))
+        loaded = [x for x in sm if self.smax and x > 0.5 * self.smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": self.smax, "reasons": reasons,
+                "samples": len(sm), "sm_mhz_min": min(sm), "power_w_max": max(x[2] for x in self.samples),
+                "source": "NVML, every 2 ms during the timed region"}
 
 
 # ---------------------------------------------------------------------------- distributed
@@ -210,13 +250,15 @@ def run_cuda(args):
         a.record(); b.record()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(dev) as clocks:
         barrier(pg, local)
         torch.cuda.synchronize(dev)
+        launches0 = la.la_launch_count()
         start.record(stream)
         for i in range(args.steps):
             step(timers[i])
         stop.record(stream)
+        launches = la.la_launch_count() - launches0
         torch.cuda.synchronize(dev)
         barrier(pg, local)
     elapsed_ms = max_over_ranks(pg, start.elapsed_time(stop))
@@ -266,7 +308,6 @@ def run_cuda(args):
         cpu.pop("seconds", None)
 
     if rank == 0:
-        launches_per_step = 5 if la.uses_tensor_cores(torch.bfloat16, d, B) else 5
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -279,11 +320,12 @@ def run_cuda(args):
             "tc_peak_kind": f"{pk_kind} bf16 {pk['bf16_tflops']} TFLOP/s (burst)",
             "roofline": {"bound": "hbm", "kernel": "prefill main kernel", "achieved": achieved_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
-                         "peak_kind": pk_kind, "traffic": None, "kernel_ms": kernel_ms,
+                         "peak_kind": pk_kind, "traffic": captured_traffic("prefill_fused_kernel"),
+                         "kernel_ms": kernel_ms,
                          "algorithmic_bytes": alg_bytes},
             "decode": dec,
             "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": launches,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -343,7 +385,7 @@ def run_decode(la, dev, stream, args, pk, pg, local):
             "value": gbs, "unit": "GB/s", "hbm_frac": gbs / pk["hbm_gbs"],
             "tokens_per_s": Bt / (ms / 1e3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "frac": gbs / pk["hbm_gbs"], "traffic": captured_traffic("decode_step_kernel"),
                          "algorithmic_bytes": state_bytes + io_bytes}}
 
 
@@ -364,7 +406,8 @@ def run_reference(args):
     oracle.recurrent(q1, k1, v1)
     per = (time.perf_counter() - t0) / 1024
     budget = 60.0 / max(1, args.steps + args.warmup)
-    n_heads = max(1, min(H, int(budget * threads / (per * T))))
+    # whole heads, at least one per host thread (the oracle runs heads in parallel)
+    n_heads = max(min(H, threads), min(H, int(budget * threads / (per * T))))
     q, k, v = (x.float().numpy().astype(np.float64) for x in wl.qkv(T, n_heads, d, torch.bfloat16, w.seed))
     for _ in range(args.warmup):
         oracle.recurrent(q, k, v)
@@ -380,7 +423,7 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": w.name, "tokens": T, "heads": H, "d": d, "B": B, "seed": w.seed},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(threads, n_heads), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -390,7 +433,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--no-decode", action="store_true")

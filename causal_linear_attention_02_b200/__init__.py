@@ -25,6 +25,7 @@ __all__ = [
     "la_prefill_workspace_size", "la_prefill", "la_prefill_noalloc", "LA_NOALLOC_SCRATCH_BYTES",
     "la_state_workspace_size", "la_state_from_prefill",
     "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_status_string", "la_version",
+    "la_launch_count",
     "prefill", "state_from_prefill", "decode_step", "device_status", "uses_tensor_cores",
 ]
 
@@ -88,6 +89,8 @@ def load_library():
         lib.la_set_kernel_timer.restype = i32
         lib.la_version.argtypes = []
         lib.la_version.restype = i32
+        lib.la_launch_count.argtypes = []
+        lib.la_launch_count.restype = ctypes.c_uint64
         _lib = lib
         return lib
 
@@ -149,6 +152,10 @@ def la_set_kernel_timer(start_event, stop_event) -> int:
 
 def la_version() -> int:
     return int(load_library().la_version())
+
+
+def la_launch_count() -> int:
+    return int(load_library().la_launch_count())
 
 
 # ---------------------------------------------------------------- marshalling helpers

@@ -44,8 +44,18 @@ using namespace la::sm100;
 constexpr int D = 128;
 constexpr int UM = 128;                    // rows per sub-unit (MMA M)
 constexpr int KC = 64;                     // keys per chunk
-constexpr int NQ = 3;                      // Q sub-unit stages
-constexpr int NKV = 3;                     // K/V chunk stages
+#ifndef LA_FUSED_NQ
+#define LA_FUSED_NQ 3
+#endif
+#ifndef LA_FUSED_NKV
+#define LA_FUSED_NKV 3
+#endif
+#ifndef LA_FUSED_KV_PREFETCH
+#define LA_FUSED_KV_PREFETCH 1
+#endif
+constexpr int NQ = LA_FUSED_NQ;            // Q sub-unit stages
+constexpr int NKV = LA_FUSED_NKV;          // K/V chunk stages
+static_assert(NQ * 32 + NKV * 32 + 32 <= 224, "shared memory: Q stages + K/V stages + prefix buffer");
 constexpr int W = kStateSlots;             // published-state ring slots per chain
 constexpr int L = 3;                       // look-back depth: blocks b-1 .. b-L may be read
 static_assert(W >= L + 2, "slot reuse must not wait on the look-back of the block just before");
@@ -138,7 +148,11 @@ enum TraceEvent {
     TR_A_EPI0_FREE = 26,  // P group: second epilogue sub-unit accumulator released
     TR_A_S0 = 27,         // P group: scores of the tile's first chunk seen
     TR_PUB_AGG = 28,      // publisher: aggregate hand-off seen (before its release store)
-    kTraceEvents = 32
+    TR_A_SJ = 32,         // + j (j < 4): P group, scores of chunk j of the first sub-unit seen
+    TR_A_PJ = 36,         // + j: P group, P of chunk j of the first sub-unit written
+    TR_I_SJ = 40,         // + j: issuer, score MMAs of chunk j of the first sub-unit issued
+    TR_I_PVJ = 44,        // + j: issuer, PV MMAs of chunk j of the first sub-unit issued
+    kTraceEvents = 48
 };
 #define LA_TRACE(t, ev)                                                         \
     do {                                                                       \
@@ -191,6 +205,22 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// fp32 state rows: L2-only (.cg) 16-byte accesses with an L2 eviction-priority hint.
+__device__ __forceinline__ float4 ld_state4(const float* ptr, uint64_t pol) {
+    float4 v;
+    asm volatile("ld.global.cg.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(ptr), "l"(pol) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_state4(float* ptr, float4 v, uint64_t pol) {
+    asm volatile("st.global.cg.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;"
+                 :: "l"(ptr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol) : "memory");
+}
 __device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
                                                  int32_t c0, int32_t c1, int32_t c2, uint64_t pol) {
     asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
@@ -230,6 +260,12 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                                              int32_t c2) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
                  :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1,
+                                                  int32_t c2, uint64_t pol) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;"
+                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -325,7 +361,8 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         // of this tile's sub-units. The lookahead load brings the next tile's K/V
         // into L2, where its own pass finds it a tile later.
         if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
+            const uint64_t pol = policy_evict_first();    // last read of a Q / K / V tile
+            const uint64_t keep = policy_evict_last();    // K / V tiles that are read again soon
             uint32_t q_it = 0, kv_it = 0;
             bool ok = true;
             auto load_chunk = [&](const Tile& y, int j, uint64_t hint) -> bool {
@@ -354,7 +391,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const Tile y = tile_of(tt, p);
                 if (!owns_state(y)) return true;
                 for (int j = 0; j < R * (UM / KC); ++j)
-                    if (!load_chunk(y, j, 0)) return false;
+                    if (!load_chunk(y, j, keep)) return false;   // read again by the tile itself
                 return true;
             };
             if (!load_lookahead(blockIdx.x)) ok = false;
@@ -366,6 +403,19 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         if (sub_rows(y, r) <= 0) continue;
                         tma_prefetch_l2_3d(&tmQ, 0, y.h, y.e.tok0 + UM * r);
                         tma_prefetch_l2_3d(&tmQ, 64, y.h, y.e.tok0 + UM * r);
+                    }
+                }
+                if (LA_FUSED_KV_PREFETCH && t + 2 * (int64_t)gridDim.x < ntiles) {
+                    // K / V of the tile after next into L2, ahead of its look-ahead loads
+                    const Tile y = tile_of(t + 2 * (int64_t)gridDim.x, p);
+                    if (owns_state(y)) {
+                        for (int j = 0; j < R * (UM / KC); ++j) {
+                            const int tk = y.e.tok0 + KC * j;
+                            tma_prefetch_l2_3d(&tmK, 0, y.h, tk);
+                            tma_prefetch_l2_3d(&tmK, 64, y.h, tk);
+                            tma_prefetch_l2_3d(&tmV, 0, y.h, tk);
+                            tma_prefetch_l2_3d(&tmV, 64, y.h, tk);
+                        }
                     }
                 }
                 if (!load_lookahead(t + gridDim.x)) { ok = false; break; }
@@ -384,7 +434,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     for (int j = 0; j < nkc; ++j) {
                         // chunks re-streamed by a later sub-unit of the same block stay in L2
                         const bool again = r == R - 1 && R > 1 && j < (R - 1) * (UM / KC);
-                        if (!load_chunk(x, j, again ? 0 : pol)) { ok = false; break; }
+                        if (!load_chunk(x, j, again ? keep : pol)) { ok = false; break; }
                     }
                 }
             }
@@ -459,6 +509,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                             mma_ss(d_s, sdesc_sw128(qa + (s >> 2) * QH_BYTES + (s & 3) * 32, 16, 1024),
                                    sdesc_sw128(kb + (s >> 2) * KVH_BYTES + (s & 3) * 32, 16, 1024), IDESC_S, s > 0);
                         tc_commit(&bars->s_full[(s_it + j) & 1]);
+                        if (nsub == 0 && j < 4) LA_TRACE(t, TR_I_SJ + j);
                         return true;
                     };
                     if (!issue_scores(0)) { ok = false; break; }
@@ -480,6 +531,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                             mma_ts(d_o, a_p + s * 8, sdesc_sw128(vb + s * 2048, KVH_BYTES, 1024), IDESC_PV,
                                    (j > 0 || s > 0));
                         tc_commit(&bars->kv_empty[st]);
+                        if (nsub == 0 && j < 4) LA_TRACE(t, TR_I_PVJ + j);
                     }
                     if (!ok) break;
                     kv_it += nkc;
@@ -522,6 +574,8 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const int wt = threadIdx.x - 128;                 // 0..127 within this group
         uint32_t s_it = 0, u_it = 0, o_it = 0, tile_it = 0, grp_phase = 0;
         bool ok = true;
+        const uint64_t keep = policy_evict_last();       // published states stay in L2
+        const uint64_t o_pol = policy_evict_first();     // O is never read back
         // Store the block state of tile tt (computed one tile ahead by the issuer) as
         // the aggregate of its ring slot; the publisher raises its flag.
         auto store_aggregate = [&](int64_t tt) -> bool {
@@ -542,9 +596,10 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     tmem_wait_ld();
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
-                        __stcg(reinterpret_cast<float4*>(dst + ((4 * c + w) * D + m) * 4),
-                               make_float4(__uint_as_float(u[4 * w]), __uint_as_float(u[4 * w + 1]),
-                                           __uint_as_float(u[4 * w + 2]), __uint_as_float(u[4 * w + 3])));
+                        st_state4(dst + ((4 * c + w) * D + m) * 4,
+                                  make_float4(__uint_as_float(u[4 * w]), __uint_as_float(u[4 * w + 1]),
+                                              __uint_as_float(u[4 * w + 2]), __uint_as_float(u[4 * w + 3])),
+                                  keep);
                 }
             }
             tc_fence_before();
@@ -565,6 +620,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     const uint32_t sb = s_it & 1;
                     if (!warp_all(wait_bar(&bars->s_full[sb], (s_it >> 1) & 1, ab))) { ok = false; break; }
                     if (wt == 0 && r == R - 1 && j == 0) LA_TRACE(t, TR_A_S0);
+                    if (wt == 0 && r == R - 1 && j < 4) LA_TRACE(t, TR_A_SJ + j);
                     tc_fence_after();
                     const uint32_t ts = tmem + lane_base + TM_S + sb * 64;
                     const int lim = qi - KC * j;          // key column c is kept when c <= lim
@@ -592,6 +648,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     tc_fence_before();
                     mbar_arrive(&bars->p_full[sb]);
                     if (wt == 0 && r == 0 && j + 1 == nkc) LA_TRACE(t, TR_P_END);
+                    if (wt == 0 && r == R - 1 && j < 4) LA_TRACE(t, TR_A_PJ + j);
                 }
             }
             // ---- O epilogue of each sub-unit, in the order the issuer finishes them:
@@ -649,8 +706,8 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (!warp_all(group_sync(&bars->grp_a, grp_phase, ab))) { ok = false; break; }
                     if (wt == 0) {
                         const int tq = x.e.tok0 + UM * r;
-                        tma_store_3d(&tmO, stage, 0, x.h, tq);
-                        tma_store_3d(&tmO, stage + PREH_BYTES, 64, x.h, tq);
+                        tma_store_3d_hint(&tmO, stage, 0, x.h, tq, o_pol);
+                        tma_store_3d_hint(&tmO, stage + PREH_BYTES, 64, x.h, tq, o_pol);
                         bulk_commit();
                     }
                 }
@@ -678,13 +735,14 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         uint8_t* half_buf = smem + OFF_PRE + hb * PREH_BYTES;   // prefix half (O staging between tiles)
         uint32_t tile_it = 0, u_it = 0;
         bool ok = true;
+        const uint64_t keep = policy_evict_last();       // published states stay in L2
         auto add_row = [&](float4 (&acc)[16], const float* src) {
 #pragma unroll
             for (int k0 = 0; k0 < 16; k0 += 8) {          // 8 loads in flight at a time
                 float4 v[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    v[k] = __ldcg(reinterpret_cast<const float4*>(src + ((kb + k0 + k) * D + m) * 4));
+                    v[k] = ld_state4(src + ((kb + k0 + k) * D + m) * 4, keep);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     acc[k0 + k].x += v[k].x; acc[k0 + k].y += v[k].y;
@@ -775,12 +833,13 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         float4 v[8];
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
-                            v[k] = __ldcg(reinterpret_cast<const float4*>(src + ((kb + k0 + k) * D + m) * 4));
+                            v[k] = ld_state4(src + ((kb + k0 + k) * D + m) * 4, keep);
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
                             const float4 a4 = acc[k0 + k];
-                            __stcg(reinterpret_cast<float4*>(dst + ((kb + k0 + k) * D + m) * 4),
-                                   make_float4(a4.x + v[k].x, a4.y + v[k].y, a4.z + v[k].z, a4.w + v[k].w));
+                            st_state4(dst + ((kb + k0 + k) * D + m) * 4,
+                                      make_float4(a4.x + v[k].x, a4.y + v[k].y, a4.z + v[k].z, a4.w + v[k].w),
+                                      keep);
                         }
                     }
                 }

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <stdint.h>
 #include <string.h>
@@ -125,6 +126,10 @@ int num_sms() {
 
 la_status cuda_check() { return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
+// Kernels launched by the library since the process started (la_launch_count).
+std::atomic<uint64_t> g_launches{0};
+inline void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 // Test hook (la_debug_set_fault): a tile that publishes nothing and a shorter wait limit.
 thread_local long long t_suppress_tile = -1;
 thread_local uint64_t t_wait_ns = 0;
@@ -156,9 +161,11 @@ la_status launch_block_table(const int32_t* cu, int nseq, int64_t T, int B, int 
     BlockEntry* table = reinterpret_cast<BlockEntry*>(ws + L.off_table);
     int32_t* flags = L.nflag_arrays ? reinterpret_cast<int32_t*>(ws + L.off_flags) : nullptr;
     la::seq_blocks_kernel<<<1, 1024, 0, st>>>(cu, nseq, T, B, seq_blk, seq_slot, ctrl);
+    note_launch();
     const int64_t nb = (L.max_blocks + 255) / 256;
     la::fill_block_table_kernel<<<(unsigned)nb, 256, 0, st>>>(cu, nseq, T, B, seq_blk, seq_slot, ctrl, table,
                                                               L.max_blocks, flags, L.nflag_arrays, H);
+    note_launch();
     return cuda_check();
 }
 
@@ -175,6 +182,7 @@ la_status prefill_simt_main(const void* q, const void* k, const void* v, void* o
     const int64_t grid = L.max_blocks * H * (B / 64);
     la::simt::prefill_simt<Tin, D><<<(unsigned)grid, la::simt::THREADS, smem, st>>>(
         (const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, prefix, table, ctrl, H, B);
+    note_launch();
     return cuda_check();
 }
 
@@ -185,6 +193,7 @@ la_status state_simt_launch(const void* k, const void* v, int H, const Layout& L
     float* U = reinterpret_cast<float*>(ws + L.off_U);
     la::simt::block_state_simt<Tin, D><<<(unsigned)(L.max_blocks * H), la::simt::THREADS, 0, st>>>(
         (const Tin*)k, (const Tin*)v, table, ctrl, H, U);
+    note_launch();
     return cuda_check();
 }
 
@@ -225,6 +234,7 @@ la_status decode_launch(la_dtype dt, const void* q, const void* k, const void* v
     else
         la::decode_step_kernel<float, D><<<(unsigned)pairs, nt, 0, st>>>(
             (const float*)q, (const float*)k, (const float*)v, state, (float*)o);
+    note_launch();
     return cuda_check();
 }
 
@@ -331,6 +341,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
         MainKernelTimer timer(st);
         la::fused::prefill_fused_kernel<<<grid, la::fused::NTHREADS, la::fused::SMEM_BYTES, st>>>(tq, tk, tv, to,
                                                                                                    prm);
+        note_launch();
         return cuda_check();
     }
 
@@ -339,6 +350,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     dim3 sg((dd + 1023) / 1024, num_seqs * heads);
     la::chain_scan_kernel<float><<<sg, 256, 0, st>>>(U, reinterpret_cast<float*>(ws + L.off_prefix), init_state,
                                                      nullptr, seq_blk, ctrl, num_seqs, heads, dd, true);
+    note_launch();
     if ((s = cuda_check()) != LA_OK) return s;
     MainKernelTimer timer(st);
     return simt_prefill_d(d, dtype, q, k, v, o, heads, B, L, ws, st);
@@ -369,6 +381,7 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
         reinterpret_cast<const float*>(ws + L.off_U), static_cast<float*>(nullptr), init_state, state_out,
         reinterpret_cast<const int32_t*>(ws + L.off_seq_blk), reinterpret_cast<const Control*>(ws), num_seqs,
         heads, dd, false);
+    note_launch();
     return cuda_check();
 }
 
@@ -407,6 +420,8 @@ la_status la_debug_set_fault(long long suppress_tile, uint64_t wait_ns) {
     t_wait_ns = wait_ns;
     return LA_OK;
 }
+
+uint64_t la_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 la_status la_debug_set_trace(void* device_buffer, size_t bytes) {
     if ((device_buffer == nullptr) != (bytes == 0)) return LA_ERR_INVALID_ARGUMENT;

@@ -172,17 +172,24 @@ la_status la_debug_set_fault(long long suppress_tile, uint64_t wait_ns);
 /*
  * Tracing (no counterpart on the pages). While a buffer is set, every
  * la_prefill call made by this host thread on the tensor-core path records,
- * for each tile (block * heads + head over the blocks of all sequences), 32
+ * for each tile (block * heads + head over the blocks of all sequences), 48
  * uint64 globaltimer stamps (ns) of its phases into `device_buffer`: [0] first
  * Q tile ready, [1] chunk MMAs issued, [2] prefix available, [3]/[4] look-back
  * start/end, [5] prefix written, [6] inclusive state published, [7] output
- * stored, [8] aggregate published, [9] last P written, [10..31] finer steps of
+ * stored, [8] aggregate published, [9] last P written, [10..47] finer steps of
  * the worker roles; unused slots are left as they were. The buffer must hold
- * max_tiles * 256 bytes, max_tiles =
+ * max_tiles * 384 bytes, max_tiles =
  * (ceil(total_tokens / B) + num_seqs) * heads, or the call records nothing.
  * NULL, 0 stops tracing.
  */
 la_status la_debug_set_trace(void* device_buffer, size_t bytes);
+
+/*
+ * Number of kernels this library has launched, from every host thread, since
+ * the process loaded it (no counterpart on the pages). Read it before and
+ * after a sequence of calls to count the launches they made. Never fails.
+ */
+uint64_t la_launch_count(void);
 
 /* Static, human-readable name of a status code. */
 const char* la_status_string(la_status s);
