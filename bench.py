@@ -58,7 +58,8 @@ def flops_per_token_head(B, d):
 # SHA-256 of the kernel's source files at capture time. A figure is reported
 # only while those sources are unchanged; otherwise traffic is null.
 KERNEL_SOURCES = {
-    "prefill_fused_kernel": ("fused.cuh", "sm100.cuh", "common.cuh"),
+    "prefill_chain_kernel": ("chain.cuh", "pipe.cuh", "sm100.cuh", "common.cuh"),
+    "prefill_fused_kernel": ("fused.cuh", "pipe.cuh", "sm100.cuh", "common.cuh"),
     "decode_step_kernel": ("decode.cuh", "common.cuh"),
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
@@ -318,9 +319,9 @@ def run_cuda(args):
             "tflops": tflops,
             "tc_peak_frac": tflops / world / pk["bf16_tflops"],
             "tc_peak_kind": f"{pk_kind} bf16 {pk['bf16_tflops']} TFLOP/s (burst)",
-            "roofline": {"bound": "hbm", "kernel": "prefill main kernel", "achieved": achieved_gbs,
+            "roofline": {"bound": "hbm", "kernel": "prefill_chain_kernel", "achieved": achieved_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
-                         "peak_kind": pk_kind, "traffic": captured_traffic("prefill_fused_kernel"),
+                         "peak_kind": pk_kind, "traffic": captured_traffic("prefill_chain_kernel"),
                          "kernel_ms": kernel_ms,
                          "algorithmic_bytes": alg_bytes},
             "decode": dec,

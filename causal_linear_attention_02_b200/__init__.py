@@ -24,7 +24,7 @@ __all__ = [
     "LightningError", "LA_BF16", "LA_FP32", "STATUS", "library_path", "load_library",
     "la_prefill_workspace_size", "la_prefill", "la_prefill_noalloc", "LA_NOALLOC_SCRATCH_BYTES",
     "la_state_workspace_size", "la_state_from_prefill",
-    "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_status_string", "la_version",
+    "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
     "la_launch_count",
     "prefill", "state_from_prefill", "decode_step", "device_status", "uses_tensor_cores",
 ]
@@ -89,6 +89,8 @@ def load_library():
         lib.la_set_kernel_timer.restype = i32
         lib.la_version.argtypes = []
         lib.la_version.restype = i32
+        lib.la_debug_set_path.argtypes = [i32]
+        lib.la_debug_set_path.restype = i32
         lib.la_launch_count.argtypes = []
         lib.la_launch_count.restype = ctypes.c_uint64
         _lib = lib
@@ -140,6 +142,10 @@ def la_status_string(status: int) -> str:
 
 def la_debug_set_fault(suppress_tile: int, wait_ns: int) -> int:
     return int(load_library().la_debug_set_fault(suppress_tile, wait_ns))
+
+
+def la_debug_set_path(path: int) -> int:
+    return int(load_library().la_debug_set_path(path))
 
 
 def la_debug_set_trace(device_buffer, nbytes: int) -> int:

@@ -1,0 +1,656 @@
+// Lightning Attention prefill with the running state kept on chip: one
+// persistent CTA per (sequence, head, half of the value columns), blocks of
+// that sequence walked in order. bf16, d = 128, B in {128, 256}.
+//
+// Method (page "MiniMax-01 Lightning Attention", section "Lightning Attention
+// 设计"; page "首个线性注意力架构的大模型来了…", section "4.1 创新的线性注意力",
+// 双阶段计算):
+//   O_b = (Q_b K_b^T, causal mask) V_b  +  Q_b . KV_b,
+//   KV_0 = S0,  KV_{b+1} = KV_b + K_b^T V_b   (exclusive prefix over the blocks).
+// Column j of O_b and of KV depends on column j of V only, so one (sequence,
+// head) splits into two independent halves of 64 value columns. Each half is
+// one work item; work items are taken round-robin by the CTAs, longest
+// sequence first. Inside a work item the exclusive prefix is a running sum:
+// the tensor cores accumulate K_b^T V_b into a fp32 TMEM accumulator block
+// after block, and before block b's keys are added the state group copies
+// KV_b (+ S0) out as the bf16 operand of the inter-block product. No block
+// state ever goes to global memory, so Q, K, V are read once per work item
+// and O is written once.
+//
+// A block of B rows is R = B/128 sub-units of 128 query rows; keys arrive in
+// chunks of 128 (chunk j = keys 128j .. 128j+127 of the block). Items
+// (chunk j, sub-unit r) with j <= r, in the order (0,1), (0,0), (1,1):
+//   scores  S = Q_r K_j^T               (M=128, N=128, K=128)  -> TMEM
+//   P       = bf16(mask(S)), written back into TMEM (two warpgroups, one per
+//             64-key half of the chunk)
+//   PV      O_r += P V_j                (M=128, N=64,  K=128)  A from TMEM
+//   state   KV += K_j^T V_j             (M=128, N=64,  K=128)  after the chunk's last item
+//   inter   O_r += Q_r . bf16(KV_b)     (M=128, N=64,  K=128)  after sub-unit r's last item
+// Roles (512 threads):
+//   warp 0 (lane 0)  TMA producer of K / V chunks (+ L2 prefetch of the next block)
+//   warp 1 (lane 0)  tcgen05 issuer: a non-blocking event loop; score MMAs run
+//                    ahead of the PV cursor as far as the rings allow
+//   warp 2 (lane 0)  TMA producer of Q sub-units (+ L2 prefetch of the next block)
+//   warps 4-7, 8-11  scores -> P, keys 0-63 and 64-127 of every item
+//   warps 12-15      state copy-out (TMEM fp32 -> bf16 shared operand) and O
+//                    epilogue (TMEM -> bf16 -> swizzled staging -> TMA store;
+//                    a ragged last sub-unit by masked direct stores)
+// Every wait is bounded (globaltimer); on expiry the CTA records
+// LA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
+#pragma once
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "pipe.cuh"
+
+namespace la {
+namespace chain {
+
+using namespace la::sm100;
+
+constexpr int D = 128;                     // head dim (d_k = d_v)
+constexpr int DV = 64;                     // value columns per work item
+constexpr int UM = 128;                    // rows per sub-unit (MMA M)
+constexpr int KC = 128;                    // keys per chunk
+constexpr int NQ = 3;                      // Q sub-unit stages
+constexpr int NKV = 2;                     // K/V chunk stages
+constexpr int NS = 2;                      // score buffers in TMEM
+constexpr int NTHREADS = 512;
+
+constexpr uint32_t QH_BYTES = UM * 64 * 2;       // 16 KB: 128 rows x 64 columns
+constexpr uint32_t Q_BYTES = 2 * QH_BYTES;       // 32 KB
+constexpr uint32_t KH_BYTES = KC * 64 * 2;       // 16 KB: 128 keys x 64 columns
+constexpr uint32_t K_BYTES = 2 * KH_BYTES;       // 32 KB
+constexpr uint32_t V_BYTES = KC * DV * 2;        // 16 KB
+constexpr uint32_t KV_STAGE = K_BYTES + V_BYTES; // 48 KB
+constexpr uint32_t SB_BYTES = D * DV * 2;        // 16 KB: bf16 KV_b, 128 rows x 64 columns
+constexpr uint32_t STG_BYTES = UM * DV * 2;      // 16 KB: O staging, 128 rows x 64 columns
+
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_KV = OFF_Q + NQ * Q_BYTES;
+constexpr uint32_t OFF_SB = OFF_KV + NKV * KV_STAGE;
+constexpr uint32_t OFF_STG = OFF_SB + SB_BYTES;
+constexpr uint32_t OFF_BAR = OFF_STG + STG_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;   // + barriers + 1 KB alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+
+// TMEM columns (512 x 32-bit, 128 lanes): three O slots, the state, NS score buffers.
+constexpr uint32_t TM_O = 0, TM_KV = 192, TM_S = 256, TM_COLS = 512;
+static_assert(TM_S + NS * KC <= TM_COLS, "TMEM budget");
+
+constexpr uint32_t IDESC_S = idesc_bf16(UM, KC, false, false);   // Q (K-major) x K (K-major)
+constexpr uint32_t IDESC_PV = idesc_bf16(UM, DV, false, true);   // P (TMEM) x V (MN-major)
+constexpr uint32_t IDESC_KV = idesc_bf16(D, DV, true, true);     // K^T (MN-major) x V (MN-major)
+constexpr uint32_t IDESC_C = idesc_bf16(UM, DV, false, true);    // Q (K-major) x KV (MN-major)
+
+struct Bars {
+    uint64_t q_full[NQ], q_empty[NQ];
+    uint64_t kv_full[NKV], kv_empty[NKV];
+    uint64_t s_full[NS], p_full[NS];
+    uint64_t o_full[3], o_empty[3];
+    uint64_t kv_ready;        // issuer -> state group: KV accumulator holds the next block's prefix
+    uint64_t kv_read[2];      // state group -> issuer: accumulator read for block n (n & 1)
+    uint64_t sb_full, sb_empty;
+    uint64_t grp;             // bounded barrier of the state / epilogue group
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(Bars) <= 512, "barrier block");
+
+struct Params {
+    __nv_bfloat16* out;
+    const SeqEntry* seqs;     // [nseq] first token and length
+    const int32_t* order;     // [nseq] sequences, longest first
+    const Control* ctrl;
+    const float* init;        // [nseq][H][D][D] carried-in state, or nullptr
+    int H, B, nseq;
+    uint64_t wait_ns;
+    long long suppress_item;  // test hook: this work item never hands over its second block's prefix (-1: none)
+    uint64_t* trace;          // optional [gridDim.x][trace_blocks][kTraceEvents] clock64 stamps, or nullptr
+    int trace_blocks;         // blocks per CTA the trace buffer holds
+};
+
+// Phase stamps of the optional per-block trace (la_debug_set_trace), in SM
+// clock cycles (clock64), indexed by the CTA's block counter n.
+enum TraceEvent {
+    TR_Q0 = 0,         // Q producer: first Q sub-unit load of the block issued
+    TR_KV0 = 1,        // K/V producer: chunk 0 load issued
+    TR_KVL = 2,        // K/V producer: last chunk load issued
+    TR_S0 = 3,         // issuer: first score MMA of the block issued
+    TR_PV0 = 4,        // issuer: first PV MMA issued (its P was ready)
+    TR_C0 = 5,         // issuer: inter-block MMA of sub-unit 0 issued
+    TR_KVR = 6,        // issuer: last state MMA issued (kv_ready committed)
+    TR_CL = 7,         // issuer: inter-block MMA of the last sub-unit issued
+    TR_P0 = 8,         // P groups: P of the first item written
+    TR_PL = 9,         // P groups: P of the last item written
+    TR_XR = 10,        // state group: accumulator ready seen
+    TR_SB = 11,        // state group: bf16 prefix handed over
+    TR_E0 = 12,        // state group: first sub-unit accumulator complete
+    TR_EL = 13,        // state group: last sub-unit accumulator complete
+    TR_ST = 14,        // state group: last O store issued
+    TR_PVL = 15,       // issuer: last PV MMA issued
+    kTraceEvents = 16
+};
+// Per-item stamps of CTA 0 (compile-time option LA_CHAIN_ITEM_TRACE): eight
+// clock64 values per item after the block table in the trace buffer.
+#ifdef LA_CHAIN_ITEM_TRACE
+#define LA_ITRACE(i, ev)                                                                                    \
+    do {                                                                                                    \
+        if (p.trace && blockIdx.x == 0 && (int)(i) < 4096)                                                  \
+            p.trace[(int64_t)gridDim.x * p.trace_blocks * kTraceEvents + (int64_t)(i) * 8 + (ev)] = clock64(); \
+    } while (0)
+#else
+#define LA_ITRACE(i, ev) do {} while (0)
+#endif
+#define LA_CTRACE(n, ev)                                                                                   \
+    do {                                                                                                   \
+        if (p.trace && (int)(n) < p.trace_blocks)                                                          \
+            p.trace[((int64_t)blockIdx.x * p.trace_blocks + (n)) * kTraceEvents + (ev)] = clock64();       \
+    } while (0)
+
+// Walks this CTA's work items -> blocks -> items in the order every role uses,
+// with the running counters that index the rings: n (blocks), q0 (Q
+// sub-units), kc0 (K/V chunks), o0 (uses of O slot 0) at the current block,
+// and i (items). A block has Rb = ceil(rows / 128) sub-units and as many
+// 128-key chunks; its items are (0,1), (0,0), (1,1) when Rb = 2 and (0,0)
+// when Rb = 1.
+struct Cursor {
+    int64_t w, nitems;
+    int step;
+    int seq, h, half, tok_s, len, nb;    // work item
+    int b, tok0, rows, Rb;               // block
+    bool add_state;                      // the block's K^T V is needed (not the last block)
+    uint32_t n, q0, kc0, o0;
+    int k;                               // item within the block
+    int j, r;                            // its chunk and sub-unit
+    uint32_t i;
+    bool valid;
+
+    __device__ __forceinline__ void set_item() {
+        if (Rb == 2) {
+            j = k == 2 ? 1 : 0;
+            r = k == 1 ? 0 : 1;
+        } else {
+            j = 0;
+            r = 0;
+        }
+    }
+    __device__ __forceinline__ void load_block(const Params& p) {
+        tok0 = tok_s + b * p.B;
+        rows = min(p.B, len - b * p.B);
+        Rb = (rows + UM - 1) / UM;
+        add_state = b + 1 < nb;
+        k = 0;
+        set_item();
+    }
+    __device__ __forceinline__ bool load_work(const Params& p) {
+        for (; w < nitems; w += step) {
+            const int64_t pair = w >> 1;
+            seq = p.order[pair / p.H];
+            h = (int)(pair % p.H);
+            half = (int)(w & 1);
+            const SeqEntry e = p.seqs[seq];
+            tok_s = e.tok0;
+            len = e.len;
+            if (len > 0) {
+                nb = (len + p.B - 1) / p.B;
+                b = 0;
+                load_block(p);
+                return true;
+            }
+        }
+        return false;
+    }
+    __device__ __forceinline__ void init(const Params& p) {
+        w = blockIdx.x;
+        step = gridDim.x;
+        nitems = (int64_t)p.nseq * p.H * 2;
+        n = q0 = kc0 = o0 = 0;
+        i = 0;
+        valid = p.ctrl->ok && load_work(p);
+    }
+    __device__ __forceinline__ void next_block(const Params& p) {
+        ++n;
+        q0 += Rb;
+        kc0 += Rb;
+        if (Rb == 2) ++o0;
+        if (++b < nb) {
+            load_block(p);
+            return;
+        }
+        w += step;
+        valid = load_work(p);
+    }
+    __device__ __forceinline__ void next_item(const Params& p) {
+        ++i;
+        if (++k < (Rb == 2 ? 3 : 1)) {
+            set_item();
+            return;
+        }
+        next_block(p);
+    }
+    // item properties
+    __device__ __forceinline__ bool first_of_chunk() const { return k != 1; }     // (0,1) or (0,0) alone, (1,1)
+    __device__ __forceinline__ bool last_of_chunk() const { return k != 0 || Rb == 1; }
+    __device__ __forceinline__ bool last_of_block() const { return k == (Rb == 2 ? 2 : 0); }
+    // O slot of sub-unit rr: the sub-unit that finishes last alternates between
+    // slots 1 and 2 from block to block; sub-unit 0 of a two-sub-unit block
+    // (finished mid-block) always uses slot 0.
+    __device__ __forceinline__ uint32_t oslot(int rr) const { return rr == Rb - 1 ? 1 + (n & 1) : 0; }
+    __device__ __forceinline__ uint32_t ouse(int rr) const { return rr == Rb - 1 ? (n >> 1) : o0; }
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Abort ab{&bars->abort_flag, const_cast<volatile int*>(&p.ctrl->abort), p.wait_ns};
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NQ; ++i) { mbar_init(&bars->q_full[i], 1); mbar_init(&bars->q_empty[i], 1); }
+        for (int i = 0; i < NKV; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
+        for (int i = 0; i < NS; ++i) { mbar_init(&bars->s_full[i], 1); mbar_init(&bars->p_full[i], 256); }
+        for (int i = 0; i < 3; ++i) { mbar_init(&bars->o_full[i], 1); mbar_init(&bars->o_empty[i], 128); }
+        mbar_init(&bars->kv_ready, 1);
+        mbar_init(&bars->kv_read[0], 128);
+        mbar_init(&bars->kv_read[1], 128);
+        mbar_init(&bars->sb_full, 128);
+        mbar_init(&bars->sb_empty, 1);
+        mbar_init(&bars->grp, 128);
+        mbar_init(&bars->drain, 1);
+        bars->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, TM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmO);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0 || warp == 2) {
+        // ================================================================ TMA producers
+        if (lane == 0) {
+            const bool kv_role = warp == 0;
+            const uint64_t once = policy_evict_first();      // V: read by this CTA only
+            Cursor c;
+            c.init(p);
+            uint32_t issued = 0;                              // loads issued (ring index)
+            bool ok = true;
+            while (ok && c.valid) {
+                // the next block's tiles into L2 while this block's are loaded
+                Cursor nx = c;
+                nx.next_block(p);
+                if (nx.valid) {
+                    for (int r = 0; r < nx.Rb; ++r) {
+                        const int t = nx.tok0 + UM * r;
+                        if (kv_role) {
+                            tma_prefetch_l2_3d(&tmK, 0, nx.h, t);
+                            tma_prefetch_l2_3d(&tmK, 64, nx.h, t);
+                            tma_prefetch_l2_3d(&tmV, DV * nx.half, nx.h, t);
+                        } else {
+                            tma_prefetch_l2_3d(&tmQ, 0, nx.h, t);
+                            tma_prefetch_l2_3d(&tmQ, 64, nx.h, t);
+                        }
+                    }
+                }
+                for (int r = 0; r < c.Rb; ++r) {      // sub-unit r's Q rows; chunk r's keys
+                    const int t = c.tok0 + UM * r;
+                    if (kv_role) {
+                        const uint32_t kc = c.kc0 + r, st = kc % NKV;
+                        if (!wait_bar(&bars->kv_empty[st], ((kc / NKV) & 1) ^ 1, ab)) { ok = false; break; }
+                        uint8_t* kd = smem + OFF_KV + st * KV_STAGE;
+                        mbar_expect_tx(&bars->kv_full[st], KV_STAGE);
+                        tma_load_3d(kd, &tmK, &bars->kv_full[st], 0, c.h, t);
+                        tma_load_3d(kd + KH_BYTES, &tmK, &bars->kv_full[st], 64, c.h, t);
+                        tma_load_3d_hint(kd + K_BYTES, &tmV, &bars->kv_full[st], DV * c.half, c.h, t, once);
+                        issued = kc + 1;
+                        if (r == 0) LA_CTRACE(c.n, TR_KV0);
+                        if (r == c.Rb - 1) LA_CTRACE(c.n, TR_KVL);
+                    } else {
+                        const uint32_t qc = c.q0 + r, qs = qc % NQ;
+                        if (!wait_bar(&bars->q_empty[qs], ((qc / NQ) & 1) ^ 1, ab)) { ok = false; break; }
+                        uint8_t* qd = smem + OFF_Q + qs * Q_BYTES;
+                        mbar_expect_tx(&bars->q_full[qs], Q_BYTES);
+                        tma_load_3d(qd, &tmQ, &bars->q_full[qs], 0, c.h, t);
+                        tma_load_3d(qd + QH_BYTES, &tmQ, &bars->q_full[qs], 64, c.h, t);
+                        issued = qc + 1;
+                        if (r == 0) LA_CTRACE(c.n, TR_Q0);
+                    }
+                }
+                c.next_block(p);
+            }
+            // On abort, wait (bounded) for this producer's copies still in flight
+            // into shared memory: only the latest load of each stage can be pending.
+            if (!ok) {
+                const uint32_t nst = kv_role ? NKV : NQ;
+                uint64_t* full = kv_role ? bars->kv_full : bars->q_full;
+                for (uint32_t i = (issued > nst ? issued - nst : 0); i < issued; ++i) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(&full[i % nst], (i / nst) & 1) && globaltimer_ns() - t0 < 100000000ull) {}
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================================ tcgen05 issuer
+        if (lane == 0) {
+            // Shared-memory descriptors: the base of each region once, then a
+            // 16-byte-unit offset per operand step (the address field is the low 14 bits).
+            const uint64_t dq = sdesc_sw128(smem_u32(smem + OFF_Q), 16, 1024);             // K-major
+            const uint64_t dk = sdesc_sw128(smem_u32(smem + OFF_KV), 16, 1024);            // K-major (scores)
+            const uint64_t dkt = sdesc_sw128(smem_u32(smem + OFF_KV), KH_BYTES, 1024);     // MN-major (state)
+            const uint64_t dv = sdesc_sw128(smem_u32(smem + OFF_KV + K_BYTES), V_BYTES, 1024);
+            const uint64_t dsb = sdesc_sw128(smem_u32(smem + OFF_SB), SB_BYTES, 1024);
+            Cursor sc, pc;
+            sc.init(p);
+            pc.init(p);
+            // Event loop: every step is taken only when its inputs are ready (non-
+            // blocking mbarrier tests), so a score waiting for its K/V chunk never
+            // holds back a PV whose P is already in TMEM. The score cursor runs ahead
+            // of the PV cursor only as far as the rings allow without waiting on this
+            // thread's own later work: a score buffer is reused after the PV that
+            // read it, a K/V or Q stage is refilled after the commit that released it.
+            uint32_t pv_issued = 0, kv_released = 0, q_released = 0;
+            int stage = 0;                        // PV cursor's item: 0 PV, 1 state MMA, 2 inter MMA, 3 done
+            uint32_t kvr_blk = 0xffffffffu;       // block whose state copy-out has been seen
+            uint32_t idle = 0;
+            uint64_t t_idle = 0;
+            while (pc.valid) {
+                bool prog = false;
+                // ---- (a) score MMAs ahead of the PV cursor
+                if (sc.valid && sc.i < pv_issued + NS && sc.kc0 + sc.j < kv_released + NKV &&
+                    sc.q0 + sc.r < q_released + NQ) {
+                    const uint32_t kc = sc.kc0 + sc.j, st = kc % NKV;
+                    const uint32_t qc = sc.q0 + sc.r, qs = qc % NQ;
+                    if ((!sc.first_of_chunk() || mbar_test_wait(&bars->kv_full[st], (kc / NKV) & 1)) &&
+                        (sc.j != 0 || mbar_test_wait(&bars->q_full[qs], (qc / NQ) & 1))) {
+                        tc_fence_after();
+                        LA_ITRACE(sc.i, 0);
+                        const uint64_t a = dq + ((qs * Q_BYTES) >> 4), b = dk + ((st * KV_STAGE) >> 4);
+                        const uint32_t d_s = tmem + TM_S + (sc.i % NS) * KC;
+#pragma unroll
+                        for (int s = 0; s < D / 16; ++s)
+                            mma_ss(d_s, a + (((s >> 2) * QH_BYTES + (s & 3) * 32) >> 4),
+                                   b + (((s >> 2) * KH_BYTES + (s & 3) * 32) >> 4), IDESC_S, s > 0);
+                        tc_commit(&bars->s_full[sc.i % NS]);
+                        LA_ITRACE(sc.i, 1);
+                        if (sc.k == 0) LA_CTRACE(sc.n, TR_S0);
+                        sc.next_item(p);
+                        prog = true;
+                    }
+                }
+                // ---- (b) the PV cursor's item, once its scores are issued
+                if (!sc.valid || sc.i > pc.i) {
+                    const uint32_t sbuf = pc.i % NS;
+                    const uint32_t slot = pc.oslot(pc.r);
+                    const uint32_t kc = pc.kc0 + pc.j, st = kc % NKV;
+                    const uint32_t d_o = tmem + TM_O + slot * 64;
+                    if (stage == 0 && mbar_test_wait(&bars->p_full[sbuf], (pc.i / NS) & 1) &&
+                        (pc.j != 0 || mbar_test_wait(&bars->o_empty[slot], (pc.ouse(pc.r) & 1) ^ 1))) {
+                        // O_r += P V_j; P of keys 0-63 in columns 0-31, of keys 64-127 in 64-95
+                        tc_fence_after();
+                        LA_ITRACE(pc.i, 4);
+                        const uint64_t b = dv + ((st * KV_STAGE) >> 4);
+                        const uint32_t a_p = tmem + TM_S + sbuf * KC;
+#pragma unroll
+                        for (int s = 0; s < KC / 16; ++s)
+                            mma_ts(d_o, a_p + (s < 4 ? s * 8 : 64 + (s - 4) * 8), b + ((s * 2048) >> 4), IDESC_PV,
+                                   (pc.j > 0 || s > 0));
+                        ++pv_issued;
+                        LA_ITRACE(pc.i, 5);
+                        if (pc.k == 0) LA_CTRACE(pc.n, TR_PV0);
+                        if (pc.last_of_block()) LA_CTRACE(pc.n, TR_PVL);
+                        stage = 1;
+                        prog = true;
+                    }
+                    if (stage == 1) {
+                        if (!pc.last_of_chunk()) {
+                            stage = 2;
+                        } else {
+                            // KV += K_j^T V_j once the state group has copied out this block's prefix
+                            if (pc.add_state && pc.j == 0 && kvr_blk != pc.n &&
+                                mbar_test_wait(&bars->kv_read[pc.n & 1], (pc.n >> 1) & 1)) {
+                                kvr_blk = pc.n;
+                                tc_fence_after();
+                            }
+                            if (!pc.add_state || pc.j > 0 || kvr_blk == pc.n) {
+                                if (pc.add_state) {
+                                    const uint64_t a = dkt + ((st * KV_STAGE) >> 4), b = dv + ((st * KV_STAGE) >> 4);
+#pragma unroll
+                                    for (int s = 0; s < KC / 16; ++s)
+                                        mma_ss(tmem + TM_KV, a + ((s * 2048) >> 4), b + ((s * 2048) >> 4), IDESC_KV,
+                                               (pc.b > 0 || pc.j > 0 || s > 0));
+                                    if (pc.j == pc.Rb - 1) {
+                                        tc_commit(&bars->kv_ready);
+                                        LA_CTRACE(pc.n, TR_KVR);
+                                    }
+                                }
+                                tc_commit(&bars->kv_empty[st]);
+                                ++kv_released;
+                                LA_ITRACE(pc.i, 6);
+                                stage = 2;
+                                prog = true;
+                            }
+                        }
+                    }
+                    if (stage == 2) {
+                        // O_r += Q_r . bf16(KV_b) after sub-unit r's last item (every item is
+                        // the last of its sub-unit except (0,1))
+                        if (pc.k == 0 && pc.Rb == 2) {
+                            stage = 3;
+                        } else {
+                            bool ready = true;
+                            if (pc.r == 0) {
+                                if (kvr_blk != pc.n) {
+                                    if (mbar_test_wait(&bars->kv_read[pc.n & 1], (pc.n >> 1) & 1)) kvr_blk = pc.n;
+                                    else ready = false;
+                                }
+                                if (ready && !mbar_test_wait(&bars->sb_full, pc.n & 1)) ready = false;
+                            }
+                            if (ready) {
+                                tc_fence_after();
+                                const uint32_t qc = pc.q0 + pc.r, qs = qc % NQ;
+                                const uint64_t a = dq + ((qs * Q_BYTES) >> 4);
+#pragma unroll
+                                for (int s = 0; s < D / 16; ++s)
+                                    mma_ss(d_o, a + (((s >> 2) * QH_BYTES + (s & 3) * 32) >> 4),
+                                           dsb + ((s * 2048) >> 4), IDESC_C, 1);
+                                tc_commit(&bars->q_empty[qs]);
+                                ++q_released;
+                                tc_commit(&bars->o_full[slot]);
+                                if (pc.r == pc.Rb - 1) tc_commit(&bars->sb_empty);
+                                LA_CTRACE(pc.n, pc.r == 0 ? TR_C0 : TR_CL);
+                                LA_ITRACE(pc.i, 7);
+                                stage = 3;
+                                prog = true;
+                            }
+                        }
+                    }
+                    if (stage == 3) {
+                        pc.next_item(p);
+                        stage = 0;
+                    }
+                }
+                // ---- nothing ready: bounded idle time, launch-wide abort
+                if (prog) {
+                    idle = 0;
+                } else if ((++idle & 63u) == 0) {
+                    if (ab.raised()) { *ab.cta = 1; break; }
+                    const uint64_t now = globaltimer_ns();
+                    if (idle == 64) t_idle = now;
+                    else if (now - t_idle > ab.limit_ns) { ab.raise(); break; }
+                }
+            }
+            // every MMA issued by this thread has completed once `drain` fires
+            tc_commit(&bars->drain);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&bars->drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ================================================================ scores -> P
+        const int hk = warp >= 8 ? 1 : 0;                // keys 0-63 or 64-127 of the chunk
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;                  // query row of the sub-unit (TMEM lane)
+        const uint32_t lane_base = uint32_t(quad * 32) << 16;
+        bool ok = true;
+        Cursor c;
+        c.init(p);
+        while (ok && c.valid) {
+            const uint32_t sbuf = c.i % NS;
+            if (!warp_all(wait_bar(&bars->s_full[sbuf], (c.i / NS) & 1, ab))) { ok = false; break; }
+            if (m == 0 && hk == 0) LA_ITRACE(c.i, 2);
+            tc_fence_after();
+            const uint32_t ts = tmem + lane_base + TM_S + sbuf * KC + 64 * hk;
+            const int lim = UM * (c.r - c.j) + m - 64 * hk;    // key column kept when col <= lim
+            uint32_t pk[32];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a[32];
+                tmem_ld_x32(ts + 32 * hh, a);
+                tmem_wait_ld();
+                if (lim >= 63) {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int c0 = 32 * hh + 2 * q;
+                        pk[16 * hh + q] = pack_bf16x2(c0 <= lim ? __uint_as_float(a[2 * q]) : 0.f,
+                                                      c0 + 1 <= lim ? __uint_as_float(a[2 * q + 1]) : 0.f);
+                    }
+                }
+            }
+            tmem_st_x32(ts, pk);             // P of these 64 keys over the first 32 of their columns
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[sbuf]);
+            if (m == 0 && hk == 0) LA_ITRACE(c.i, 3);
+            if (m == 0 && hk == 0 && c.k == 0) LA_CTRACE(c.n, TR_P0);
+            if (m == 0 && hk == 0 && c.last_of_block()) LA_CTRACE(c.n, TR_PL);
+            c.next_item(p);
+        }
+    } else if (warp >= 12) {
+        // ================================================================ state copy-out, O epilogue
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;                  // TMEM lane: state row i / query row
+        const int wt = threadIdx.x - 384;                // 0..127
+        const uint32_t lane_base = uint32_t(quad * 32) << 16;
+        uint8_t* sb = smem + OFF_SB;
+        uint8_t* stage = smem + OFF_STG;
+        const uint64_t o_pol = policy_evict_first();     // O is never read back
+        uint32_t grp_phase = 0, kvc = 0;                 // kvc: blocks whose state was added
+        bool stored = false, ok = true;
+        Cursor c;
+        c.init(p);
+        while (ok && c.valid) {
+            // ---- KV_b (+ S0) -> bf16 operand of the inter-block product (row m, 64 columns)
+            uint32_t pk[32];
+            {
+                float x[64];
+                if (c.b == 0) {
+#pragma unroll
+                    for (int q = 0; q < 64; ++q) x[q] = 0.f;
+                } else {
+                    if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
+                    ++kvc;
+                    if (wt == 0) LA_CTRACE(c.n, TR_XR);
+                    tc_fence_after();
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t a[32];
+                        tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) x[32 * hh + q] = __uint_as_float(a[q]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->kv_read[c.n & 1]);    // the accumulator may take this block's keys
+                if (p.init) {
+                    const float4* s0 = reinterpret_cast<const float4*>(
+                        p.init + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 v = __ldg(s0 + q);
+                        x[4 * q] += v.x; x[4 * q + 1] += v.y; x[4 * q + 2] += v.z; x[4 * q + 3] += v.w;
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q) pk[q] = pack_bf16x2(x[2 * q], x[2 * q + 1]);
+            }
+            if (!warp_all(wait_bar(&bars->sb_empty, (c.n & 1) ^ 1, ab))) { ok = false; break; }
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+                *reinterpret_cast<uint4*>(sb + (m >> 3) * 1024 + (m & 7) * 128 + ((g ^ (m & 7)) << 4)) =
+                    make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+            fence_proxy_async_smem();
+            if (!(c.w == p.suppress_item && c.b == 1)) mbar_arrive(&bars->sb_full);
+            if (wt == 0) LA_CTRACE(c.n, TR_SB);
+            // ---- O epilogue of each sub-unit, in the order the issuer finishes them
+            for (int r = 0; ok && r < c.Rb; ++r) {
+                const uint32_t slot = c.oslot(r);
+                if (!warp_all(wait_bar(&bars->o_full[slot], c.ouse(r) & 1, ab))) { ok = false; break; }
+                if (wt == 0) LA_CTRACE(c.n, r == 0 ? TR_E0 : TR_EL);
+                tc_fence_after();
+                uint32_t ov[32];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a[32];
+                    tmem_ld_x32(tmem + lane_base + TM_O + slot * 64 + 32 * hh, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        ov[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->o_empty[slot]);
+                const int rows = min(UM, c.rows - UM * r);
+                if (rows == UM) {
+                    if (wt == 0 && stored) bulk_wait_read0();    // the previous store has read the staging
+                    if (!warp_all(group_sync(&bars->grp, grp_phase, ab))) { ok = false; break; }
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        *reinterpret_cast<uint4*>(stage + (m >> 3) * 1024 + (m & 7) * 128 + ((g ^ (m & 7)) << 4)) =
+                            make_uint4(ov[4 * g], ov[4 * g + 1], ov[4 * g + 2], ov[4 * g + 3]);
+                    fence_proxy_async_smem();
+                    if (!warp_all(group_sync(&bars->grp, grp_phase, ab))) { ok = false; break; }
+                    if (wt == 0) {
+                        tma_store_3d_hint(&tmO, stage, DV * c.half, c.h, c.tok0 + UM * r, o_pol);
+                        bulk_commit();
+                        stored = true;
+                        if (r == c.Rb - 1) LA_CTRACE(c.n, TR_ST);
+                    }
+                } else if (m < rows) {
+                    __nv_bfloat16* orow = p.out + ((int64_t)(c.tok0 + UM * r + m) * p.H + c.h) * D + DV * c.half;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        __stcs(reinterpret_cast<uint4*>(orow + 8 * g),
+                               make_uint4(ov[4 * g], ov[4 * g + 1], ov[4 * g + 2], ov[4 * g + 3]));
+                }
+            }
+            c.next_block(p);
+        }
+        if (wt == 0) bulk_wait0();            // every O store has landed before the CTA exits
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TM_COLS);
+    }
+}
+
+}  // namespace chain
+}  // namespace la

@@ -34,6 +34,13 @@ struct BlockEntry {
 };
 static_assert(sizeof(BlockEntry) == 32, "block table entries are 32 bytes");
 
+// One sequence of a packed batch (the on-chip-state prefill walks sequences).
+struct SeqEntry {
+    int32_t tok0;   // first token (global row in the packed [T][H][d] tensors)
+    int32_t len;    // tokens
+};
+static_assert(sizeof(SeqEntry) == 8, "sequence entries are 8 bytes");
+
 // Published-state ring slots per (sequence, head) of the single-pass prefill.
 constexpr int kStateSlots = 6;
 

@@ -17,6 +17,7 @@
 #include "simt.cuh"
 #include "decode.cuh"
 #include "fused.cuh"
+#include "chain.cuh"
 
 namespace {
 
@@ -40,11 +41,26 @@ bool supported_d(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
 bool supported_B(int B) { return B == 64 || B == 128 || B == 256; }
 bool use_tensor_cores(la_dtype dt, int d, int B) { return dt == LA_BF16 && d == 128 && (B == 128 || B == 256); }
 
+// Tensor-core prefill variants. The on-chip-state kernel gives one CTA to each
+// (sequence, head, value-column half) and so needs enough of them to fill the
+// GPU; below kChainMinItems work items the block-parallel look-back kernel
+// (one CTA per SM over (block, head) tiles) is used instead.
+enum class Path { simt, lookback, chain };
+constexpr int64_t kChainMinItems = 64;
+thread_local int t_force_path = 0;     // la_debug_set_path: 0 automatic, 1 on-chip state, 2 look-back
+
+Path prefill_path(la_dtype dt, int d, int B, int nseq, int H) {
+    if (!use_tensor_cores(dt, d, B)) return Path::simt;
+    if (t_force_path == 1) return Path::chain;
+    if (t_force_path == 2) return Path::lookback;
+    return 2 * (int64_t)nseq * H >= kChainMinItems ? Path::chain : Path::lookback;
+}
+
 // ------------------------------------------------------------------ workspace layouts
 struct Layout {
     int64_t max_blocks = 0, max_slots = 0;
     size_t off_seq_blk = 0, off_seq_slot = 0, off_table = 0, off_flags = 0, off_U = 0, off_prefix = 0,
-           off_states = 0, total = 0;
+           off_states = 0, off_seqs = 0, off_order = 0, total = 0;
     int nflag_arrays = 0;
 };
 
@@ -60,9 +76,18 @@ size_t layout_head(Layout& L, int64_t T, int nseq, int B) {
 
 Layout prefill_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt) {
     Layout L;
+    const Path path = prefill_path(dt, d, B, nseq, H);
+    if (path == Path::chain) {
+        // Control | sequence table | processing order
+        size_t off = sizeof(Control);
+        L.off_seqs = off;  off = align_up(off + sizeof(la::SeqEntry) * (size_t)nseq, 256);
+        L.off_order = off; off = align_up(off + sizeof(int32_t) * (size_t)nseq, 256);
+        L.total = off;
+        return L;
+    }
     size_t off = layout_head(L, T, nseq, B);
     const size_t dd = (size_t)d * d;
-    if (use_tensor_cores(dt, d, B)) {
+    if (path == Path::lookback) {
         // single pass: per-block flags (aggregate, inclusive, look-back done) and a
         // ring of kStateSlots published states per (sequence, head); a sequence with
         // n blocks uses min(n - 1, kStateSlots) slots.
@@ -302,6 +327,54 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const Control* ctrl = reinterpret_cast<const Control*>(ws);
+    const Path path = prefill_path(dtype, d, B, num_seqs, heads);
+
+    if (path == Path::chain) {
+        la::SeqEntry* seqs = reinterpret_cast<la::SeqEntry*>(ws + L.off_seqs);
+        int32_t* order = reinterpret_cast<int32_t*>(ws + L.off_order);
+        la::seq_table_kernel<<<1, 1024, 0, st>>>(cu_seqlens, num_seqs, total_tokens, seqs, order,
+                                                 reinterpret_cast<Control*>(ws));
+        note_launch();
+        if ((s = cuda_check()) != LA_OK) return s;
+        CUtensorMap tq, tk, tv, to;
+        if (!map_tokens(&tq, q, total_tokens, heads, d, la::chain::UM) ||
+            !map_tokens(&tk, k, total_tokens, heads, d, la::chain::KC) ||
+            !map_tokens(&tv, v, total_tokens, heads, d, la::chain::KC) ||
+            !map_tokens(&to, o, total_tokens, heads, d, la::chain::UM))
+            return LA_ERR_CUDA;
+        la::chain::Params prm;
+        prm.out = static_cast<__nv_bfloat16*>(o);
+        prm.seqs = seqs;
+        prm.order = order;
+        prm.ctrl = ctrl;
+        prm.init = init_state;
+        prm.H = heads;
+        prm.B = B;
+        prm.nseq = num_seqs;
+        prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
+        prm.suppress_item = t_suppress_tile;
+        const int64_t items = 2 * (int64_t)num_seqs * heads;
+        const int sms = num_sms();
+        if (sms <= 0) return LA_ERR_CUDA;
+        const unsigned grid = (unsigned)(items < sms ? items : sms);
+        const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
+#ifdef LA_CHAIN_ITEM_TRACE
+        const size_t reserved = 4096 * 8 * sizeof(uint64_t);   // per-item stamps of CTA 0 after the block table
+#else
+        const size_t reserved = 0;
+#endif
+        prm.trace = (t_trace && t_trace_bytes >= per_block + reserved) ? t_trace : nullptr;
+        prm.trace_blocks = prm.trace ? (int)std::min<size_t>((t_trace_bytes - reserved) / per_block, 1 << 30) : 0;
+        if (cudaFuncSetAttribute(la::chain::prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)la::chain::SMEM_BYTES) != cudaSuccess)
+            return LA_ERR_CUDA;
+        MainKernelTimer timer(st);
+        la::chain::prefill_chain_kernel<<<grid, la::chain::NTHREADS, la::chain::SMEM_BYTES, st>>>(tq, tk, tv, to,
+                                                                                                   prm);
+        note_launch();
+        return cuda_check();
+    }
+
     const int32_t* seq_blk = reinterpret_cast<const int32_t*>(ws + L.off_seq_blk);
     const BlockEntry* table = reinterpret_cast<const BlockEntry*>(ws + L.off_table);
     float* U = reinterpret_cast<float*>(ws + L.off_U);
@@ -309,7 +382,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
 
     if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, B, heads, L, ws, st)) != LA_OK) return s;
 
-    if (use_tensor_cores(dtype, d, B)) {
+    if (path == Path::lookback) {
         CUtensorMap tq, tk, tv, to;
         if (!map_tokens(&tq, q, total_tokens, heads, d, 128) || !map_tokens(&tk, k, total_tokens, heads, d, 64) ||
             !map_tokens(&tv, v, total_tokens, heads, d, 64) || !map_tokens(&to, o, total_tokens, heads, d, 128))
@@ -422,6 +495,12 @@ la_status la_debug_set_fault(long long suppress_tile, uint64_t wait_ns) {
 }
 
 uint64_t la_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+la_status la_debug_set_path(int path) {
+    if (path < 0 || path > 2) return LA_ERR_INVALID_ARGUMENT;
+    t_force_path = path;
+    return LA_OK;
+}
 
 la_status la_debug_set_trace(void* device_buffer, size_t bytes) {
     if ((device_buffer == nullptr) != (bytes == 0)) return LA_ERR_INVALID_ARGUMENT;

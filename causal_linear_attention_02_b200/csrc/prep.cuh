@@ -129,6 +129,69 @@ __global__ void fill_block_table_kernel(const int32_t* __restrict__ cu, int nseq
         for (int h = 0; h < H; ++h) flags[((int64_t)a * max_blocks + g) * H + h] = 0;
 }
 
+// Sequences longest first, so that work items of equal cost start together
+// and the longest chains start first. Sorted by counting when nseq is at
+// most kSortMax (ties keep their input order), else left in input order.
+constexpr int kSortMax = 2048;
+
+// Validates cu_seqlens like seq_blocks_kernel and writes, per sequence,
+// its first token and length (seqs) and the processing order (order,
+// longest first). One CTA of 1024 threads. cu == nullptr means one
+// sequence of T tokens.
+__global__ void __launch_bounds__(1024) seq_table_kernel(const int32_t* __restrict__ cu, int nseq, int64_t T,
+                                                         SeqEntry* __restrict__ seqs,
+                                                         int32_t* __restrict__ order,
+                                                         Control* __restrict__ ctrl) {
+    __shared__ int32_t lens[kSortMax];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    if (cu != nullptr) {
+        for (int s = tid; s < nseq; s += blockDim.x)
+            if (cu[s + 1] < cu[s]) bad = 1;
+        if (tid == 0 && (cu[0] != 0 || (int64_t)cu[nseq] != T)) bad = 1;
+    }
+    __syncthreads();
+    if (bad) {
+        if (tid == 0) {
+            ctrl->nblocks = 0;
+            ctrl->ok = 0;
+            ctrl->nslots = 0;
+            ctrl->abort = 0;
+            record_status(LA_ERR_BAD_SEQLENS);
+        }
+        return;
+    }
+    const bool sort = nseq <= kSortMax;
+    for (int s = tid; s < nseq; s += blockDim.x) {
+        SeqEntry e;
+        e.tok0 = cu ? cu[s] : 0;
+        e.len = cu ? cu[s + 1] - cu[s] : (int32_t)T;
+        seqs[s] = e;
+        if (sort) lens[s] = e.len;
+        else order[s] = s;
+    }
+    __syncthreads();
+    if (sort) {
+        for (int s = tid; s < nseq; s += blockDim.x) {
+            const int32_t l = lens[s];
+            int rank = 0;
+            for (int t = 0; t < nseq; ++t) {
+                const int32_t lt = lens[t];
+                rank += (lt > l) || (lt == l && t < s);
+            }
+            order[rank] = s;
+        }
+    }
+    if (tid == 0) {
+        ctrl->nblocks = 0;
+        ctrl->ok = 1;
+        ctrl->nslots = 0;
+        ctrl->abort = 0;
+    }
+}
+
 // Exclusive prefix over the blocks of every (sequence, head) chain:
 //   prefix[g] = S0 + sum_{blocks c of the same sequence before g} U[c]
 // and, optionally, the chain total S0 + sum_all U into state_out.

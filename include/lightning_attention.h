@@ -67,8 +67,12 @@ typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
 /*
  * Supported shapes: heads >= 1, d a multiple of 16 with 16 <= d <= 128,
  * B in {64, 128, 256}, total_tokens >= 0, num_seqs >= 1.
- * bf16 with d = 128 and B in {128, 256} runs on the tcgen05 tensor-core path;
- * every other supported combination runs on the CUDA-core (SIMT) path.
+ * bf16 with d = 128 and B in {128, 256} runs on a tcgen05 tensor-core kernel:
+ * the on-chip-state kernel (one CTA per sequence, head and half of the value
+ * columns, the running state kept in tensor memory) when num_seqs * heads * 2
+ * >= 64, else the block-parallel kernel (block prefixes by a single-pass
+ * decoupled look-back scan); la_debug_set_path overrides the choice. Every
+ * other supported combination runs on the CUDA-core (SIMT) path.
  */
 
 /* Bytes of device workspace la_prefill needs for these sizes (0 if unsupported). */
@@ -160,29 +164,56 @@ la_status la_set_kernel_timer(void* start_event, void* stop_event);
 
 /*
  * Test hook (no counterpart on the pages). For the following la_prefill calls
- * made by this host thread on the tensor-core path: tile `suppress_tile` (index
- * block * heads + head over the blocks of all sequences, -1 = none) publishes
- * no state, and every device-side wait gives up after `wait_ns` nanoseconds
- * (0 = the default of 4 s). A suppressed tile makes its successors' bounded
- * waits expire: the launch then ends by itself, la_get_device_status reports
- * LA_ERR_TIMEOUT and the CUDA context stays usable. Call with (-1, 0) to reset.
+ * made by this host thread on the tensor-core path, every device-side wait
+ * gives up after `wait_ns` nanoseconds (0 = the default of 4 s), and
+ * `suppress_tile` (-1 = none) names a unit of work that withholds one hand-off:
+ *  - block-parallel kernel: tile block * heads + head (over the blocks of all
+ *    sequences) publishes no state, so its successors' look-backs wait;
+ *  - on-chip-state kernel: work item w (2 * (rank * heads + head) + half, rank
+ *    = position of the sequence in longest-first order) never hands the prefix
+ *    of its second block to the tensor cores.
+ * The bounded waits then expire: the launch ends by itself,
+ * la_get_device_status reports LA_ERR_TIMEOUT and the CUDA context stays
+ * usable. Call with (-1, 0) to reset.
  */
 la_status la_debug_set_fault(long long suppress_tile, uint64_t wait_ns);
 
 /*
  * Tracing (no counterpart on the pages). While a buffer is set, every
- * la_prefill call made by this host thread on the tensor-core path records,
- * for each tile (block * heads + head over the blocks of all sequences), 48
- * uint64 globaltimer stamps (ns) of its phases into `device_buffer`: [0] first
- * Q tile ready, [1] chunk MMAs issued, [2] prefix available, [3]/[4] look-back
- * start/end, [5] prefix written, [6] inclusive state published, [7] output
- * stored, [8] aggregate published, [9] last P written, [10..47] finer steps of
- * the worker roles; unused slots are left as they were. The buffer must hold
- * max_tiles * 384 bytes, max_tiles =
- * (ceil(total_tokens / B) + num_seqs) * heads, or the call records nothing.
+ * la_prefill call made by this host thread on a tensor-core path records
+ * phase stamps into `device_buffer`; unused slots are left as they were.
+ *  - Block-parallel kernel: for each tile (block * heads + head over the
+ *    blocks of all sequences), 48 uint64 globaltimer stamps (ns): [0] first Q
+ *    tile ready, [1] chunk MMAs issued, [2] prefix available, [3]/[4]
+ *    look-back start/end, [5] prefix written, [6] inclusive state published,
+ *    [7] output stored, [8] aggregate published, [9] last P written, [10..47]
+ *    finer steps of the worker roles. The buffer must hold max_tiles * 384
+ *    bytes, max_tiles = (ceil(total_tokens / B) + num_seqs) * heads, or the
+ *    call records nothing.
+ *  - On-chip-state kernel: for each CTA and each block it processes (in
+ *    order), 16 uint64 SM-clock stamps (clock64) of its roles: [0] Q load,
+ *    [1]/[2] first/last K/V load, [3] first score MMA, [4] first PV MMA,
+ *    [5]/[7] inter-block MMAs, [6] last state MMA, [8]/[9] first/last P,
+ *    [10] state ready, [11] prefix handed over, [12]/[13] output accumulators
+ *    complete, [14] last output store, [15] last PV MMA. The buffer holds
+ *    grid * blocks_per_cta * 128 bytes for as many blocks per CTA as fit
+ *    (grid = min(2 * num_seqs * heads, SM count)).
  * NULL, 0 stops tracing.
  */
 la_status la_debug_set_trace(void* device_buffer, size_t bytes);
+
+/*
+ * Test hook (no counterpart on the pages). Chooses, for the following calls
+ * made by this host thread, which tensor-core prefill kernel la_prefill,
+ * la_prefill_noalloc and la_prefill_workspace_size use for bf16, d = 128,
+ * B in {128, 256}: 0 = automatic (the default), 1 = the on-chip-state kernel
+ * (one CTA per sequence, head and half of the value columns, blocks walked in
+ * order), 2 = the block-parallel kernel (one CTA per SM over (block, head)
+ * tiles, block prefixes by a single-pass decoupled look-back scan). Automatic
+ * picks the on-chip-state kernel when num_seqs * heads * 2 >= 64. Results are
+ * the same up to rounding. Returns LA_ERR_INVALID_ARGUMENT for any other value.
+ */
+la_status la_debug_set_path(int path);
 
 /*
  * Number of kernels this library has launched, from every host thread, since

@@ -60,6 +60,20 @@ def cu_of(lengths):
     return wl.cu_seqlens(lengths, device=DEV)
 
 
+# The two tensor-core prefill kernels (la_debug_set_path): 1 = on-chip state,
+# one CTA per (sequence, head, value-column half); 2 = block-parallel with a
+# decoupled look-back scan. Tests taking `tc_path` run under both.
+@pytest.fixture(params=[1, 2], ids=["onchip", "lookback"])
+def tc_path(request):
+    assert la.la_debug_set_path(request.param) == 0
+    yield request.param
+    la.la_debug_set_path(0)
+
+
+def force_path(path):
+    assert la.la_debug_set_path(path) == 0
+
+
 # ------------------------------------------------------------------ decode
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
 @pytest.mark.parametrize("d", [16, 48, 64, 128])
@@ -89,7 +103,7 @@ def test_prefill_fp32_small_workload():
 # ------------------------------------------------------------------ prefill, tensor-core path
 @pytest.mark.parametrize("B", [128, 256])
 @pytest.mark.parametrize("T", [1, 37, 128, 255, 256, 257, 1000, 1500])
-def test_prefill_tc_random(B, T):
+def test_prefill_tc_random(B, T, tc_path):
     H, d = 3, 128
     q, k, v = inputs(T, H, d, torch.bfloat16, seed=T * 7 + B)
     o = la.prefill(q, k, v, B=B)
@@ -99,7 +113,7 @@ def test_prefill_tc_random(B, T):
 
 
 @pytest.mark.parametrize("B,T", [(256, 512), (128, 384), (256, 300), (128, 200)])
-def test_prefill_tc_integer_exact(B, T):
+def test_prefill_tc_integer_exact(B, T, tc_path):
     """{-1,0,1} inputs: scores, P, every prefix entry and O are exact integers in
     bf16/fp32, so the result must equal the oracle's rounded to bf16 bit for bit."""
     H, d = 2, 128
@@ -115,7 +129,7 @@ def test_prefill_tc_integer_exact(B, T):
 
 
 @pytest.mark.parametrize("B", [128, 256])
-def test_prefill_tc_varlen(B):
+def test_prefill_tc_varlen(B, tc_path):
     lengths = [1, 255, 256, 0, 257, 700, 64, 513, 128]
     H, d = 2, 128
     T = sum(lengths)
@@ -129,7 +143,7 @@ def test_prefill_tc_varlen(B):
 
 @pytest.mark.parametrize("dtype,d,B", [(torch.bfloat16, 128, 256), (torch.bfloat16, 128, 128),
                                        (torch.float32, 64, 64), (torch.bfloat16, 64, 128)])
-def test_prefill_init_state(dtype, d, B):
+def test_prefill_init_state(dtype, d, B, tc_path):
     lengths = [300, 1, 520]
     H = 2
     T = sum(lengths)
@@ -240,13 +254,17 @@ def test_bad_seqlens_reported_on_device():
 ])
 def test_prefill_single_pass_chains(T, H, B):
     q, k, v = inputs(T, H, 128, torch.bfloat16, seed=T + H + B)
-    o = la.prefill(q, k, v, B=B)
+    force_path(2)
+    try:
+        o = la.prefill(q, k, v, B=B)
+    finally:
+        force_path(0)
     status_ok()
     ref = oracle.recurrent(f64(q), f64(k), f64(v))
     assert_close(f64(o), ref, 1e-2, f"single pass T={T} H={H} B={B}")
 
 
-def test_prefill_many_sequences_share_slots():
+def test_prefill_many_sequences_share_slots(tc_path):
     """Many packed sequences (some shorter than one block, some spanning many
     slot-ring generations) in one launch."""
     lengths = wl.varlen_lengths(40, 1, 3000, seed=8)
@@ -269,6 +287,7 @@ def test_lost_publication_ends_in_timeout_not_hang():
     q, k, v = inputs(T, H, 128, torch.bfloat16, seed=5150)
     suppress = 5 * H + 1                      # block 5 of head 1
     assert la.la_debug_set_fault(suppress, 200_000_000) == 0
+    force_path(2)
     try:
         t0 = time.time()
         la.prefill(q, k, v, B=B)
@@ -276,8 +295,56 @@ def test_lost_publication_ends_in_timeout_not_hang():
         elapsed = time.time() - t0
     finally:
         la.la_debug_set_fault(-1, 0)
+        force_path(0)
     assert st == 6, f"expected LA_ERR_TIMEOUT, got {la.STATUS.get(st, st)}"
     assert elapsed < 30, f"timed-out launch took {elapsed:.1f}s"
     o = la.prefill(q, k, v, B=B)
     status_ok()
+    assert_close(f64(o), oracle.recurrent(f64(q), f64(k), f64(v)), 1e-2, "run after a timeout")
+
+
+# ------------------------------------------------------------------ on-chip-state scheduling corners
+@pytest.mark.parametrize("lengths,H,B", [
+    ([8192], 2, 256),                       # 4 work items, 32 blocks each
+    ([3000] * 3, 64, 256),                  # 384 work items: every CTA takes two or three
+    ([4096], 148, 128),                     # 296 work items of equal length
+    ([20001], 7, 128),                      # ragged tail, odd head count
+    ([1, 2, 255, 256, 257, 4000, 0, 129, 1024, 3], 9, 256),   # mixed lengths, longest first
+])
+def test_prefill_onchip_scheduling(lengths, H, B):
+    T = sum(lengths)
+    q, k, v = inputs(T, H, 128, torch.bfloat16, seed=T + H + B + 1)
+    cu = cu_of(lengths)
+    force_path(1)
+    try:
+        o = la.prefill(q, k, v, cu, B=B)
+    finally:
+        force_path(0)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy())
+    assert_close(f64(o), ref, 1e-2, f"on-chip state lengths={lengths[:4]} H={H} B={B}")
+
+
+def test_withheld_prefix_ends_in_timeout_not_hang():
+    """On the on-chip-state kernel, a work item whose state group never hands
+    over a block prefix makes the tensor-core issuer's bounded wait expire:
+    the launch ends by itself with LA_ERR_TIMEOUT and the next call is right."""
+    T, H, B = 4096, 4, 256
+    q, k, v = inputs(T, H, 128, torch.bfloat16, seed=5151)
+    assert la.la_debug_set_fault(3, 200_000_000) == 0
+    force_path(1)
+    try:
+        t0 = time.time()
+        la.prefill(q, k, v, B=B)
+        st = la.device_status()
+        elapsed = time.time() - t0
+    finally:
+        la.la_debug_set_fault(-1, 0)
+    try:
+        assert st == 6, f"expected LA_ERR_TIMEOUT, got {la.STATUS.get(st, st)}"
+        assert elapsed < 30, f"timed-out launch took {elapsed:.1f}s"
+        o = la.prefill(q, k, v, B=B)
+        status_ok()
+    finally:
+        force_path(0)
     assert_close(f64(o), oracle.recurrent(f64(q), f64(k), f64(v)), 1e-2, "run after a timeout")
