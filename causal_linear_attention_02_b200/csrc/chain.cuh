@@ -19,22 +19,33 @@
 //
 // A block of B rows is R = B/128 sub-units of 128 query rows; keys arrive in
 // chunks of 128 (chunk j = keys 128j .. 128j+127 of the block). Items
-// (chunk j, sub-unit r) with j <= r, in the order (0,1), (0,0), (1,1):
+// (chunk j, sub-unit r) with j <= r, in the order (0,0), (0,1), (1,1):
+//   inter   O_r  = Q_r . bf16(KV_b)     (M=128, N=64,  K=128)  before sub-unit r's first PV
 //   scores  S = Q_r K_j^T               (M=128, N=128, K=128)  -> TMEM
 //   P       = bf16(mask(S)), written back into TMEM (two warpgroups, one per
 //             64-key half of the chunk)
 //   PV      O_r += P V_j                (M=128, N=64,  K=128)  A from TMEM
-//   state   KV += K_j^T V_j             (M=128, N=64,  K=128)  after the chunk's last item
-//   inter   O_r += Q_r . bf16(KV_b)     (M=128, N=64,  K=128)  after sub-unit r's last item
-// Roles (512 threads):
-//   warp 0 (lane 0)  TMA producer of K / V chunks (+ L2 prefetch of the next block)
-//   warp 1 (lane 0)  tcgen05 issuer: a non-blocking event loop; score MMAs run
-//                    ahead of the PV cursor as far as the rings allow
-//   warp 2 (lane 0)  TMA producer of Q sub-units (+ L2 prefetch of the next block)
+//   state   KV += K_j^T V_j             (M=128, N=64,  K=128)  as soon as chunk j is loaded
+// This order retires shared-memory stages in ring order and early. K, V and
+// Q have rings of their own, sized by how long a stage is held: a K chunk
+// until its scores and state MMA (3 stages of 32 KB), a V chunk until its PVs
+// and state MMA (2 of 16 KB), a Q sub-unit until its scores and inter-block
+// MMA (2 of 32 KB); together they keep about one block of loads in flight.
+// Roles (640 threads):
+//   warp 0 (lane 0)  TMA producer of K and V chunks, warp 2 (lane 0) of Q
+//                    sub-units
+//   warp 1 (lane 0)  tcgen05 issuer A: score MMAs and state MMAs (chunk by
+//                    chunk as they land), a non-blocking event loop
+//   warp 3 (lane 0)  tcgen05 issuer B: inter-block and PV MMAs, in item order
+//                    Two issuing threads keep the tensor pipe fed while either
+//                    one waits or does its bookkeeping; their MMAs are not
+//                    ordered with each other, so every hand-off between them
+//                    goes through an mbarrier (a score buffer is rewritten only
+//                    after the PV that read it has completed).
 //   warps 4-7, 8-11  scores -> P, keys 0-63 and 64-127 of every item
-//   warps 12-15      state copy-out (TMEM fp32 -> bf16 shared operand) and O
-//                    epilogue (TMEM -> bf16 -> swizzled staging -> TMA store;
-//                    a ragged last sub-unit by masked direct stores)
+//   warps 12-15      state copy-out: TMEM fp32 (+ S0) -> bf16 shared operand
+//   warps 16-19      O epilogue: TMEM -> bf16 -> swizzled staging -> TMA store (a
+//                    ragged last sub-unit of a sequence by masked direct stores)
 // Every wait is bounded (globaltimer); on expiry the CTA records
 // LA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
 #pragma once
@@ -52,23 +63,38 @@ constexpr int D = 128;                     // head dim (d_k = d_v)
 constexpr int DV = 64;                     // value columns per work item
 constexpr int UM = 128;                    // rows per sub-unit (MMA M)
 constexpr int KC = 128;                    // keys per chunk
-constexpr int NQ = 3;                      // Q sub-unit stages
-constexpr int NKV = 2;                     // K/V chunk stages
+#ifndef LA_CHAIN_NQ
+#define LA_CHAIN_NQ 2
+#endif
+#ifndef LA_CHAIN_NK
+#define LA_CHAIN_NK 3
+#endif
+#ifndef LA_CHAIN_NV
+#define LA_CHAIN_NV 2
+#endif
+constexpr int NQ = LA_CHAIN_NQ;            // Q sub-unit stages
+constexpr int NK = LA_CHAIN_NK;            // K chunk stages
+constexpr int NV = LA_CHAIN_NV;            // V chunk stages
 constexpr int NS = 2;                      // score buffers in TMEM
-constexpr int NTHREADS = 512;
+constexpr int NTHREADS = 640;
 
 constexpr uint32_t QH_BYTES = UM * 64 * 2;       // 16 KB: 128 rows x 64 columns
 constexpr uint32_t Q_BYTES = 2 * QH_BYTES;       // 32 KB
 constexpr uint32_t KH_BYTES = KC * 64 * 2;       // 16 KB: 128 keys x 64 columns
 constexpr uint32_t K_BYTES = 2 * KH_BYTES;       // 32 KB
 constexpr uint32_t V_BYTES = KC * DV * 2;        // 16 KB
-constexpr uint32_t KV_STAGE = K_BYTES + V_BYTES; // 48 KB
 constexpr uint32_t SB_BYTES = D * DV * 2;        // 16 KB: bf16 KV_b, 128 rows x 64 columns
-constexpr uint32_t STG_BYTES = UM * DV * 2;      // 16 KB: O staging, 128 rows x 64 columns
+#ifndef LA_CHAIN_DIRECT_O
+#define LA_CHAIN_DIRECT_O 1
+#endif
+// O staging for the TMA store, 128 rows x 64 columns (16 KB), unless O rows are
+// stored directly from registers.
+constexpr uint32_t STG_BYTES = LA_CHAIN_DIRECT_O ? 0 : UM * DV * 2;
 
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_KV = OFF_Q + NQ * Q_BYTES;
-constexpr uint32_t OFF_SB = OFF_KV + NKV * KV_STAGE;
+constexpr uint32_t OFF_K = OFF_Q + NQ * Q_BYTES;
+constexpr uint32_t OFF_V = OFF_K + NK * K_BYTES;
+constexpr uint32_t OFF_SB = OFF_V + NV * V_BYTES;
 constexpr uint32_t OFF_STG = OFF_SB + SB_BYTES;
 constexpr uint32_t OFF_BAR = OFF_STG + STG_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;   // + barriers + 1 KB alignment slack
@@ -85,14 +111,15 @@ constexpr uint32_t IDESC_C = idesc_bf16(UM, DV, false, true);    // Q (K-major) 
 
 struct Bars {
     uint64_t q_full[NQ], q_empty[NQ];
-    uint64_t kv_full[NKV], kv_empty[NKV];
-    uint64_t s_full[NS], p_full[NS];
+    uint64_t k_full[NK], k_empty[NK];     // k_empty: two arrivals, the chunk's scores and its state MMA
+    uint64_t v_full[NV], v_empty[NV];     // v_empty: two arrivals, the chunk's PVs and its state MMA
+    uint64_t s_full[NS], p_full[NS], s_free[NS];
     uint64_t o_full[3], o_empty[3];
     uint64_t kv_ready;        // issuer -> state group: KV accumulator holds the next block's prefix
-    uint64_t kv_read[2];      // state group -> issuer: accumulator read for block n (n & 1)
+    uint64_t kv_read[4];      // state group -> issuer: accumulator read for block n (n % 4)
     uint64_t sb_full, sb_empty;
-    uint64_t grp;             // bounded barrier of the state / epilogue group
-    uint64_t drain;
+    uint64_t grp;             // bounded barrier of the epilogue group
+    uint64_t drain, drain_b;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -128,20 +155,29 @@ enum TraceEvent {
     TR_SB = 11,        // state group: bf16 prefix handed over
     TR_E0 = 12,        // state group: first sub-unit accumulator complete
     TR_EL = 13,        // state group: last sub-unit accumulator complete
-    TR_ST = 14,        // state group: last O store issued
+    TR_ST = 14,        // epilogue group: last O store of the block issued
     TR_PVL = 15,       // issuer: last PV MMA issued
     kTraceEvents = 16
 };
-// Per-item stamps of CTA 0 (compile-time option LA_CHAIN_ITEM_TRACE): eight
-// clock64 values per item after the block table in the trace buffer.
+// Per-item stamps of CTA 0 (compile-time option LA_CHAIN_ITEM_TRACE): sixteen
+// clock64 values per item after the block table in the trace buffer; LA_ITRACE1
+// records only the first time (for conditions polled by the issuer).
 #ifdef LA_CHAIN_ITEM_TRACE
 #define LA_ITRACE(i, ev)                                                                                    \
     do {                                                                                                    \
-        if (p.trace && blockIdx.x == 0 && (int)(i) < 4096)                                                  \
-            p.trace[(int64_t)gridDim.x * p.trace_blocks * kTraceEvents + (int64_t)(i) * 8 + (ev)] = clock64(); \
+        if (p.trace && blockIdx.x == 0 && (int)(i) < 2048)                                                  \
+            p.trace[(int64_t)gridDim.x * p.trace_blocks * kTraceEvents + (int64_t)(i) * 16 + (ev)] = clock64(); \
+    } while (0)
+#define LA_ITRACE1(i, ev)                                                                                   \
+    do {                                                                                                    \
+        if (p.trace && blockIdx.x == 0 && (int)(i) < 2048) {                                                \
+            uint64_t* q_ = p.trace + (int64_t)gridDim.x * p.trace_blocks * kTraceEvents + (int64_t)(i) * 16 + (ev); \
+            if (*q_ == 0) *q_ = clock64();                                                                  \
+        }                                                                                                   \
     } while (0)
 #else
 #define LA_ITRACE(i, ev) do {} while (0)
+#define LA_ITRACE1(i, ev) do {} while (0)
 #endif
 #define LA_CTRACE(n, ev)                                                                                   \
     do {                                                                                                   \
@@ -153,7 +189,7 @@ enum TraceEvent {
 // with the running counters that index the rings: n (blocks), q0 (Q
 // sub-units), kc0 (K/V chunks), o0 (uses of O slot 0) at the current block,
 // and i (items). A block has Rb = ceil(rows / 128) sub-units and as many
-// 128-key chunks; its items are (0,1), (0,0), (1,1) when Rb = 2 and (0,0)
+// 128-key chunks; its items are (0,0), (0,1), (1,1) when Rb = 2 and (0,0)
 // when Rb = 1.
 struct Cursor {
     int64_t w, nitems;
@@ -170,7 +206,7 @@ struct Cursor {
     __device__ __forceinline__ void set_item() {
         if (Rb == 2) {
             j = k == 2 ? 1 : 0;
-            r = k == 1 ? 0 : 1;
+            r = k == 0 ? 0 : 1;
         } else {
             j = 0;
             r = 0;
@@ -231,8 +267,10 @@ struct Cursor {
         next_block(p);
     }
     // item properties
-    __device__ __forceinline__ bool first_of_chunk() const { return k != 1; }     // (0,1) or (0,0) alone, (1,1)
-    __device__ __forceinline__ bool last_of_chunk() const { return k != 0 || Rb == 1; }
+    __device__ __forceinline__ bool first_of_chunk() const { return k != 1; }     // (0,0), (1,1)
+    __device__ __forceinline__ bool last_of_chunk() const { return k != 0 || Rb == 1; }   // (0,1), (1,1)
+    __device__ __forceinline__ bool first_of_sub() const { return j == 0; }       // (0,0), (0,1)
+    __device__ __forceinline__ bool last_of_sub() const { return k != 1 || Rb == 1; }     // (0,0), (1,1)
     __device__ __forceinline__ bool last_of_block() const { return k == (Rb == 2 ? 2 : 0); }
     // O slot of sub-unit rr: the sub-unit that finishes last alternates between
     // slots 1 and 2 from block to block; sub-unit 0 of a two-sub-unit block
@@ -252,17 +290,22 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const Abort ab{&bars->abort_flag, const_cast<volatile int*>(&p.ctrl->abort), p.wait_ns};
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NQ; ++i) { mbar_init(&bars->q_full[i], 1); mbar_init(&bars->q_empty[i], 1); }
-        for (int i = 0; i < NKV; ++i) { mbar_init(&bars->kv_full[i], 1); mbar_init(&bars->kv_empty[i], 1); }
-        for (int i = 0; i < NS; ++i) { mbar_init(&bars->s_full[i], 1); mbar_init(&bars->p_full[i], 256); }
+        for (int i = 0; i < NQ; ++i) { mbar_init(&bars->q_full[i], 1); mbar_init(&bars->q_empty[i], 2); }
+        for (int i = 0; i < NK; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 2); }
+        for (int i = 0; i < NV; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 2); }
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 256);
+            mbar_init(&bars->s_free[i], 1);
+        }
         for (int i = 0; i < 3; ++i) { mbar_init(&bars->o_full[i], 1); mbar_init(&bars->o_empty[i], 128); }
         mbar_init(&bars->kv_ready, 1);
-        mbar_init(&bars->kv_read[0], 128);
-        mbar_init(&bars->kv_read[1], 128);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars->kv_read[i], 128);
         mbar_init(&bars->sb_full, 128);
         mbar_init(&bars->sb_empty, 1);
         mbar_init(&bars->grp, 128);
         mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain_b, 1);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -285,46 +328,34 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint64_t once = policy_evict_first();      // V: read by this CTA only
             Cursor c;
             c.init(p);
-            uint32_t issued = 0;                              // loads issued (ring index)
+            uint32_t k_issued = 0, v_issued = 0, q_issued = 0;   // loads issued (ring indices)
             bool ok = true;
             while (ok && c.valid) {
-                // the next block's tiles into L2 while this block's are loaded
-                Cursor nx = c;
-                nx.next_block(p);
-                if (nx.valid) {
-                    for (int r = 0; r < nx.Rb; ++r) {
-                        const int t = nx.tok0 + UM * r;
-                        if (kv_role) {
-                            tma_prefetch_l2_3d(&tmK, 0, nx.h, t);
-                            tma_prefetch_l2_3d(&tmK, 64, nx.h, t);
-                            tma_prefetch_l2_3d(&tmV, DV * nx.half, nx.h, t);
-                        } else {
-                            tma_prefetch_l2_3d(&tmQ, 0, nx.h, t);
-                            tma_prefetch_l2_3d(&tmQ, 64, nx.h, t);
-                        }
-                    }
-                }
-                for (int r = 0; r < c.Rb; ++r) {      // sub-unit r's Q rows; chunk r's keys
+                for (int r = 0; ok && r < c.Rb; ++r) {      // chunk r's keys / sub-unit r's query rows
                     const int t = c.tok0 + UM * r;
                     if (kv_role) {
-                        const uint32_t kc = c.kc0 + r, st = kc % NKV;
-                        if (!wait_bar(&bars->kv_empty[st], ((kc / NKV) & 1) ^ 1, ab)) { ok = false; break; }
-                        uint8_t* kd = smem + OFF_KV + st * KV_STAGE;
-                        mbar_expect_tx(&bars->kv_full[st], KV_STAGE);
-                        tma_load_3d(kd, &tmK, &bars->kv_full[st], 0, c.h, t);
-                        tma_load_3d(kd + KH_BYTES, &tmK, &bars->kv_full[st], 64, c.h, t);
-                        tma_load_3d_hint(kd + K_BYTES, &tmV, &bars->kv_full[st], DV * c.half, c.h, t, once);
-                        issued = kc + 1;
+                        const uint32_t kc = c.kc0 + r;
+                        if (!wait_bar(&bars->k_empty[kc % NK], ((kc / NK) & 1) ^ 1, ab)) { ok = false; break; }
+                        uint8_t* kd = smem + OFF_K + (kc % NK) * K_BYTES;
+                        mbar_expect_tx(&bars->k_full[kc % NK], K_BYTES);
+                        tma_load_3d(kd, &tmK, &bars->k_full[kc % NK], 0, c.h, t);
+                        tma_load_3d(kd + KH_BYTES, &tmK, &bars->k_full[kc % NK], 64, c.h, t);
+                        k_issued = kc + 1;
                         if (r == 0) LA_CTRACE(c.n, TR_KV0);
+                        if (!wait_bar(&bars->v_empty[kc % NV], ((kc / NV) & 1) ^ 1, ab)) { ok = false; break; }
+                        mbar_expect_tx(&bars->v_full[kc % NV], V_BYTES);
+                        tma_load_3d_hint(smem + OFF_V + (kc % NV) * V_BYTES, &tmV, &bars->v_full[kc % NV],
+                                         DV * c.half, c.h, t, once);
+                        v_issued = kc + 1;
                         if (r == c.Rb - 1) LA_CTRACE(c.n, TR_KVL);
                     } else {
-                        const uint32_t qc = c.q0 + r, qs = qc % NQ;
-                        if (!wait_bar(&bars->q_empty[qs], ((qc / NQ) & 1) ^ 1, ab)) { ok = false; break; }
-                        uint8_t* qd = smem + OFF_Q + qs * Q_BYTES;
-                        mbar_expect_tx(&bars->q_full[qs], Q_BYTES);
-                        tma_load_3d(qd, &tmQ, &bars->q_full[qs], 0, c.h, t);
-                        tma_load_3d(qd + QH_BYTES, &tmQ, &bars->q_full[qs], 64, c.h, t);
-                        issued = qc + 1;
+                        const uint32_t qc = c.q0 + r;
+                        if (!wait_bar(&bars->q_empty[qc % NQ], ((qc / NQ) & 1) ^ 1, ab)) { ok = false; break; }
+                        uint8_t* qd = smem + OFF_Q + (qc % NQ) * Q_BYTES;
+                        mbar_expect_tx(&bars->q_full[qc % NQ], Q_BYTES);
+                        tma_load_3d(qd, &tmQ, &bars->q_full[qc % NQ], 0, c.h, t);
+                        tma_load_3d(qd + QH_BYTES, &tmQ, &bars->q_full[qc % NQ], 64, c.h, t);
+                        q_issued = qc + 1;
                         if (r == 0) LA_CTRACE(c.n, TR_Q0);
                     }
                 }
@@ -333,152 +364,94 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             // On abort, wait (bounded) for this producer's copies still in flight
             // into shared memory: only the latest load of each stage can be pending.
             if (!ok) {
-                const uint32_t nst = kv_role ? NKV : NQ;
-                uint64_t* full = kv_role ? bars->kv_full : bars->q_full;
-                for (uint32_t i = (issued > nst ? issued - nst : 0); i < issued; ++i) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(&full[i % nst], (i / nst) & 1) && globaltimer_ns() - t0 < 100000000ull) {}
+                auto drain = [&](uint64_t* full, uint32_t issued, uint32_t nst) {
+                    for (uint32_t i = (issued > nst ? issued - nst : 0); i < issued; ++i) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (!mbar_try_wait(&full[i % nst], (i / nst) & 1) && globaltimer_ns() - t0 < 100000000ull) {}
+                    }
+                };
+                if (kv_role) {
+                    drain(bars->k_full, k_issued, NK);
+                    drain(bars->v_full, v_issued, NV);
+                } else {
+                    drain(bars->q_full, q_issued, NQ);
                 }
             }
         }
-    } else if (warp == 1) {
-        // ================================================================ tcgen05 issuer
-        if (lane == 0) {
-            // Shared-memory descriptors: the base of each region once, then a
-            // 16-byte-unit offset per operand step (the address field is the low 14 bits).
-            const uint64_t dq = sdesc_sw128(smem_u32(smem + OFF_Q), 16, 1024);             // K-major
-            const uint64_t dk = sdesc_sw128(smem_u32(smem + OFF_KV), 16, 1024);            // K-major (scores)
-            const uint64_t dkt = sdesc_sw128(smem_u32(smem + OFF_KV), KH_BYTES, 1024);     // MN-major (state)
-            const uint64_t dv = sdesc_sw128(smem_u32(smem + OFF_KV + K_BYTES), V_BYTES, 1024);
-            const uint64_t dsb = sdesc_sw128(smem_u32(smem + OFF_SB), SB_BYTES, 1024);
-            Cursor sc, pc;
+    } else if (warp == 1 || warp == 3) {
+        // Shared-memory descriptors: the base of each region once, then a 16-byte-unit
+        // offset per operand step (the address field is the low 14 bits).
+        const uint64_t dq = sdesc_sw128(smem_u32(smem + OFF_Q), 16, 1024);             // K-major
+        const uint64_t dk = sdesc_sw128(smem_u32(smem + OFF_K), 16, 1024);             // K-major (scores)
+        const uint64_t dkt = sdesc_sw128(smem_u32(smem + OFF_K), KH_BYTES, 1024);      // MN-major (state)
+        const uint64_t dv = sdesc_sw128(smem_u32(smem + OFF_V), V_BYTES, 1024);
+        const uint64_t dsb = sdesc_sw128(smem_u32(smem + OFF_SB), SB_BYTES, 1024);
+        if (warp == 1 && lane == 0) {
+            // ============================================================ issuer A: scores, state MMAs
+            // Event loop over two cursors; every step is taken only when its inputs are
+            // ready (non-blocking mbarrier tests). The score cursor needs its score buffer
+            // back (the PV that read it completed), its K chunk and, for a sub-unit's first
+            // item, its Q rows. The state cursor follows it: chunk j's state MMA once the V
+            // chunk is loaded and, for the block's first chunk, the state group has copied
+            // the previous prefix out.
+            Cursor sc, dc;
             sc.init(p);
-            pc.init(p);
-            // Event loop: every step is taken only when its inputs are ready (non-
-            // blocking mbarrier tests), so a score waiting for its K/V chunk never
-            // holds back a PV whose P is already in TMEM. The score cursor runs ahead
-            // of the PV cursor only as far as the rings allow without waiting on this
-            // thread's own later work: a score buffer is reused after the PV that
-            // read it, a K/V or Q stage is refilled after the commit that released it.
-            uint32_t pv_issued = 0, kv_released = 0, q_released = 0;
-            int stage = 0;                        // PV cursor's item: 0 PV, 1 state MMA, 2 inter MMA, 3 done
+            dc.init(p);
+            uint32_t s_issued = 0;
             uint32_t kvr_blk = 0xffffffffu;       // block whose state copy-out has been seen
             uint32_t idle = 0;
             uint64_t t_idle = 0;
-            while (pc.valid) {
+            while (sc.valid || dc.valid) {
                 bool prog = false;
-                // ---- (a) score MMAs ahead of the PV cursor
-                if (sc.valid && sc.i < pv_issued + NS && sc.kc0 + sc.j < kv_released + NKV &&
-                    sc.q0 + sc.r < q_released + NQ) {
-                    const uint32_t kc = sc.kc0 + sc.j, st = kc % NKV;
-                    const uint32_t qc = sc.q0 + sc.r, qs = qc % NQ;
-                    if ((!sc.first_of_chunk() || mbar_test_wait(&bars->kv_full[st], (kc / NKV) & 1)) &&
-                        (sc.j != 0 || mbar_test_wait(&bars->q_full[qs], (qc / NQ) & 1))) {
+                if (sc.valid) {
+                    const uint32_t kc = sc.kc0 + sc.j, qc = sc.q0 + sc.r, sbuf = sc.i % NS;
+                    if ((sc.i < NS || mbar_test_wait(&bars->s_free[sbuf], ((sc.i / NS) - 1) & 1)) &&
+                        (!sc.first_of_chunk() || mbar_test_wait(&bars->k_full[kc % NK], (kc / NK) & 1)) &&
+                        (!sc.first_of_sub() || mbar_test_wait(&bars->q_full[qc % NQ], (qc / NQ) & 1))) {
                         tc_fence_after();
-                        LA_ITRACE(sc.i, 0);
-                        const uint64_t a = dq + ((qs * Q_BYTES) >> 4), b = dk + ((st * KV_STAGE) >> 4);
-                        const uint32_t d_s = tmem + TM_S + (sc.i % NS) * KC;
+                        const uint64_t a = dq + (((qc % NQ) * Q_BYTES) >> 4), b = dk + (((kc % NK) * K_BYTES) >> 4);
+                        const uint32_t d_s = tmem + TM_S + sbuf * KC;
 #pragma unroll
                         for (int s = 0; s < D / 16; ++s)
                             mma_ss(d_s, a + (((s >> 2) * QH_BYTES + (s & 3) * 32) >> 4),
                                    b + (((s >> 2) * KH_BYTES + (s & 3) * 32) >> 4), IDESC_S, s > 0);
-                        tc_commit(&bars->s_full[sc.i % NS]);
-                        LA_ITRACE(sc.i, 1);
+                        tc_commit(&bars->s_full[sbuf]);
+                        if (sc.last_of_chunk()) tc_commit(&bars->k_empty[kc % NK]);   // the scores' share
+                        if (sc.last_of_sub()) tc_commit(&bars->q_empty[qc % NQ]);     // the scores' share
+                        ++s_issued;
                         if (sc.k == 0) LA_CTRACE(sc.n, TR_S0);
                         sc.next_item(p);
                         prog = true;
                     }
                 }
-                // ---- (b) the PV cursor's item, once its scores are issued
-                if (!sc.valid || sc.i > pc.i) {
-                    const uint32_t sbuf = pc.i % NS;
-                    const uint32_t slot = pc.oslot(pc.r);
-                    const uint32_t kc = pc.kc0 + pc.j, st = kc % NKV;
-                    const uint32_t d_o = tmem + TM_O + slot * 64;
-                    if (stage == 0 && mbar_test_wait(&bars->p_full[sbuf], (pc.i / NS) & 1) &&
-                        (pc.j != 0 || mbar_test_wait(&bars->o_empty[slot], (pc.ouse(pc.r) & 1) ^ 1))) {
-                        // O_r += P V_j; P of keys 0-63 in columns 0-31, of keys 64-127 in 64-95
-                        tc_fence_after();
-                        LA_ITRACE(pc.i, 4);
-                        const uint64_t b = dv + ((st * KV_STAGE) >> 4);
-                        const uint32_t a_p = tmem + TM_S + sbuf * KC;
-#pragma unroll
-                        for (int s = 0; s < KC / 16; ++s)
-                            mma_ts(d_o, a_p + (s < 4 ? s * 8 : 64 + (s - 4) * 8), b + ((s * 2048) >> 4), IDESC_PV,
-                                   (pc.j > 0 || s > 0));
-                        ++pv_issued;
-                        LA_ITRACE(pc.i, 5);
-                        if (pc.k == 0) LA_CTRACE(pc.n, TR_PV0);
-                        if (pc.last_of_block()) LA_CTRACE(pc.n, TR_PVL);
-                        stage = 1;
-                        prog = true;
-                    }
-                    if (stage == 1) {
-                        if (!pc.last_of_chunk()) {
-                            stage = 2;
-                        } else {
-                            // KV += K_j^T V_j once the state group has copied out this block's prefix
-                            if (pc.add_state && pc.j == 0 && kvr_blk != pc.n &&
-                                mbar_test_wait(&bars->kv_read[pc.n & 1], (pc.n >> 1) & 1)) {
-                                kvr_blk = pc.n;
-                                tc_fence_after();
-                            }
-                            if (!pc.add_state || pc.j > 0 || kvr_blk == pc.n) {
-                                if (pc.add_state) {
-                                    const uint64_t a = dkt + ((st * KV_STAGE) >> 4), b = dv + ((st * KV_STAGE) >> 4);
-#pragma unroll
-                                    for (int s = 0; s < KC / 16; ++s)
-                                        mma_ss(tmem + TM_KV, a + ((s * 2048) >> 4), b + ((s * 2048) >> 4), IDESC_KV,
-                                               (pc.b > 0 || pc.j > 0 || s > 0));
-                                    if (pc.j == pc.Rb - 1) {
-                                        tc_commit(&bars->kv_ready);
-                                        LA_CTRACE(pc.n, TR_KVR);
-                                    }
-                                }
-                                tc_commit(&bars->kv_empty[st]);
-                                ++kv_released;
-                                LA_ITRACE(pc.i, 6);
-                                stage = 2;
-                                prog = true;
-                            }
+                if (dc.valid && dc.i < s_issued) {
+                    if (!dc.last_of_chunk()) {
+                        dc.next_item(p);
+                    } else {
+                        const uint32_t kc = dc.kc0 + dc.j;
+                        bool ready = mbar_test_wait(&bars->v_full[kc % NV], (kc / NV) & 1);
+                        if (ready && dc.add_state && dc.j == 0 && kvr_blk != dc.n) {
+                            if (mbar_test_wait(&bars->kv_read[dc.n & 3], (dc.n >> 2) & 1)) kvr_blk = dc.n;
+                            else ready = false;
                         }
-                    }
-                    if (stage == 2) {
-                        // O_r += Q_r . bf16(KV_b) after sub-unit r's last item (every item is
-                        // the last of its sub-unit except (0,1))
-                        if (pc.k == 0 && pc.Rb == 2) {
-                            stage = 3;
-                        } else {
-                            bool ready = true;
-                            if (pc.r == 0) {
-                                if (kvr_blk != pc.n) {
-                                    if (mbar_test_wait(&bars->kv_read[pc.n & 1], (pc.n >> 1) & 1)) kvr_blk = pc.n;
-                                    else ready = false;
-                                }
-                                if (ready && !mbar_test_wait(&bars->sb_full, pc.n & 1)) ready = false;
-                            }
-                            if (ready) {
+                        if (ready) {
+                            if (dc.add_state) {
                                 tc_fence_after();
-                                const uint32_t qc = pc.q0 + pc.r, qs = qc % NQ;
-                                const uint64_t a = dq + ((qs * Q_BYTES) >> 4);
+                                const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4), b = dv + (((kc % NV) * V_BYTES) >> 4);
 #pragma unroll
-                                for (int s = 0; s < D / 16; ++s)
-                                    mma_ss(d_o, a + (((s >> 2) * QH_BYTES + (s & 3) * 32) >> 4),
-                                           dsb + ((s * 2048) >> 4), IDESC_C, 1);
-                                tc_commit(&bars->q_empty[qs]);
-                                ++q_released;
-                                tc_commit(&bars->o_full[slot]);
-                                if (pc.r == pc.Rb - 1) tc_commit(&bars->sb_empty);
-                                LA_CTRACE(pc.n, pc.r == 0 ? TR_C0 : TR_CL);
-                                LA_ITRACE(pc.i, 7);
-                                stage = 3;
-                                prog = true;
+                                for (int s = 0; s < KC / 16; ++s)
+                                    mma_ss(tmem + TM_KV, a + ((s * 2048) >> 4), b + ((s * 2048) >> 4), IDESC_KV,
+                                           (dc.b > 0 || dc.j > 0 || s > 0));
+                                if (dc.j == dc.Rb - 1) {
+                                    tc_commit(&bars->kv_ready);
+                                    LA_CTRACE(dc.n, TR_KVR);
+                                }
                             }
+                            tc_commit(&bars->k_empty[kc % NK]);          // the state MMA's shares
+                            tc_commit(&bars->v_empty[kc % NV]);
+                            dc.next_item(p);
+                            prog = true;
                         }
-                    }
-                    if (stage == 3) {
-                        pc.next_item(p);
-                        stage = 0;
                     }
                 }
                 // ---- nothing ready: bounded idle time, launch-wide abort
@@ -495,6 +468,51 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             tc_commit(&bars->drain);
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&bars->drain, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
+        } else if (warp == 3 && lane == 0) {
+            // ============================================================ issuer B: inter-block, PV
+            // Item by item: the inter-block MMA first for a sub-unit's first item (it
+            // initialises the accumulator), then the PV once the P groups have written P.
+            Cursor c;
+            c.init(p);
+            bool ok = true;
+            while (ok && c.valid) {
+                const uint32_t sbuf = c.i % NS, slot = c.oslot(c.r);
+                const uint32_t kc = c.kc0 + c.j, qc = c.q0 + c.r;
+                const uint32_t d_o = tmem + TM_O + slot * 64;
+                if (c.first_of_sub()) {
+                    // O_r = Q_r . bf16(KV_b)
+                    if (!wait_bar(&bars->o_empty[slot], (c.ouse(c.r) & 1) ^ 1, ab)) { ok = false; break; }
+                    if (c.r == 0 && !wait_bar(&bars->sb_full, c.n & 1, ab)) { ok = false; break; }
+                    if (!wait_bar(&bars->q_full[qc % NQ], (qc / NQ) & 1, ab)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t a = dq + (((qc % NQ) * Q_BYTES) >> 4);
+#pragma unroll
+                    for (int s = 0; s < D / 16; ++s)
+                        mma_ss(d_o, a + (((s >> 2) * QH_BYTES + (s & 3) * 32) >> 4), dsb + ((s * 2048) >> 4), IDESC_C,
+                               s > 0);
+                    if (c.r == c.Rb - 1) tc_commit(&bars->sb_empty);
+                    tc_commit(&bars->q_empty[qc % NQ]);                  // the inter-block MMA's share
+                    LA_CTRACE(c.n, c.r == 0 ? TR_C0 : TR_CL);
+                }
+                // O_r += P V_j; P of keys 0-63 in columns 0-31, of keys 64-127 in 64-95
+                if (!wait_bar(&bars->p_full[sbuf], (c.i / NS) & 1, ab)) { ok = false; break; }
+                if (c.first_of_chunk() && !wait_bar(&bars->v_full[kc % NV], (kc / NV) & 1, ab)) { ok = false; break; }
+                tc_fence_after();
+                const uint64_t b = dv + (((kc % NV) * V_BYTES) >> 4);
+                const uint32_t a_p = tmem + TM_S + sbuf * KC;
+#pragma unroll
+                for (int s = 0; s < KC / 16; ++s)
+                    mma_ts(d_o, a_p + (s < 4 ? s * 8 : 64 + (s - 4) * 8), b + ((s * 2048) >> 4), IDESC_PV, 1);
+                tc_commit(&bars->s_free[sbuf]);
+                if (c.last_of_chunk()) tc_commit(&bars->v_empty[kc % NV]);   // the PVs' share
+                if (c.last_of_sub()) tc_commit(&bars->o_full[slot]);
+                if (c.k == 0) LA_CTRACE(c.n, TR_PV0);
+                if (c.last_of_block()) LA_CTRACE(c.n, TR_PVL);
+                c.next_item(p);
+            }
+            tc_commit(&bars->drain_b);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&bars->drain_b, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
         }
     } else if (warp >= 4 && warp < 12) {
         // ================================================================ scores -> P
@@ -535,59 +553,56 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_full[sbuf]);
-            if (m == 0 && hk == 0) LA_ITRACE(c.i, 3);
+            if (m == 0) LA_ITRACE(c.i, 3 + 5 * hk);
             if (m == 0 && hk == 0 && c.k == 0) LA_CTRACE(c.n, TR_P0);
             if (m == 0 && hk == 0 && c.last_of_block()) LA_CTRACE(c.n, TR_PL);
             c.next_item(p);
         }
-    } else if (warp >= 12) {
-        // ================================================================ state copy-out, O epilogue
+    } else if (warp >= 12 && warp < 16) {
+        // ================================================================ state copy-out
         const int quad = warp & 3;
-        const int m = quad * 32 + lane;                  // TMEM lane: state row i / query row
+        const int m = quad * 32 + lane;                  // TMEM lane: state row i
         const int wt = threadIdx.x - 384;                // 0..127
         const uint32_t lane_base = uint32_t(quad * 32) << 16;
         uint8_t* sb = smem + OFF_SB;
-        uint8_t* stage = smem + OFF_STG;
-        const uint64_t o_pol = policy_evict_first();     // O is never read back
-        uint32_t grp_phase = 0, kvc = 0;                 // kvc: blocks whose state was added
-        bool stored = false, ok = true;
+        uint32_t kvc = 0;                                // blocks whose state was added
+        bool ok = true;
         Cursor c;
         c.init(p);
         while (ok && c.valid) {
-            // ---- KV_b (+ S0) -> bf16 operand of the inter-block product (row m, 64 columns)
+            // KV_b (+ S0) -> bf16 operand of the inter-block product (row m, 64 columns)
+            if (c.b > 0) {
+                if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
+                ++kvc;
+                if (wt == 0) LA_CTRACE(c.n, TR_XR);
+                tc_fence_after();
+            }
+            const float* s0 = p.init ? p.init + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half : nullptr;
             uint32_t pk[32];
-            {
-                float x[64];
-                if (c.b == 0) {
 #pragma unroll
-                    for (int q = 0; q < 64; ++q) x[q] = 0.f;
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t a[32];
+                if (c.b > 0) {
+                    tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                    tmem_wait_ld();
                 } else {
-                    if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
-                    ++kvc;
-                    if (wt == 0) LA_CTRACE(c.n, TR_XR);
-                    tc_fence_after();
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t a[32];
-                        tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) x[32 * hh + q] = __uint_as_float(a[q]);
-                    }
+                    for (int q = 0; q < 32; ++q) a[q] = 0u;
                 }
-                tc_fence_before();
-                mbar_arrive(&bars->kv_read[c.n & 1]);    // the accumulator may take this block's keys
-                if (p.init) {
-                    const float4* s0 = reinterpret_cast<const float4*>(
-                        p.init + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 v = __ldg(s0 + q);
-                        x[4 * q] += v.x; x[4 * q + 1] += v.y; x[4 * q + 2] += v.z; x[4 * q + 3] += v.w;
-                    }
+                if (hh == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&bars->kv_read[c.n & 3]);    // the accumulator may take this block's keys
                 }
 #pragma unroll
-                for (int q = 0; q < 32; ++q) pk[q] = pack_bf16x2(x[2 * q], x[2 * q + 1]);
+                for (int q = 0; q < 16; ++q) {
+                    float x0 = __uint_as_float(a[2 * q]), x1 = __uint_as_float(a[2 * q + 1]);
+                    if (s0) {
+                        const float2 v = __ldg(reinterpret_cast<const float2*>(s0 + 32 * hh + 2 * q));
+                        x0 += v.x;
+                        x1 += v.y;
+                    }
+                    pk[16 * hh + q] = pack_bf16x2(x0, x1);
+                }
             }
             if (!warp_all(wait_bar(&bars->sb_empty, (c.n & 1) ^ 1, ab))) { ok = false; break; }
 #pragma unroll
@@ -597,7 +612,22 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             fence_proxy_async_smem();
             if (!(c.w == p.suppress_item && c.b == 1)) mbar_arrive(&bars->sb_full);
             if (wt == 0) LA_CTRACE(c.n, TR_SB);
-            // ---- O epilogue of each sub-unit, in the order the issuer finishes them
+            c.next_block(p);
+        }
+    } else if (warp >= 16) {
+        // ================================================================ O epilogue
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;                  // TMEM lane: query row of the sub-unit
+        const int wt = threadIdx.x - 512;                // 0..127
+        const uint32_t lane_base = uint32_t(quad * 32) << 16;
+        uint8_t* stage = smem + OFF_STG;
+        const uint64_t o_pol = policy_evict_first();     // O is never read back
+        uint32_t grp_phase = 0;
+        bool stored = false, ok = true;
+        Cursor c;
+        c.init(p);
+        while (ok && c.valid) {
+            // each sub-unit in the order the issuer finishes them
             for (int r = 0; ok && r < c.Rb; ++r) {
                 const uint32_t slot = c.oslot(r);
                 if (!warp_all(wait_bar(&bars->o_full[slot], c.ouse(r) & 1, ab))) { ok = false; break; }
@@ -616,7 +646,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 tc_fence_before();
                 mbar_arrive(&bars->o_empty[slot]);
                 const int rows = min(UM, c.rows - UM * r);
-                if (rows == UM) {
+                if (!LA_CHAIN_DIRECT_O && rows == UM) {
                     if (wt == 0 && stored) bulk_wait_read0();    // the previous store has read the staging
                     if (!warp_all(group_sync(&bars->grp, grp_phase, ab))) { ok = false; break; }
 #pragma unroll
@@ -629,7 +659,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         tma_store_3d_hint(&tmO, stage, DV * c.half, c.h, c.tok0 + UM * r, o_pol);
                         bulk_commit();
                         stored = true;
-                        if (r == c.Rb - 1) LA_CTRACE(c.n, TR_ST);
                     }
                 } else if (m < rows) {
                     __nv_bfloat16* orow = p.out + ((int64_t)(c.tok0 + UM * r + m) * p.H + c.h) * D + DV * c.half;
@@ -638,6 +667,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         __stcs(reinterpret_cast<uint4*>(orow + 8 * g),
                                make_uint4(ov[4 * g], ov[4 * g + 1], ov[4 * g + 2], ov[4 * g + 3]));
                 }
+                if (wt == 0 && r == c.Rb - 1) LA_CTRACE(c.n, TR_ST);
             }
             c.next_block(p);
         }
