@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "fused.cuh"
 #include "chain.cuh"
+#include "state.cuh"
 
 namespace {
 
@@ -103,8 +104,16 @@ Layout prefill_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt) {
     return L;
 }
 
-Layout state_layout(int64_t T, int nseq, int H, int d) {
+Layout state_layout(int64_t T, int nseq, int H, int d, la_dtype dt) {
     Layout L;
+    if (dt == LA_BF16 && d == 128) {
+        // tensor-core path: Control | sequence table | order (unused here)
+        size_t off = sizeof(Control);
+        L.off_seqs = off;  off = align_up(off + sizeof(la::SeqEntry) * (size_t)nseq, 256);
+        L.off_order = off; off = align_up(off + sizeof(int32_t) * (size_t)nseq, 256);
+        L.total = off;
+        return L;
+    }
     size_t off = layout_head(L, T, nseq, kStateBlock);
     L.off_U = off; off = align_up(off + 4 * (size_t)d * d * (size_t)H * (size_t)L.max_blocks, 256);
     L.total = off;
@@ -301,7 +310,7 @@ size_t la_prefill_workspace_size(int64_t total_tokens, int num_seqs, int heads, 
 size_t la_state_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, la_dtype dtype) {
     if (total_tokens < 0 || num_seqs < 1 || heads < 1 || !supported_d(d) || (dtype != LA_BF16 && dtype != LA_FP32))
         return 0;
-    return state_layout(total_tokens, num_seqs, heads, d).total;
+    return state_layout(total_tokens, num_seqs, heads, d, dtype).total;
 }
 
 la_status la_prefill(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
@@ -359,7 +368,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
         const unsigned grid = (unsigned)(items < sms ? items : sms);
         const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
 #ifdef LA_CHAIN_ITEM_TRACE
-        const size_t reserved = 4096 * 8 * sizeof(uint64_t);   // per-item stamps of CTA 0 after the block table
+        const size_t reserved = (4096 * 8 + 2 * 4096 * 4) * sizeof(uint64_t);  // item and MMA-group stamps of CTA 0
 #else
         const size_t reserved = 0;
 #endif
@@ -440,12 +449,44 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
     const size_t state_bytes = (size_t)num_seqs * heads * d * d * 4;
     if (init_state && init_state != state_out && overlaps(init_state, state_bytes, state_out, state_bytes))
         return LA_ERR_INVALID_ARGUMENT;
-    const Layout L = state_layout(total_tokens, num_seqs, heads, d);
+    const Layout L = state_layout(total_tokens, num_seqs, heads, d, dtype);
     if (!workspace) return LA_ERR_INVALID_ARGUMENT;
     if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
     if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (dtype == LA_BF16 && d == 128) {
+        // tensor cores: one CTA per (sequence, head, value-column half)
+        la::SeqEntry* seqs = reinterpret_cast<la::SeqEntry*>(ws + L.off_seqs);
+        la::seq_table_kernel<<<1, 1024, 0, st>>>(cu_seqlens, num_seqs, total_tokens, seqs,
+                                                 reinterpret_cast<int32_t*>(ws + L.off_order),
+                                                 reinterpret_cast<Control*>(ws));
+        note_launch();
+        if ((s = cuda_check()) != LA_OK) return s;
+        CUtensorMap tk, tv;
+        const int64_t rows = total_tokens > 0 ? total_tokens : 1;
+        if (!map_tokens(&tk, k ? k : state_out, rows, heads, d, la::state::KC) ||
+            !map_tokens(&tv, v ? v : state_out, rows, heads, d, la::state::KC))
+            return LA_ERR_CUDA;
+        la::state::Params prm;
+        prm.out = state_out;
+        prm.init = init_state;
+        prm.seqs = seqs;
+        prm.ctrl = reinterpret_cast<const Control*>(ws);
+        prm.H = heads;
+        prm.nseq = num_seqs;
+        prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
+        if (cudaFuncSetAttribute(la::state::state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)la::state::SMEM_BYTES) != cudaSuccess)
+            return LA_ERR_CUDA;
+        const int64_t items = 2 * (int64_t)num_seqs * heads;
+        const int sms = num_sms();
+        if (sms <= 0) return LA_ERR_CUDA;
+        const unsigned grid = (unsigned)(items < sms ? items : sms);
+        la::state::state_kernel<<<grid, la::state::NTHREADS, la::state::SMEM_BYTES, st>>>(tk, tv, prm);
+        note_launch();
+        return cuda_check();
+    }
     if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, kStateBlock, heads, L, ws, st)) != LA_OK) return s;
     if (total_tokens > 0 && (s = simt_states_d(d, dtype, k, v, heads, L, ws, st)) != LA_OK) return s;
     const int dd = d * d;
