@@ -23,10 +23,10 @@ import torch
 __all__ = [
     "LightningError", "LA_BF16", "LA_FP32", "STATUS", "library_path", "load_library",
     "la_prefill_workspace_size", "la_prefill", "la_prefill_noalloc", "LA_NOALLOC_SCRATCH_BYTES",
-    "la_state_workspace_size", "la_state_from_prefill",
+    "la_state_workspace_size", "la_state_from_prefill", "la_state_exclusive_prefix",
     "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
     "la_launch_count",
-    "prefill", "state_from_prefill", "decode_step", "device_status", "uses_tensor_cores",
+    "prefill", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status", "uses_tensor_cores",
 ]
 
 LA_BF16 = 0
@@ -75,6 +75,8 @@ def load_library():
         lib.la_state_workspace_size.restype = sz
         lib.la_state_from_prefill.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, sz, vp]
         lib.la_state_from_prefill.restype = i32
+        lib.la_state_exclusive_prefix.argtypes = [vp, i32, i32, i64, i32, vp, vp, vp]
+        lib.la_state_exclusive_prefix.restype = i32
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         lib.la_decode_step.restype = i32
         lib.la_get_device_status.argtypes = [vp]
@@ -126,6 +128,10 @@ def la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dt
                           workspace, workspace_bytes, stream) -> int:
     return int(load_library().la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype,
                                                     init_state, state_out, workspace, workspace_bytes, stream))
+
+
+def la_state_exclusive_prefix(gathered, world, rank, n, d, init, out, stream) -> int:
+    return int(load_library().la_state_exclusive_prefix(gathered, world, rank, n, d, init, out, stream))
 
 
 def la_decode_step(q, k, v, state, o, batch, heads, d, dtype, stream) -> int:
@@ -261,6 +267,26 @@ def state_from_prefill(k, v, cu_seqlens=None, init_state=None, out=None, workspa
                                    _p(workspace), workspace.numel() * workspace.element_size(),
                                    _stream_handle(stream, k.device))
     _raise(status, "la_state_from_prefill")
+    return out
+
+
+def state_exclusive_prefix(gathered, rank, init=None, out=None, stream=None):
+    """init + sum of gathered[:rank] for fp32 gathered [world, *S], S = [num_seqs, H, d, d]
+    (see la_state_exclusive_prefix; rank = world gives the state after the last segment)."""
+    _need(gathered, "gathered")
+    if gathered.dtype != torch.float32 or gathered.dim() != 5 or gathered.shape[-1] != gathered.shape[-2]:
+        raise LightningError("gathered must be fp32 [world, num_seqs, H, d, d]", 1)
+    world, nseq, H, d = gathered.shape[0], gathered.shape[1], gathered.shape[2], gathered.shape[3]
+    if out is None:
+        out = torch.empty(gathered.shape[1:], dtype=torch.float32, device=gathered.device)
+    _need(out, "out", gathered.device)
+    if init is not None:
+        _need(init, "init", gathered.device)
+        if init.dtype != torch.float32 or init.shape != out.shape:
+            raise LightningError("init must be fp32 [num_seqs, H, d, d]", 1)
+    status = la_state_exclusive_prefix(_p(gathered), world, rank, nseq * H, d, _p(init), _p(out),
+                                       _stream_handle(stream, gathered.device))
+    _raise(status, "la_state_exclusive_prefix")
     return out
 
 

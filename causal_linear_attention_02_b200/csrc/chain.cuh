@@ -120,7 +120,6 @@ struct Bars {
     uint64_t sb_full, sb_empty;
     uint64_t grp;             // bounded barrier of the epilogue group
     uint64_t drain, drain_b;
-    uint64_t tgrp[2];         // per-issuer MMA-group completion stamps (LA_CHAIN_ITEM_TRACE builds)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -160,33 +159,6 @@ enum TraceEvent {
     TR_PVL = 15,       // issuer: last PV MMA issued
     kTraceEvents = 16
 };
-// Debug stamps of CTA 0 (compile-time option LA_CHAIN_ITEM_TRACE), after the
-// block table in the trace buffer: eight clock64 values per item (LA_ITRACE),
-// then per issuer a log of its MMA groups, {code, issue start, issue end,
-// completion} (LA_GSTART / LA_GEND; completion stamped by a waiter lane).
-#ifdef LA_CHAIN_ITEM_TRACE
-#define LA_ITRACE(i, ev)                                                                                    \
-    do {                                                                                                    \
-        if (p.trace && blockIdx.x == 0 && (int)(i) < 4096)                                                  \
-            p.trace[(int64_t)gridDim.x * p.trace_blocks * kTraceEvents + (int64_t)(i) * 8 + (ev)] = clock64(); \
-    } while (0)
-#define LA_GREC(w, g) (p.trace + (int64_t)gridDim.x * p.trace_blocks * kTraceEvents + 4096 * 8 + \
-                       (int64_t)(w) * 4096 * 4 + (int64_t)(g) * 4)
-#define LA_GSTART() do { g_t0 = clock64(); } while (0)
-#define LA_GEND(w, code)                                                                                     \
-    do {                                                                                                    \
-        if (p.trace && blockIdx.x == 0 && g_n < 4096) {                                                     \
-            tc_commit(&bars->tgrp[w]);                                                                      \
-            uint64_t* r_ = LA_GREC(w, g_n);                                                                 \
-            r_[0] = (code); r_[1] = g_t0; r_[2] = clock64();                                                \
-        }                                                                                                   \
-        ++g_n;                                                                                              \
-    } while (0)
-#else
-#define LA_ITRACE(i, ev) do {} while (0)
-#define LA_GSTART() do {} while (0)
-#define LA_GEND(w, code) do {} while (0)
-#endif
 #define LA_CTRACE(n, ev)                                                                                   \
     do {                                                                                                   \
         if (p.trace && (int)(n) < p.trace_blocks)                                                          \
@@ -314,8 +286,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars->grp, 128);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->drain_b, 1);
-        mbar_init(&bars->tgrp[0], 1);
-        mbar_init(&bars->tgrp[1], 1);
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -331,21 +301,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-#ifdef LA_CHAIN_ITEM_TRACE
-    if (warp == 2 && (lane == 1 || lane == 2) && p.trace && blockIdx.x == 0) {
-        // completion stamps of issuer A's (lane 1) or B's (lane 2) MMA groups, in order
-        const int w = lane - 1;
-        for (uint32_t g = 0; g < 4096; ++g) {
-            const uint64_t t0 = globaltimer_ns();
-            bool done = true;
-            while (!mbar_try_wait(&bars->tgrp[w], g & 1)) {
-                if (globaltimer_ns() - t0 > 50000000ull) { done = false; break; }
-            }
-            if (!done) break;
-            LA_GREC(w, g)[3] = clock64();
-        }
-    }
-#endif
     if (warp == 0 || warp == 2) {
         // ================================================================ TMA producers
         if (lane == 0) {
@@ -424,10 +379,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             dc.init(p);
             uint32_t s_issued = 0;
             uint32_t kvr_blk = 0xffffffffu;       // block whose state copy-out has been seen
-#ifdef LA_CHAIN_ITEM_TRACE
-            uint32_t g_n = 0;
-            uint64_t g_t0 = 0;
-#endif
             uint32_t idle = 0;
             uint64_t t_idle = 0;
             while (sc.valid || dc.valid) {
@@ -438,7 +389,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         (!sc.first_of_chunk() || mbar_test_wait(&bars->k_full[kc % NK], (kc / NK) & 1)) &&
                         (!sc.first_of_sub() || mbar_test_wait(&bars->q_full[qc % NQ], (qc / NQ) & 1))) {
                         tc_fence_after();
-                        LA_GSTART();
                         const uint64_t a = dq + (((qc % NQ) * Q_BYTES) >> 4), b = dk + (((kc % NK) * K_BYTES) >> 4);
                         const uint32_t d_s = tmem + TM_S + sbuf * KC;
 #pragma unroll
@@ -449,7 +399,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         if (sc.last_of_chunk()) tc_commit(&bars->k_empty[kc % NK]);   // the scores' share
                         if (sc.last_of_sub()) tc_commit(&bars->q_empty[qc % NQ]);     // the scores' share
                         ++s_issued;
-                        LA_GEND(0, 0x10000u | sc.i);
                         if (sc.k == 0) LA_CTRACE(sc.n, TR_S0);
                         sc.next_item(p);
                         prog = true;
@@ -468,7 +417,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         if (ready) {
                             if (dc.add_state) {
                                 tc_fence_after();
-                                LA_GSTART();
                                 const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4), b = dv + (((kc % NV) * V_BYTES) >> 4);
 #pragma unroll
                                 for (int s = 0; s < KC / 16; ++s)
@@ -478,7 +426,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                                     tc_commit(&bars->kv_ready);
                                     LA_CTRACE(dc.n, TR_KVR);
                                 }
-                                LA_GEND(0, 0x20000u | dc.i);
                             }
                             tc_commit(&bars->k_empty[kc % NK]);          // the state MMA's shares
                             tc_commit(&bars->v_empty[kc % NV]);
@@ -508,10 +455,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             Cursor c;
             c.init(p);
             bool ok = true;
-#ifdef LA_CHAIN_ITEM_TRACE
-            uint32_t g_n = 0;
-            uint64_t g_t0 = 0;
-#endif
             while (ok && c.valid) {
                 const uint32_t sbuf = c.i % NS, slot = c.oslot(c.r);
                 const uint32_t kc = c.kc0 + c.j, qc = c.q0 + c.r;
@@ -522,7 +465,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (c.r == 0 && !wait_bar(&bars->sb_full, c.n & 1, ab)) { ok = false; break; }
                     if (!wait_bar(&bars->q_full[qc % NQ], (qc / NQ) & 1, ab)) { ok = false; break; }
                     tc_fence_after();
-                    LA_GSTART();
                     const uint64_t a = dq + (((qc % NQ) * Q_BYTES) >> 4);
 #pragma unroll
                     for (int s = 0; s < D / 16; ++s)
@@ -531,13 +473,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (c.r == c.Rb - 1) tc_commit(&bars->sb_empty);
                     tc_commit(&bars->q_empty[qc % NQ]);                  // the inter-block MMA's share
                     LA_CTRACE(c.n, c.r == 0 ? TR_C0 : TR_CL);
-                    LA_GEND(1, 0x30000u | c.i);
                 }
                 // O_r += P V_j; P of keys 0-63 in columns 0-31, of keys 64-127 in 64-95
                 if (!wait_bar(&bars->p_full[sbuf], (c.i / NS) & 1, ab)) { ok = false; break; }
                 if (c.first_of_chunk() && !wait_bar(&bars->v_full[kc % NV], (kc / NV) & 1, ab)) { ok = false; break; }
                 tc_fence_after();
-                LA_GSTART();
                 const uint64_t b = dv + (((kc % NV) * V_BYTES) >> 4);
                 const uint32_t a_p = tmem + TM_S + sbuf * KC;
 #pragma unroll
@@ -546,7 +486,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 tc_commit(&bars->s_free[sbuf]);
                 if (c.last_of_chunk()) tc_commit(&bars->v_empty[kc % NV]);   // the PVs' share
                 if (c.last_of_sub()) tc_commit(&bars->o_full[slot]);
-                LA_GEND(1, 0x40000u | c.i);
                 if (c.k == 0) LA_CTRACE(c.n, TR_PV0);
                 if (c.last_of_block()) LA_CTRACE(c.n, TR_PVL);
                 c.next_item(p);
@@ -567,7 +506,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         while (ok && c.valid) {
             const uint32_t sbuf = c.i % NS;
             if (!warp_all(wait_bar(&bars->s_full[sbuf], (c.i / NS) & 1, ab))) { ok = false; break; }
-            if (m == 0 && hk == 0) LA_ITRACE(c.i, 2);
             tc_fence_after();
             const uint32_t ts = tmem + lane_base + TM_S + sbuf * KC + 64 * hk;
             const int lim = UM * (c.r - c.j) + m - 64 * hk;    // key column kept when col <= lim
@@ -594,7 +532,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_full[sbuf]);
-            if (m == 0) LA_ITRACE(c.i, 3 + hk);
             if (m == 0 && hk == 0 && c.k == 0) LA_CTRACE(c.n, TR_P0);
             if (m == 0 && hk == 0 && c.last_of_block()) LA_CTRACE(c.n, TR_PL);
             c.next_item(p);

@@ -19,6 +19,7 @@
 #include "fused.cuh"
 #include "chain.cuh"
 #include "state.cuh"
+#include "lasp.cuh"
 
 namespace {
 
@@ -367,13 +368,8 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
         if (sms <= 0) return LA_ERR_CUDA;
         const unsigned grid = (unsigned)(items < sms ? items : sms);
         const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
-#ifdef LA_CHAIN_ITEM_TRACE
-        const size_t reserved = (4096 * 8 + 2 * 4096 * 4) * sizeof(uint64_t);  // item and MMA-group stamps of CTA 0
-#else
-        const size_t reserved = 0;
-#endif
-        prm.trace = (t_trace && t_trace_bytes >= per_block + reserved) ? t_trace : nullptr;
-        prm.trace_blocks = prm.trace ? (int)std::min<size_t>((t_trace_bytes - reserved) / per_block, 1 << 30) : 0;
+        prm.trace = (t_trace && t_trace_bytes >= per_block) ? t_trace : nullptr;
+        prm.trace_blocks = prm.trace ? (int)std::min<size_t>(t_trace_bytes / per_block, 1 << 30) : 0;
         if (cudaFuncSetAttribute(la::chain::prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)la::chain::SMEM_BYTES) != cudaSuccess)
             return LA_ERR_CUDA;
@@ -518,6 +514,29 @@ la_status la_decode_step(const void* q, const void* k, const void* v, float* sta
     if (pairs >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;
     MainKernelTimer timer(reinterpret_cast<cudaStream_t>(stream));
     return decode_d(d, dtype, q, k, v, state, o, pairs, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_state_exclusive_prefix(const float* gathered, int world, int rank, int64_t n, int d, const float* init,
+                                    float* out, void* stream) {
+    if (world < 1 || rank < 0 || rank > world || n < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (!supported_d(d)) return LA_ERR_UNSUPPORTED;
+    if (n == 0) return LA_OK;
+    if (!gathered || !out) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(gathered, 16) || !aligned(out, 16) || (init && !aligned(init, 16))) return LA_ERR_MISALIGNED;
+    const int64_t per_rank = n * d * d;                 // floats of one rank's states
+    const size_t bytes = (size_t)per_rank * 4;
+    if (overlaps(out, bytes, gathered, bytes * (size_t)world)) return LA_ERR_INVALID_ARGUMENT;
+    if (init && init != out && overlaps(out, bytes, init, bytes)) return LA_ERR_INVALID_ARGUMENT;
+    const int sms = num_sms();
+    if (sms <= 0) return LA_ERR_CUDA;
+    const int64_t per_rank4 = per_rank / 4;             // d*d is a multiple of 4 for every supported d
+    const int64_t want = (per_rank4 + 255) / 256;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)sms * 8);
+    la::state_prefix_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const float4*>(gathered), rank, per_rank4, reinterpret_cast<const float4*>(init),
+        reinterpret_cast<float4*>(out));
+    note_launch();
+    return cuda_check();
 }
 
 la_status la_get_device_status(void* stream) {

@@ -1,0 +1,67 @@
+"""Sequence parallelism for the prefill (LASP+), one process per GPU.
+
+Each rank holds a contiguous segment of the same sequences (rank r holds the
+r-th segment of every sequence, ranks in sequence order). The prefill of a
+segment needs only the state of everything before it, so the ranks
+
+  1. compute their segments' states from a zero state (la_state_from_prefill),
+  2. exchange them with one all-gather (torch.distributed; NCCL on GPUs),
+  3. take a local exclusive prefix sum (la_state_exclusive_prefix), and
+  4. run their own prefill from that state (la_prefill with init_state).
+
+This is the all-gather + local prefix sum that replaces the serial
+send/receive chain of linear-attention sequence parallelism (page "MiniMax-01
+Lightning Attention", section "计算优化", item 3; page "首个线性注意力架构的大
+模型来了…", section "4.2 计算优化"). Steps 1, 3 and 4 run in the library's
+kernels; this module only moves tensors between them and the collective.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+import torch.distributed as dist
+
+from . import prefill, state_exclusive_prefix, state_from_prefill
+
+__all__ = ["LibraryOps", "lasp_prefill"]
+
+
+class LibraryOps:
+    """The three compute steps, on the library's CUDA kernels."""
+
+    @staticmethod
+    def segment_state(k, v, cu_seqlens):
+        return state_from_prefill(k, v, cu_seqlens)
+
+    @staticmethod
+    def exclusive_prefix(gathered, rank, init_state):
+        return state_exclusive_prefix(gathered, rank, init_state)
+
+    @staticmethod
+    def prefill(q, k, v, cu_seqlens, B, init_state, out):
+        return prefill(q, k, v, cu_seqlens, B=B, init_state=init_state, out=out)
+
+
+def lasp_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None, *,
+                 B: int = 256, init_state: Optional[torch.Tensor] = None, group=None, out=None,
+                 return_state: bool = False, ops=LibraryOps):
+    """O of this rank's segment [T_r, H, d] of the sequences (see the module docstring).
+
+    cu_seqlens (int32, [num_seqs + 1]) delimits this rank's segments of the
+    num_seqs sequences, in sequence order; None means one sequence. init_state
+    (fp32 [num_seqs, H, d, d]) is the state before the first segment, the same
+    tensor on every rank. Every rank of `group` must call this with the same
+    num_seqs, H and d. With return_state, also returns the state after the last
+    segment (the state a decode continues from), identical on every rank.
+    """
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    local = ops.segment_state(k, v, cu_seqlens)                        # [num_seqs, H, d, d], zero start
+    gathered = torch.empty((world,) + tuple(local.shape), dtype=local.dtype, device=local.device)
+    dist.all_gather(list(gathered.unbind(0)), local.contiguous(), group=group)
+    start = ops.exclusive_prefix(gathered, rank, init_state)
+    o = ops.prefill(q, k, v, cu_seqlens, B, start, out)
+    if not return_state:
+        return o
+    return o, ops.exclusive_prefix(gathered, world, init_state)

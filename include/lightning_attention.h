@@ -132,6 +132,29 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sequence parallelism (LASP+): each of `world` ranks holds a contiguous
+ * segment of the same sequences, computes its segments' states from a zero
+ * state (la_state_from_prefill with init_state = NULL), exchanges them with
+ * one all-gather, and takes a local prefix sum as the init_state of its own
+ * la_prefill (page "MiniMax-01 Lightning Attention", section "计算优化",
+ * item 3: AllGather + local prefix sum instead of serial send/receive; page
+ * "首个线性注意力架构的大模型来了…", section "4.2 计算优化"). This call is
+ * that local prefix sum:
+ *   out[i] = init[i] + sum_{r < rank} gathered[r][i]     (fp32, rank order)
+ *   gathered  in   fp32 [world][n][d][d], n = num_seqs * heads, the gathered
+ *                  segment states (device)
+ *   init      in   fp32 [n][d][d], the state before the first segment, or NULL
+ *                  (zero); may equal out, must not partially overlap it
+ *   out       out  fp32 [n][d][d] (device); must not overlap gathered
+ * rank = world gives the state after the last segment (the decode state).
+ * Errors: LA_ERR_INVALID_ARGUMENT (world < 1, rank outside [0, world], n < 0,
+ * null pointers, overlaps), LA_ERR_UNSUPPORTED (d), LA_ERR_MISALIGNED (any
+ * pointer not 16-byte aligned). Asynchronous on `stream`; allocates nothing.
+ */
+la_status la_state_exclusive_prefix(const float* gathered, int world, int rank, int64_t n, int d,
+                                    const float* init, float* out, void* stream);
+
+/*
  * One recurrent decode step for `batch` independent sequences:
  *   S <- S + k^T v ;  o = q S      (o sees the updated state: s <= t)
  *   q, k, v  in      [batch][heads][d] (dtype)

@@ -6,6 +6,7 @@ Tolerances (bound on the whole output, relative to its largest magnitude):
 Integer-valued inputs are exact in every intermediate, so there the bf16
 output must equal the oracle result rounded to bf16, bit for bit.
 """
+import ctypes
 import time
 
 import numpy as np
@@ -348,3 +349,62 @@ def test_withheld_prefix_ends_in_timeout_not_hang():
     finally:
         force_path(0)
     assert_close(f64(o), oracle.recurrent(f64(q), f64(k), f64(v)), 1e-2, "run after a timeout")
+
+
+# ---------------------------------------------------------------- sequence parallelism (LASP+)
+@pytest.mark.gpu
+def test_state_exclusive_prefix():
+    W, nseq, H, d = 4, 3, 2, 128
+    g = torch.randn(W, nseq, H, d, d, device=DEV, generator=torch.Generator(DEV).manual_seed(5))
+    init = torch.randn(nseq, H, d, d, device=DEV, generator=torch.Generator(DEV).manual_seed(6))
+    g64, i64 = g.double().cpu().numpy(), init.double().cpu().numpy()
+    for rank in range(W + 1):
+        for ini in (None, init):
+            out = la.state_exclusive_prefix(g, rank, ini)
+            ref = g64[:rank].sum(0) + (0.0 if ini is None else i64)
+            assert_close(out.cpu().double().numpy(), ref, 1e-6, f"rank {rank}")
+    inplace = init.clone()
+    la.state_exclusive_prefix(g, 2, inplace, out=inplace)
+    assert_close(inplace.cpu().double().numpy(), g64[:2].sum(0) + i64, 1e-6, "in place")
+    status_ok()
+    sh = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    n = nseq * H
+    assert la.la_state_exclusive_prefix(P(g), W, W + 1, n, d, None, P(init), sh) == 1      # rank > world
+    assert la.la_state_exclusive_prefix(P(g), W, 1, n, 100, None, P(init), sh) == 2        # d
+    assert la.la_state_exclusive_prefix(P(g), W, 1, n, d, None, P(g[1]), sh) == 1          # out inside gathered
+    assert la.la_state_exclusive_prefix(ctypes.c_void_p(g.data_ptr() + 4), W, 1, n, d, None, P(init), sh) == 3
+    assert la.la_state_exclusive_prefix(P(g), W, 1, 0, d, None, P(init), sh) == 0          # nothing to do
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("W,B", [(2, 256), (4, 256), (3, 128)])
+def test_lasp_segments_on_one_gpu(W, B):
+    """LASP+ composed from the library calls, the ranks emulated one after another
+    on one GPU (the all-gather is a stack): every segment's output and the final
+    state equal those of the whole sequences."""
+    lengths, H, d = [1500, 777], 2, 128
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, torch.bfloat16, seed=70 + W)
+    init = wl.state_init(len(lengths), H, d, seed=9, device=DEV)
+    rng = np.random.default_rng(W)
+    cuts = [[0, *np.sort(rng.choice(np.arange(1, L), size=W - 1, replace=False)).tolist(), L] for L in lengths]
+    starts = np.cumsum([0] + lengths[:-1])
+    rows = [np.concatenate([np.arange(s0 + c[r], s0 + c[r + 1]) for s0, c in zip(starts, cuts)]) for r in range(W)]
+    segs = []
+    for r in range(W):
+        idx = torch.from_numpy(rows[r]).to(DEV)
+        cu = cu_of([c[r + 1] - c[r] for c in cuts])
+        segs.append((q[idx].contiguous(), k[idx].contiguous(), v[idx].contiguous(), cu))
+    gathered = torch.stack([la.state_from_prefill(kr, vr, cu) for _, kr, vr, cu in segs])
+    o = torch.empty_like(q)
+    for r, (qr, kr, vr, cu) in enumerate(segs):
+        start = la.state_exclusive_prefix(gathered, r, init)
+        o[torch.from_numpy(rows[r]).to(DEV)] = la.prefill(qr, kr, vr, cu, B=B, init_state=start)
+    final = la.state_exclusive_prefix(gathered, W, init)
+    status_ok()
+    cu_all = cu_of(lengths).cpu().numpy()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v), cu_all, init=init.cpu().double().numpy())
+    assert_close(f64(o), ref, TOL[torch.bfloat16], "LASP+ output")
+    ref_state = oracle.state(f64(k), f64(v), cu_all, init=init.cpu().double().numpy())
+    assert_close(final.cpu().double().numpy(), ref_state, 1e-5, "LASP+ final state")
