@@ -32,8 +32,8 @@
 // and state MMA (2 of 16 KB), a Q sub-unit until its scores and inter-block
 // MMA (2 of 32 KB); together they keep about one block of loads in flight.
 // Roles (640 threads):
-//   warp 0 (lane 0)  TMA producer of K and V chunks, warp 2 (lane 0) of Q
-//                    sub-units
+//   warp 0 (lane 0)  TMA producer of Q sub-units, K and V chunks: one
+//                    non-blocking event loop over the three rings
 //   warp 1 (lane 0)  tcgen05 issuer A: score MMAs and state MMAs (chunk by
 //                    chunk as they land), a non-blocking event loop
 //   warp 3 (lane 0)  tcgen05 issuer B: inter-block and PV MMAs, in item order
@@ -43,9 +43,15 @@
 //                    goes through an mbarrier (a score buffer is rewritten only
 //                    after the PV that read it has completed).
 //   warps 4-7, 8-11  scores -> P, keys 0-63 and 64-127 of every item
-//   warps 12-15      state copy-out: TMEM fp32 (+ S0) -> bf16 shared operand
-//   warps 16-19      O epilogue: TMEM -> bf16 -> swizzled staging -> TMA store (a
-//                    ragged last sub-unit of a sequence by masked direct stores)
+//   warps 12-15      state copy-out: TMEM fp32 -> bf16 shared operand (S0, when
+//                    given, is stored into the accumulator at a work item's start)
+//   warps 16-19      O epilogue: TMEM -> bf16 -> 16-byte stores of each row
+//                    (masked for a ragged last sub-unit of a sequence)
+// The instruction working set of the 20 warps is what limits the block rate
+// once many SMs run the kernel (instruction fetch stalls grow with the number
+// of SMs), so cold paths (finding the next work item, the waiting loop of a
+// bounded wait, trace stamps) are out of line and the score masking has a
+// single code path.
 // Every wait is bounded (globaltimer); on expiry the CTA records
 // LA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
 #pragma once
@@ -84,19 +90,12 @@ constexpr uint32_t KH_BYTES = KC * 64 * 2;       // 16 KB: 128 keys x 64 columns
 constexpr uint32_t K_BYTES = 2 * KH_BYTES;       // 32 KB
 constexpr uint32_t V_BYTES = KC * DV * 2;        // 16 KB
 constexpr uint32_t SB_BYTES = D * DV * 2;        // 16 KB: bf16 KV_b, 128 rows x 64 columns
-#ifndef LA_CHAIN_DIRECT_O
-#define LA_CHAIN_DIRECT_O 1
-#endif
-// O staging for the TMA store, 128 rows x 64 columns (16 KB), unless O rows are
-// stored directly from registers.
-constexpr uint32_t STG_BYTES = LA_CHAIN_DIRECT_O ? 0 : UM * DV * 2;
 
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + NQ * Q_BYTES;
 constexpr uint32_t OFF_V = OFF_K + NK * K_BYTES;
 constexpr uint32_t OFF_SB = OFF_V + NV * V_BYTES;
-constexpr uint32_t OFF_STG = OFF_SB + SB_BYTES;
-constexpr uint32_t OFF_BAR = OFF_STG + STG_BYTES;
+constexpr uint32_t OFF_BAR = OFF_SB + SB_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;   // + barriers + 1 KB alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
@@ -118,7 +117,6 @@ struct Bars {
     uint64_t kv_ready;        // issuer -> state group: KV accumulator holds the next block's prefix
     uint64_t kv_read[4];      // state group -> issuer: accumulator read for block n (n % 4)
     uint64_t sb_full, sb_empty;
-    uint64_t grp;             // bounded barrier of the epilogue group
     uint64_t drain, drain_b;
     uint32_t tmem_base;
     int abort_flag;
@@ -131,7 +129,7 @@ struct Params {
     const int32_t* order;     // [nseq] sequences, longest first
     const Control* ctrl;
     const float* init;        // [nseq][H][D][D] carried-in state, or nullptr
-    int H, B, nseq;
+    int H, B, log2B, nseq;
     uint64_t wait_ns;
     long long suppress_item;  // test hook: this work item never hands over its second block's prefix (-1: none)
     uint64_t* trace;          // optional [gridDim.x][trace_blocks][kTraceEvents] clock64 stamps, or nullptr
@@ -159,11 +157,58 @@ enum TraceEvent {
     TR_PVL = 15,       // issuer: last PV MMA issued
     kTraceEvents = 16
 };
+// The stamps cost instruction-cache space in every role, so they are compiled
+// only into trace builds (-DLA_CHAIN_TRACE); otherwise a trace buffer is ignored.
+#ifdef LA_CHAIN_TRACE
 #define LA_CTRACE(n, ev)                                                                                   \
     do {                                                                                                   \
         if (p.trace && (int)(n) < p.trace_blocks)                                                          \
             p.trace[((int64_t)blockIdx.x * p.trace_blocks + (n)) * kTraceEvents + (ev)] = clock64();       \
     } while (0)
+#else
+#define LA_CTRACE(n, ev) do {} while (0)
+#endif
+
+// The block a cursor is at: its work item (w, seq, h, the sequence's first
+// token tok_s and length len) and, within it, block b with its first token,
+// rows, sub-units Rb and whether its K^T V is needed by a later block (more).
+// len = 0: no block left.
+struct Blk { int w, seq, h, tok_s, len, b, tok0, rows, Rb, more; };
+
+// The block after `c` (the first block of the next work item with tokens,
+// from w + step on, after the last block of one); with `first`, the CTA's first
+// block. Out of line: every role's cursor shares this one copy.
+__device__ __noinline__ Blk next_blk(Blk c, bool first, int step, int nitems, const int32_t* order,
+                                     const SeqEntry* seqs, int H, int log2B) {
+    const int bs = 1 << log2B;
+    int nb = (c.len + bs - 1) >> log2B;
+    if (!first && c.b + 1 < nb) {
+        ++c.b;
+    } else {
+        int w = first ? c.w : c.w + step;
+        c.len = 0;
+        for (; w < nitems; w += step) {
+            const unsigned pair = (unsigned)w >> 1;
+            const int seq = order[pair / (unsigned)H];
+            const SeqEntry e = seqs[seq];
+            if (e.len > 0) {
+                c.seq = seq;
+                c.h = (int)(pair % (unsigned)H);
+                c.tok_s = e.tok0;
+                c.len = e.len;
+                break;
+            }
+        }
+        c.w = w;
+        c.b = 0;
+        nb = (c.len + bs - 1) >> log2B;
+    }
+    c.tok0 = c.tok_s + (c.b << log2B);
+    c.rows = min(bs, c.len - (c.b << log2B));
+    c.Rb = (c.rows + UM - 1) / UM;
+    c.more = c.b + 1 < nb;
+    return c;
+}
 
 // Walks this CTA's work items -> blocks -> items in the order every role uses,
 // with the running counters that index the rings: n (blocks), q0 (Q
@@ -172,10 +217,8 @@ enum TraceEvent {
 // 128-key chunks; its items are (0,0), (0,1), (1,1) when Rb = 2 and (0,0)
 // when Rb = 1.
 struct Cursor {
-    int64_t w, nitems;
-    int step;
-    int seq, h, half, tok_s, len, nb;    // work item
-    int b, tok0, rows, Rb;               // block
+    Blk bk;
+    int w, seq, h, half, tok0, rows, Rb, b;
     bool add_state;                      // the block's K^T V is needed (not the last block)
     uint32_t n, q0, kc0, o0;
     int k;                               // item within the block
@@ -192,51 +235,36 @@ struct Cursor {
             r = 0;
         }
     }
-    __device__ __forceinline__ void load_block(const Params& p) {
-        tok0 = tok_s + b * p.B;
-        rows = min(p.B, len - b * p.B);
-        Rb = (rows + UM - 1) / UM;
-        add_state = b + 1 < nb;
+    __device__ __forceinline__ void take(const Params& p, bool first) {
+        bk = next_blk(bk, first, gridDim.x, 2 * p.nseq * p.H, p.order, p.seqs, p.H, p.log2B);   // 2 nseq H < 2^31
+        valid = bk.len > 0;
+        w = bk.w;
+        seq = bk.seq;
+        h = bk.h;
+        half = bk.w & 1;
+        tok0 = bk.tok0;
+        rows = bk.rows;
+        Rb = bk.Rb;
+        b = bk.b;
+        add_state = bk.more != 0;
         k = 0;
         set_item();
     }
-    __device__ __forceinline__ bool load_work(const Params& p) {
-        for (; w < nitems; w += step) {
-            const int64_t pair = w >> 1;
-            seq = p.order[pair / p.H];
-            h = (int)(pair % p.H);
-            half = (int)(w & 1);
-            const SeqEntry e = p.seqs[seq];
-            tok_s = e.tok0;
-            len = e.len;
-            if (len > 0) {
-                nb = (len + p.B - 1) / p.B;
-                b = 0;
-                load_block(p);
-                return true;
-            }
-        }
-        return false;
-    }
     __device__ __forceinline__ void init(const Params& p) {
-        w = blockIdx.x;
-        step = gridDim.x;
-        nitems = (int64_t)p.nseq * p.H * 2;
         n = q0 = kc0 = o0 = 0;
         i = 0;
-        valid = p.ctrl->ok && load_work(p);
+        bk.w = blockIdx.x;
+        bk.len = 0;
+        bk.b = 0;
+        if (p.ctrl->ok) take(p, true);
+        else valid = false;
     }
     __device__ __forceinline__ void next_block(const Params& p) {
         ++n;
         q0 += Rb;
         kc0 += Rb;
         if (Rb == 2) ++o0;
-        if (++b < nb) {
-            load_block(p);
-            return;
-        }
-        w += step;
-        valid = load_work(p);
+        take(p, false);
     }
     __device__ __forceinline__ void next_item(const Params& p) {
         ++i;
@@ -261,8 +289,7 @@ struct Cursor {
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                     const Params p) {
+                     const __grid_constant__ CUtensorMap tmV, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -283,7 +310,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         for (int i = 0; i < 4; ++i) mbar_init(&bars->kv_read[i], 128);
         mbar_init(&bars->sb_full, 128);
         mbar_init(&bars->sb_empty, 1);
-        mbar_init(&bars->grp, 128);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->drain_b, 1);
         bars->abort_flag = 0;
@@ -294,52 +320,79 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV); prefetch_tmap(&tmO);
+        prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 0 || warp == 2) {
-        // ================================================================ TMA producers
+    if (warp == 0) {
+        // ================================================================ TMA producer (Q, K, V)
+        // One thread, three streams in a non-blocking event loop: each issues its next
+        // load as soon as that load's stage is free, so no stream waits behind another.
         if (lane == 0) {
-            const bool kv_role = warp == 0;
             const uint64_t once = policy_evict_first();      // V: read by this CTA only
-            Cursor c;
-            c.init(p);
+            Cursor cq, ck, cv;
+            cq.init(p);
+            ck.init(p);
+            cv.init(p);
+            int rq = 0, rk = 0, rv = 0;                      // sub-unit / chunk within each stream's block
             uint32_t k_issued = 0, v_issued = 0, q_issued = 0;   // loads issued (ring indices)
             bool ok = true;
-            while (ok && c.valid) {
-                for (int r = 0; ok && r < c.Rb; ++r) {      // chunk r's keys / sub-unit r's query rows
-                    const int t = c.tok0 + UM * r;
-                    if (kv_role) {
-                        const uint32_t kc = c.kc0 + r;
-                        if (!wait_bar(&bars->k_empty[kc % NK], ((kc / NK) & 1) ^ 1, ab)) { ok = false; break; }
-                        uint8_t* kd = smem + OFF_K + (kc % NK) * K_BYTES;
-                        mbar_expect_tx(&bars->k_full[kc % NK], K_BYTES);
-                        tma_load_3d(kd, &tmK, &bars->k_full[kc % NK], 0, c.h, t);
-                        tma_load_3d(kd + KH_BYTES, &tmK, &bars->k_full[kc % NK], 64, c.h, t);
-                        k_issued = kc + 1;
-                        if (r == 0) LA_CTRACE(c.n, TR_KV0);
-                        if (!wait_bar(&bars->v_empty[kc % NV], ((kc / NV) & 1) ^ 1, ab)) { ok = false; break; }
-                        mbar_expect_tx(&bars->v_full[kc % NV], V_BYTES);
-                        tma_load_3d_hint(smem + OFF_V + (kc % NV) * V_BYTES, &tmV, &bars->v_full[kc % NV],
-                                         DV * c.half, c.h, t, once);
-                        v_issued = kc + 1;
-                        if (r == c.Rb - 1) LA_CTRACE(c.n, TR_KVL);
-                    } else {
-                        const uint32_t qc = c.q0 + r;
-                        if (!wait_bar(&bars->q_empty[qc % NQ], ((qc / NQ) & 1) ^ 1, ab)) { ok = false; break; }
+            uint32_t idle = 0;
+            uint64_t t_idle = 0;
+            while (cq.valid || ck.valid || cv.valid) {
+                bool prog = false;
+                if (cq.valid) {
+                    const uint32_t qc = cq.q0 + rq;
+                    if (mbar_test_wait(&bars->q_empty[qc % NQ], ((qc / NQ) & 1) ^ 1)) {
+                        const int t = cq.tok0 + UM * rq;
                         uint8_t* qd = smem + OFF_Q + (qc % NQ) * Q_BYTES;
                         mbar_expect_tx(&bars->q_full[qc % NQ], Q_BYTES);
-                        tma_load_3d(qd, &tmQ, &bars->q_full[qc % NQ], 0, c.h, t);
-                        tma_load_3d(qd + QH_BYTES, &tmQ, &bars->q_full[qc % NQ], 64, c.h, t);
+                        tma_load_3d(qd, &tmQ, &bars->q_full[qc % NQ], 0, cq.h, t);
+                        tma_load_3d(qd + QH_BYTES, &tmQ, &bars->q_full[qc % NQ], 64, cq.h, t);
                         q_issued = qc + 1;
-                        if (r == 0) LA_CTRACE(c.n, TR_Q0);
+                        if (rq == 0) LA_CTRACE(cq.n, TR_Q0);
+                        if (++rq == cq.Rb) { rq = 0; cq.next_block(p); }
+                        prog = true;
                     }
                 }
-                c.next_block(p);
+                if (ck.valid) {
+                    const uint32_t kc = ck.kc0 + rk;
+                    if (mbar_test_wait(&bars->k_empty[kc % NK], ((kc / NK) & 1) ^ 1)) {
+                        const int t = ck.tok0 + KC * rk;
+                        uint8_t* kd = smem + OFF_K + (kc % NK) * K_BYTES;
+                        mbar_expect_tx(&bars->k_full[kc % NK], K_BYTES);
+                        tma_load_3d(kd, &tmK, &bars->k_full[kc % NK], 0, ck.h, t);
+                        tma_load_3d(kd + KH_BYTES, &tmK, &bars->k_full[kc % NK], 64, ck.h, t);
+                        k_issued = kc + 1;
+                        if (rk == 0) LA_CTRACE(ck.n, TR_KV0);
+                        if (++rk == ck.Rb) { rk = 0; ck.next_block(p); }
+                        prog = true;
+                    }
+                }
+                if (cv.valid) {
+                    const uint32_t kc = cv.kc0 + rv;
+                    if (mbar_test_wait(&bars->v_empty[kc % NV], ((kc / NV) & 1) ^ 1)) {
+                        const int t = cv.tok0 + KC * rv;
+                        mbar_expect_tx(&bars->v_full[kc % NV], V_BYTES);
+                        tma_load_3d_hint(smem + OFF_V + (kc % NV) * V_BYTES, &tmV, &bars->v_full[kc % NV],
+                                         DV * cv.half, cv.h, t, once);
+                        v_issued = kc + 1;
+                        if (rv == cv.Rb - 1) LA_CTRACE(cv.n, TR_KVL);
+                        if (++rv == cv.Rb) { rv = 0; cv.next_block(p); }
+                        prog = true;
+                    }
+                }
+                if (prog) {
+                    idle = 0;
+                } else if ((++idle & 63u) == 0) {
+                    if (ab.raised()) { *ab.cta = 1; ok = false; break; }
+                    const uint64_t now = globaltimer_ns();
+                    if (idle == 64) t_idle = now;
+                    else if (now - t_idle > ab.limit_ns) { ab.raise(); ok = false; break; }
+                }
             }
             // On abort, wait (bounded) for this producer's copies still in flight
             // into shared memory: only the latest load of each stage can be pending.
@@ -350,12 +403,9 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         while (!mbar_try_wait(&full[i % nst], (i / nst) & 1) && globaltimer_ns() - t0 < 100000000ull) {}
                     }
                 };
-                if (kv_role) {
-                    drain(bars->k_full, k_issued, NK);
-                    drain(bars->v_full, v_issued, NV);
-                } else {
-                    drain(bars->q_full, q_issued, NQ);
-                }
+                drain(bars->q_full, q_issued, NQ);
+                drain(bars->k_full, k_issued, NK);
+                drain(bars->v_full, v_issued, NV);
             }
         }
     } else if (warp == 1 || warp == 3) {
@@ -421,7 +471,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
                                 for (int s = 0; s < KC / 16; ++s)
                                     mma_ss(tmem + TM_KV, a + ((s * 2048) >> 4), b + ((s * 2048) >> 4), IDESC_KV,
-                                           (dc.b > 0 || dc.j > 0 || s > 0));
+                                           (dc.b > 0 || dc.j > 0 || s > 0 || p.init != nullptr));
                                 if (dc.j == dc.Rb - 1) {
                                     tc_commit(&bars->kv_ready);
                                     LA_CTRACE(dc.n, TR_KVR);
@@ -515,17 +565,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 uint32_t a[32];
                 tmem_ld_x32(ts + 32 * hh, a);
                 tmem_wait_ld();
-                if (lim >= 63) {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int c0 = 32 * hh + 2 * q;
-                        pk[16 * hh + q] = pack_bf16x2(c0 <= lim ? __uint_as_float(a[2 * q]) : 0.f,
-                                                      c0 + 1 <= lim ? __uint_as_float(a[2 * q + 1]) : 0.f);
-                    }
+                for (int q = 0; q < 16; ++q) {
+                    const int c0 = 32 * hh + 2 * q;
+                    pk[16 * hh + q] = pack_bf16x2(c0 <= lim ? __uint_as_float(a[2 * q]) : 0.f,
+                                                  c0 + 1 <= lim ? __uint_as_float(a[2 * q + 1]) : 0.f);
                 }
             }
             tmem_st_x32(ts, pk);             // P of these 64 keys over the first 32 of their columns
@@ -548,39 +592,55 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         Cursor c;
         c.init(p);
         while (ok && c.valid) {
-            // KV_b (+ S0) -> bf16 operand of the inter-block product (row m, 64 columns)
+            // KV_b -> bf16 operand of the inter-block product (row m, 64 columns)
+            uint32_t pk[32];
             if (c.b > 0) {
                 if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
                 ++kvc;
                 if (wt == 0) LA_CTRACE(c.n, TR_XR);
                 tc_fence_after();
-            }
-            const float* s0 = p.init ? p.init + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half : nullptr;
-            uint32_t pk[32];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t a[32];
-                if (c.b > 0) {
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a[32];
                     tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
                     tmem_wait_ld();
+                    if (hh == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&bars->kv_read[c.n & 3]);    // the accumulator may take this block's keys
+                    }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                }
+            } else {
+                // A work item's first block: KV_0 = S0 (zero without a carried-in state).
+                // S0 also seeds the accumulator, which the state MMAs then add onto, so
+                // later prefixes already include it.
+                if (p.init) {
+                    const float* s0 = p.init + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t a[32];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 v = __ldg(reinterpret_cast<const float4*>(s0 + 32 * hh) + q);
+                            a[4 * q] = __float_as_uint(v.x);
+                            a[4 * q + 1] = __float_as_uint(v.y);
+                            a[4 * q + 2] = __float_as_uint(v.z);
+                            a[4 * q + 3] = __float_as_uint(v.w);
+                        }
+                        tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                    }
+                    tmem_wait_st();
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) a[q] = 0u;
+                    for (int q = 0; q < 32; ++q) pk[q] = 0u;
                 }
-                if (hh == 1) {
-                    tc_fence_before();
-                    mbar_arrive(&bars->kv_read[c.n & 3]);    // the accumulator may take this block's keys
-                }
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    float x0 = __uint_as_float(a[2 * q]), x1 = __uint_as_float(a[2 * q + 1]);
-                    if (s0) {
-                        const float2 v = __ldg(reinterpret_cast<const float2*>(s0 + 32 * hh + 2 * q));
-                        x0 += v.x;
-                        x1 += v.y;
-                    }
-                    pk[16 * hh + q] = pack_bf16x2(x0, x1);
-                }
+                tc_fence_before();
+                mbar_arrive(&bars->kv_read[c.n & 3]);            // the accumulator may take this block's keys
             }
             if (!warp_all(wait_bar(&bars->sb_empty, (c.n & 1) ^ 1, ab))) { ok = false; break; }
 #pragma unroll
@@ -598,10 +658,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const int m = quad * 32 + lane;                  // TMEM lane: query row of the sub-unit
         const int wt = threadIdx.x - 512;                // 0..127
         const uint32_t lane_base = uint32_t(quad * 32) << 16;
-        uint8_t* stage = smem + OFF_STG;
-        const uint64_t o_pol = policy_evict_first();     // O is never read back
-        uint32_t grp_phase = 0;
-        bool stored = false, ok = true;
+        bool ok = true;
         Cursor c;
         c.init(p);
         while (ok && c.valid) {
@@ -623,22 +680,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
                 tc_fence_before();
                 mbar_arrive(&bars->o_empty[slot]);
-                const int rows = min(UM, c.rows - UM * r);
-                if (!LA_CHAIN_DIRECT_O && rows == UM) {
-                    if (wt == 0 && stored) bulk_wait_read0();    // the previous store has read the staging
-                    if (!warp_all(group_sync(&bars->grp, grp_phase, ab))) { ok = false; break; }
-#pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        *reinterpret_cast<uint4*>(stage + (m >> 3) * 1024 + (m & 7) * 128 + ((g ^ (m & 7)) << 4)) =
-                            make_uint4(ov[4 * g], ov[4 * g + 1], ov[4 * g + 2], ov[4 * g + 3]);
-                    fence_proxy_async_smem();
-                    if (!warp_all(group_sync(&bars->grp, grp_phase, ab))) { ok = false; break; }
-                    if (wt == 0) {
-                        tma_store_3d_hint(&tmO, stage, DV * c.half, c.h, c.tok0 + UM * r, o_pol);
-                        bulk_commit();
-                        stored = true;
-                    }
-                } else if (m < rows) {
+                // row m: 64 bf16 = 128 contiguous bytes of token (tok0 + 128 r + m), head h
+                if (m < c.rows - UM * r) {
                     __nv_bfloat16* orow = p.out + ((int64_t)(c.tok0 + UM * r + m) * p.H + c.h) * D + DV * c.half;
 #pragma unroll
                     for (int g = 0; g < 8; ++g)
@@ -649,7 +692,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             }
             c.next_block(p);
         }
-        if (wt == 0) bulk_wait0();            // every O store has landed before the CTA exits
     }
 
     tc_fence_before();

@@ -53,9 +53,10 @@ thread_local int t_force_path = 0;     // la_debug_set_path: 0 automatic, 1 on-c
 
 Path prefill_path(la_dtype dt, int d, int B, int nseq, int H) {
     if (!use_tensor_cores(dt, d, B)) return Path::simt;
-    if (t_force_path == 1) return Path::chain;
+    if (t_force_path == 1 && 2 * (int64_t)nseq * H < (int64_t(1) << 31)) return Path::chain;
     if (t_force_path == 2) return Path::lookback;
-    return 2 * (int64_t)nseq * H >= kChainMinItems ? Path::chain : Path::lookback;
+    const int64_t items = 2 * (int64_t)nseq * H;
+    return items >= kChainMinItems && items < (int64_t(1) << 31) ? Path::chain : Path::lookback;
 }
 
 // ------------------------------------------------------------------ workspace layouts
@@ -346,11 +347,10 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
                                                  reinterpret_cast<Control*>(ws));
         note_launch();
         if ((s = cuda_check()) != LA_OK) return s;
-        CUtensorMap tq, tk, tv, to;
+        CUtensorMap tq, tk, tv;
         if (!map_tokens(&tq, q, total_tokens, heads, d, la::chain::UM) ||
             !map_tokens(&tk, k, total_tokens, heads, d, la::chain::KC) ||
-            !map_tokens(&tv, v, total_tokens, heads, d, la::chain::KC) ||
-            !map_tokens(&to, o, total_tokens, heads, d, la::chain::UM))
+            !map_tokens(&tv, v, total_tokens, heads, d, la::chain::KC))
             return LA_ERR_CUDA;
         la::chain::Params prm;
         prm.out = static_cast<__nv_bfloat16*>(o);
@@ -360,6 +360,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
         prm.init = init_state;
         prm.H = heads;
         prm.B = B;
+        prm.log2B = B == 256 ? 8 : 7;
         prm.nseq = num_seqs;
         prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
         prm.suppress_item = t_suppress_tile;
@@ -374,8 +375,7 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
                                  (int)la::chain::SMEM_BYTES) != cudaSuccess)
             return LA_ERR_CUDA;
         MainKernelTimer timer(st);
-        la::chain::prefill_chain_kernel<<<grid, la::chain::NTHREADS, la::chain::SMEM_BYTES, st>>>(tq, tk, tv, to,
-                                                                                                   prm);
+        la::chain::prefill_chain_kernel<<<grid, la::chain::NTHREADS, la::chain::SMEM_BYTES, st>>>(tq, tk, tv, prm);
         note_launch();
         return cuda_check();
     }

@@ -50,8 +50,10 @@ struct Abort {
     }
 };
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Abort& ab) {
-    if (mbar_try_wait(bar, parity)) return true;
+// The waiting loop of wait_bar, out of line: every role's wait shares one copy of it.
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, volatile int* cta, volatile int* global,
+                                           uint64_t limit_ns) {
+    const Abort ab{cta, global, limit_ns};
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -60,6 +62,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
             if (globaltimer_ns() - t0 > ab.limit_ns) { ab.raise(); return false; }
         }
     }
+}
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Abort& ab) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, ab.cta, ab.global, ab.limit_ns);
 }
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1,
