@@ -213,7 +213,9 @@ la_status la_debug_set_fault(long long suppress_tile, uint64_t wait_ns);
  *    finer steps of the worker roles. The buffer must hold max_tiles * 384
  *    bytes, max_tiles = (ceil(total_tokens / B) + num_seqs) * heads, or the
  *    call records nothing.
- *  - On-chip-state kernel: for each CTA and each block it processes (in
+ *  - On-chip-state kernel, in builds compiled with -DLA_CHAIN_TRACE only (the
+ *    stamps cost instruction-cache space in every role, so a default build
+ *    records nothing): for each CTA and each block it processes (in
  *    order), 16 uint64 SM-clock stamps (clock64) of its roles: [0] Q load,
  *    [1]/[2] first/last K/V load, [3] first score MMA, [4] first PV MMA,
  *    [5]/[7] inter-block MMAs, [6] last state MMA, [8]/[9] first/last P,
