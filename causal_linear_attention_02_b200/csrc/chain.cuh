@@ -139,9 +139,9 @@ struct Params {
 // Phase stamps of the optional per-block trace (la_debug_set_trace), in SM
 // clock cycles (clock64), indexed by the CTA's block counter n.
 enum TraceEvent {
-    TR_Q0 = 0,         // Q producer: first Q sub-unit load of the block issued
-    TR_KV0 = 1,        // K/V producer: chunk 0 load issued
-    TR_KVL = 2,        // K/V producer: last chunk load issued
+    TR_Q0 = 0,         // producer: first Q sub-unit load of the block issued
+    TR_KV0 = 1,        // producer: K chunk 0 load issued
+    TR_KVL = 2,        // producer: last V chunk load issued
     TR_S0 = 3,         // issuer: first score MMA of the block issued
     TR_PV0 = 4,        // issuer: first PV MMA issued (its P was ready)
     TR_C0 = 5,         // issuer: inter-block MMA of sub-unit 0 issued
