@@ -19,7 +19,11 @@ and computes O_t = q_t . S0 + sum_{s <= t, same sequence} (q_t . k_s) v_s
 Parity status: every function here is pinned by the CPU tests in
 ``tests/test_oracle_pins.py`` (closed forms, exact rational brute force, a
 hand-computed golden example, agreement of three independent associations,
-linearity, causality and varlen invariants).
+linearity, causality and varlen invariants). ``backward`` (the gradients of
+L = sum_t dO_t . O_t, the training pass; the pages give the forward only) is
+pinned by central differences through the pinned forward, which are exact
+because O is linear in each input taken alone, by a one-token closed form and
+by the independence of packed sequences.
 """
 from __future__ import annotations
 
@@ -61,6 +65,7 @@ def _load():
             lib.oracle_blocked.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, dp, dp]
             lib.oracle_state.argtypes = [dp, dp, ip, i, i, i, dp, dp]
             lib.oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, i, i, i]
+            lib.oracle_backward.argtypes = [dp, dp, dp, dp, ip, i, i, i, dp, dp, dp, dp, dp]
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -168,6 +173,23 @@ def decode_step(q, k, v, state_in):
     o = np.zeros_like(q)
     _load().oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(st), _ptr(o), batch, H, d)
     return o, st
+
+
+def backward(q, k, v, dout, cu_seqlens=None, init=None):
+    """Gradients (dq, dk, dv, dinit) of L = sum_t dout_t . O_t, O the forward output."""
+    q, k, v = _check_qkv(q, k, v)
+    dout = _f64(dout)
+    if dout.shape != q.shape:
+        raise ValueError("dout must have the shape of q")
+    T, H, d = q.shape
+    cu, cup = _cu(cu_seqlens, T)
+    nseq = cu.size - 1
+    init = _init(init, nseq, H, d)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    dinit = np.zeros((nseq, H, d, d))
+    _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), cup, nseq, H, d, _ptr(init),
+                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dinit))
+    return dq, dk, dv, dinit
 
 
 def num_threads() -> int:

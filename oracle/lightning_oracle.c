@@ -28,7 +28,11 @@
  *                       (same section, and page "首个线性注意力架构的大模型来了…",
  *                       section "4.1 创新的线性注意力", 序列划分 / 双阶段计算);
  *   oracle_state      - the final state sum_s k_s^T v_s (+ S0) per sequence;
- *   oracle_decode_step- one recurrent step on a batch of states.
+ *   oracle_decode_step- one recurrent step on a batch of states;
+ *   oracle_backward   - the gradients of L = sum_t dO_t . O_t with respect to
+ *                       q, k, v and S0 (the training pass; the pages give the
+ *                       forward only, so this is the calculus of the forward
+ *                       definition above, written out).
  *
  * Layout (all row-major, innermost index fastest):
  *   q, k, v, o   : [T][H][d]      tokens of all sequences packed back to back
@@ -202,6 +206,65 @@ void oracle_decode_step(const double* q, const double* k, const double* v,
         for (int j = 0; j < d; ++j) op[j] = 0.0;
         for (int i = 0; i < d; ++i)
             for (int j = 0; j < d; ++j) op[j] += qp[i] * S[(int64_t)i * d + j];
+    }
+}
+
+/*
+ * Gradients of L = sum_t dO_t . O_t, per (sequence, head), from the forward
+ * definition O_t = q_t S_t with S_t = S0 + sum_{s <= t} k_s^T v_s:
+ *   dq_t = dO_t S_t^T                                   (forward pass over t)
+ *   R_s  = sum_{t >= s} q_t^T dO_t                       (reverse pass over s)
+ *   dk_s = v_s R_s^T,   dv_s = k_s R_s,   dS0 = R_start  (R of the whole sequence)
+ * dinit may be NULL; init may be NULL (zero S0).
+ */
+void oracle_backward(const double* q, const double* k, const double* v, const double* dout,
+                     const int32_t* cu_seqlens, int nseq, int H, int d, const double* init,
+                     double* dq, double* dk, double* dv, double* dinit)
+{
+    int64_t npairs = (int64_t)nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int s = (int)(p / H), h = (int)(p % H);
+        int64_t start = cu_seqlens[s], end = cu_seqlens[s + 1];
+        double* S = (double*)calloc((size_t)d * d, sizeof(double));
+        if (init) memcpy(S, state_ptr(init, s, h, H, d), sizeof(double) * d * d);
+        for (int64_t t = start; t < end; ++t) {
+            const double* kt = k + at3(t, h, 0, H, d);
+            const double* vt = v + at3(t, h, 0, H, d);
+            const double* gt = dout + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j) S[(int64_t)i * d + j] += kt[i] * vt[j];
+            double* dqt = dq + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += gt[j] * S[(int64_t)i * d + j];
+                dqt[i] = acc;
+            }
+        }
+        double* R = S;                                   /* reused: reverse state */
+        memset(R, 0, sizeof(double) * d * d);
+        for (int64_t t = end - 1; t >= start; --t) {
+            const double* qt = q + at3(t, h, 0, H, d);
+            const double* kt = k + at3(t, h, 0, H, d);
+            const double* vt = v + at3(t, h, 0, H, d);
+            const double* gt = dout + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j) R[(int64_t)i * d + j] += qt[i] * gt[j];
+            double* dkt = dk + at3(t, h, 0, H, d);
+            double* dvt = dv + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += R[(int64_t)i * d + j] * vt[j];
+                dkt[i] = acc;
+            }
+            for (int j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i) acc += kt[i] * R[(int64_t)i * d + j];
+                dvt[j] = acc;
+            }
+        }
+        if (dinit) memcpy((double*)state_ptr(dinit, s, h, H, d), R, sizeof(double) * d * d);
+        free(S);
     }
 }
 

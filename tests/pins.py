@@ -283,3 +283,69 @@ def pin_resume(impl):
 ALL_PINS = [pin_golden, pin_single_token, pin_onehot, pin_cumsum, pin_bruteforce_exact,
             pin_forms_agree, pin_linearity, pin_causality, pin_varlen, pin_state,
             pin_decode_continuity, pin_resume]
+
+
+# --------------------------------------------------------------------------- backward
+# Pins for ``backward`` (the gradients of L = sum_t dO_t . O_t). The pages
+# give the forward only; these tie the gradients to the forward definition.
+def pin_backward_finite_differences(impl):
+    """Every gradient equals the central difference of L through the forward
+    (``quadratic``). O is linear in each of q, k, v and S0 taken alone, so with a
+    step of 1 the central difference is the derivative exactly, up to rounding."""
+    r = _rng(30)
+    cu = [0, 5, 9]
+    T, H, d = 9, 2, 3
+    q, k, v, do = (r.standard_normal((T, H, d)) for _ in range(4))
+    init = r.standard_normal((2, H, d, d))
+    dq, dk, dv, dinit = impl.backward(q, k, v, do, cu, init)
+    args = {"q": q, "k": k, "v": v, "init": init}
+
+    def loss(a):
+        return float((do * impl.quadratic(a["q"], a["k"], a["v"], cu, init=a["init"])).sum())
+
+    for name, grad in (("q", dq), ("k", dk), ("v", dv), ("init", dinit)):
+        x = args[name]
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            plus, minus = dict(args), dict(args)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += 1.0
+            xm[idx] -= 1.0
+            plus[name], minus[name] = xp, xm
+            fd[idx] = 0.5 * (loss(plus) - loss(minus))
+        _close(grad, fd, 1e-10, f"dL/d{name}")
+
+
+def pin_backward_single_token(impl):
+    """n = 1, O = (q . k) v + q S0: dq = (dO . v) k + S0 dO, dk = (dO . v) q,
+    dv = (q . k) dO, dS0 = q^T dO."""
+    r = _rng(31)
+    H, d = 2, 4
+    q, k, v, do = (r.standard_normal((1, H, d)) for _ in range(4))
+    S0 = r.standard_normal((1, H, d, d))
+    dq, dk, dv, dinit = impl.backward(q, k, v, do, None, S0)
+    for h in range(H):
+        a, b, c, g = q[0, h], k[0, h], v[0, h], do[0, h]
+        _close(dq[0, h], (g @ c) * b + S0[0, h] @ g, 1e-14, "dq, one token")
+        _close(dk[0, h], (g @ c) * a, 1e-14, "dk, one token")
+        _close(dv[0, h], (a @ b) * g, 1e-14, "dv, one token")
+        _close(dinit[0, h], np.outer(a, g), 1e-14, "dS0, one token")
+
+
+def pin_backward_varlen(impl):
+    """Packed sequences: the gradients of each sequence are those of the sequence alone."""
+    r = _rng(32)
+    lengths = [6, 1, 9]
+    T, H, d = sum(lengths), 2, 3
+    q, k, v, do = (r.standard_normal((T, H, d)) for _ in range(4))
+    cu = np.cumsum([0] + lengths)
+    packed = impl.backward(q, k, v, do, cu, None)
+    for s in range(len(lengths)):
+        a, b = cu[s], cu[s + 1]
+        alone = impl.backward(q[a:b], k[a:b], v[a:b], do[a:b], None, None)
+        for name, x, y in zip(("dq", "dk", "dv"), packed[:3], alone[:3]):
+            _close(x[a:b], y, 1e-12, f"{name} of sequence {s}")
+        _close(packed[3][s], alone[3][0], 1e-12, f"dS0 of sequence {s}")
+
+
+BACKWARD_PINS = [pin_backward_finite_differences, pin_backward_single_token, pin_backward_varlen]

@@ -130,6 +130,33 @@ class Twin:
         return self._post(o, d), st
 
 
+    def backward(self, q, k, v, dout, cu_seqlens=None, init=None):
+        """Gradients of L = sum dO . O (restated: forward pass for dq, reverse for the rest)."""
+        q, k, v, g = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+        dinit = np.zeros((len(cu) - 1, H, d, d))
+        for s in range(len(cu) - 1):
+            a, b = cu[s], cu[s + 1]
+            for h in range(H):
+                S = np.zeros((d, d)) if self.bug == "bwd_dq_no_init" else self._init(init, s, h, d)
+                for t in range(a, b):
+                    S = S + np.outer(k[t, h], v[t, h])
+                    dq[t, h] = g[t, h] @ S if self.bug == "bwd_dq_untransposed" else S @ g[t, h]
+                R = np.zeros((d, d))
+                for t in range(b - 1, a - 1, -1):
+                    if self.bug == "bwd_exclusive_reverse":
+                        dk[t, h], dv[t, h] = R @ v[t, h], R.T @ k[t, h]
+                        R = R + np.outer(q[t, h], g[t, h])
+                        continue
+                    R = R + np.outer(q[t, h], g[t, h])
+                    dk[t, h] = R @ v[t, h]
+                    dv[t, h] = R @ k[t, h] if self.bug == "bwd_dv_untransposed" else R.T @ k[t, h]
+                dinit[s, h] = R.T if self.bug == "bwd_dinit_transposed" else R
+        return dq, dk, dv, dinit
+
+
 BUGS = ["exclusive_mask", "anticausal", "transpose_state", "drop_init", "output_before_update",
         "no_inter", "prefix_inclusive", "no_reset", "swap_qk", "scaled", "block_nomask"]
 
@@ -152,3 +179,27 @@ def test_clean_twin_passes_every_pin():
 def test_planted_bug_is_caught(bug):
     failed = _failing_pins(Twin(bug))
     assert failed, f"no pin catches the planted bug {bug!r}"
+
+
+BACKWARD_BUGS = ["bwd_dq_no_init", "bwd_dq_untransposed", "bwd_exclusive_reverse", "bwd_dv_untransposed",
+                 "bwd_dinit_transposed"]
+
+
+def _failing_backward_pins(impl):
+    failed = []
+    for pin in pins.BACKWARD_PINS:
+        try:
+            pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+def test_clean_twin_passes_every_backward_pin():
+    assert _failing_backward_pins(Twin()) == []
+
+
+@pytest.mark.parametrize("bug", BACKWARD_BUGS)
+def test_planted_backward_bug_is_caught(bug):
+    failed = _failing_backward_pins(Twin(bug))
+    assert failed, f"no backward pin catches the planted bug {bug!r}"
