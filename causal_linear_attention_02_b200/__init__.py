@@ -24,9 +24,11 @@ __all__ = [
     "LightningError", "LA_BF16", "LA_FP32", "STATUS", "library_path", "load_library",
     "la_prefill_workspace_size", "la_prefill", "la_prefill_noalloc", "LA_NOALLOC_SCRATCH_BYTES",
     "la_state_workspace_size", "la_state_from_prefill", "la_state_exclusive_prefix",
+    "la_prefill_backward_workspace_size", "la_prefill_backward",
     "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
     "la_launch_count",
-    "prefill", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status", "uses_tensor_cores",
+    "prefill", "prefill_backward", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status",
+    "uses_tensor_cores",
 ]
 
 LA_BF16 = 0
@@ -75,6 +77,11 @@ def load_library():
         lib.la_state_workspace_size.restype = sz
         lib.la_state_from_prefill.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, sz, vp]
         lib.la_state_from_prefill.restype = i32
+        lib.la_prefill_backward_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+        lib.la_prefill_backward_workspace_size.restype = sz
+        lib.la_prefill_backward.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
+                                            sz, vp]
+        lib.la_prefill_backward.restype = i32
         lib.la_state_exclusive_prefix.argtypes = [vp, i32, i32, i64, i32, vp, vp, vp]
         lib.la_state_exclusive_prefix.restype = i32
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
@@ -128,6 +135,17 @@ def la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dt
                           workspace, workspace_bytes, stream) -> int:
     return int(load_library().la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype,
                                                     init_state, state_out, workspace, workspace_bytes, stream))
+
+
+def la_prefill_backward_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) -> int:
+    return int(load_library().la_prefill_backward_workspace_size(total_tokens, num_seqs, heads, d, B, dtype))
+
+
+def la_prefill_backward(q, k, v, dout, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state, dq, dk,
+                        dv, dinit_state, workspace, workspace_bytes, stream) -> int:
+    return int(load_library().la_prefill_backward(q, k, v, dout, cu_seqlens, num_seqs, total_tokens, heads, d, B,
+                                                  dtype, init_state, dq, dk, dv, dinit_state, workspace,
+                                                  workspace_bytes, stream))
 
 
 def la_state_exclusive_prefix(gathered, world, rank, n, d, init, out, stream) -> int:
@@ -241,6 +259,40 @@ def prefill(q, k, v, cu_seqlens=None, B: int = 256, init_state=None, out=None, w
                         _stream_handle(stream, q.device))
     _raise(status, "la_prefill")
     return out
+
+
+def prefill_backward(q, k, v, dout, cu_seqlens=None, B: int = 256, init_state=None, need_init_grad=False,
+                     workspace=None, stream=None):
+    """(dq, dk, dv, dinit) of L = sum_t dout_t . O_t for O = prefill(q, k, v, ...) (see
+    la_prefill_backward); dinit is None unless need_init_grad."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _need(t, n, q.device)
+    if q.dim() != 3 or any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, dout)):
+        raise LightningError("q, k, v, dout must share one [T, H, d] shape and dtype", 1)
+    T, H, d = q.shape
+    nseq = 1
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", q.device)
+        if cu_seqlens.dtype != torch.int32:
+            raise LightningError("cu_seqlens must be int32", 1)
+        nseq = cu_seqlens.numel() - 1
+    if init_state is not None:
+        _need(init_state, "init_state", q.device)
+        if init_state.dtype != torch.float32 or tuple(init_state.shape) != (nseq, H, d, d):
+            raise LightningError("init_state must be fp32 [num_seqs, H, d, d]", 1)
+    code = _dtype_code(q.dtype)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dinit = torch.empty((nseq, H, d, d), dtype=torch.float32, device=q.device) if need_init_grad else None
+    ws_bytes = la_prefill_backward_workspace_size(T, nseq, H, d, B, code)
+    if ws_bytes == 0:
+        raise LightningError(f"unsupported prefill shape T={T} H={H} d={d} B={B}", 2)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    status = la_prefill_backward(_p(q), _p(k), _p(v), _p(dout), _p(cu_seqlens), nseq, T, H, d, B, code,
+                                 _p(init_state), _p(dq), _p(dk), _p(dv), _p(dinit), _p(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
+    _raise(status, "la_prefill_backward")
+    return dq, dk, dv, dinit
 
 
 def state_from_prefill(k, v, cu_seqlens=None, init_state=None, out=None, workspace=None, stream=None):

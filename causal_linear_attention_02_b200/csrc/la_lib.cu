@@ -20,6 +20,7 @@
 #include "chain.cuh"
 #include "state.cuh"
 #include "lasp.cuh"
+#include "backward.cuh"
 
 namespace {
 
@@ -298,6 +299,43 @@ la_status check_tokens(int64_t T, int nseq, int H, int d, la_dtype dt, const int
     return LA_OK;
 }
 
+// Workspace of la_prefill_backward: four reversed inputs, one reversed output,
+// S0^T, and the workspaces of the prefill and of the state pass.
+struct BackwardLayout {
+    size_t tensor = 0, off_rk = 0, off_rq = 0, off_rdo = 0, off_rv = 0, off_rout = 0, off_s0t = 0, off_pws = 0,
+           pws = 0, off_sws = 0, sws = 0, total = 0;
+};
+BackwardLayout backward_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt) {
+    BackwardLayout L;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    L.tensor = (size_t)T * H * d * esize(dt);
+    size_t off = 0;
+    L.off_rk = off; off = up(off + L.tensor);
+    L.off_rq = off; off = up(off + L.tensor);
+    L.off_rdo = off; off = up(off + L.tensor);
+    L.off_rv = off; off = up(off + L.tensor);
+    L.off_rout = off; off = up(off + L.tensor);
+    L.off_s0t = off; off = up(off + (size_t)nseq * H * d * d * 4);
+    L.pws = prefill_layout(T, nseq, H, d, B, dt).total;
+    L.off_pws = off; off = up(off + L.pws);
+    L.sws = state_layout(T, nseq, H, d, dt).total;
+    L.off_sws = off; off = up(off + L.sws);
+    L.total = off;
+    return L;
+}
+
+la_status launch_reverse(const void* in, void* out, const int32_t* cu, int nseq, int64_t T, int H, int d, la_dtype dt,
+                         cudaStream_t st) {
+    const int64_t row16 = (int64_t)H * d * esize(dt) / 16;
+    const int sms = num_sms();
+    if (sms <= 0) return LA_ERR_CUDA;
+    const dim3 grid((unsigned)(2 * sms), (unsigned)std::min(nseq, 65535));
+    la::reverse_tokens_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(in), static_cast<uint4*>(out), cu, nseq,
+                                                    T, row16);
+    note_launch();
+    return cuda_check();
+}
+
 }  // namespace
 
 extern "C" {
@@ -537,6 +575,85 @@ la_status la_state_exclusive_prefix(const float* gathered, int world, int rank, 
         reinterpret_cast<float4*>(out));
     note_launch();
     return cuda_check();
+}
+
+size_t la_prefill_backward_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                          la_dtype dtype) {
+    if (la_prefill_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) == 0) return 0;
+    return backward_layout(total_tokens, num_seqs, heads, d, B, dtype).total;
+}
+
+la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout,
+                              const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d, int B,
+                              la_dtype dtype, const float* init_state, void* dq, void* dk, void* dv,
+                              float* dinit_state, void* workspace, size_t workspace_bytes, void* stream) {
+    la_status s = check_tokens(total_tokens, num_seqs, heads, d, dtype, cu_seqlens);
+    if (s != LA_OK) return s;
+    if (!supported_B(B)) return LA_ERR_UNSUPPORTED;
+    const int64_t T = total_tokens;
+    const size_t tb = (size_t)T * heads * d * esize(dtype);
+    const size_t sb = (size_t)num_seqs * heads * d * d * 4;
+    if (T > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return LA_ERR_INVALID_ARGUMENT;
+    for (const void* p : {q, k, v, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+        if (!aligned(p, 16)) return LA_ERR_MISALIGNED;
+    if ((init_state && !aligned(init_state, 16)) || (dinit_state && !aligned(dinit_state, 16))) return LA_ERR_MISALIGNED;
+    const void* outs[3] = {dq, dk, dv};
+    const void* ins[4] = {q, k, v, dout};
+    for (int a = 0; a < 3; ++a) {
+        for (int b = 0; b < 4; ++b)
+            if (overlaps(outs[a], tb, ins[b], tb)) return LA_ERR_INVALID_ARGUMENT;
+        for (int b = a + 1; b < 3; ++b)
+            if (overlaps(outs[a], tb, outs[b], tb)) return LA_ERR_INVALID_ARGUMENT;
+        if (dinit_state && overlaps(dinit_state, sb, outs[a], tb)) return LA_ERR_INVALID_ARGUMENT;
+    }
+    if (dinit_state && init_state && overlaps(dinit_state, sb, init_state, sb)) return LA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (dinit_state && cudaMemsetAsync(dinit_state, 0, sb, st) != cudaSuccess) return LA_ERR_CUDA;
+        return LA_OK;
+    }
+    const BackwardLayout L = backward_layout(T, num_seqs, heads, d, B, dtype);
+    if (!workspace) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
+    if (overlaps(workspace, L.total, dq, tb) || overlaps(workspace, L.total, dk, tb) ||
+        overlaps(workspace, L.total, dv, tb) || (dinit_state && overlaps(workspace, L.total, dinit_state, sb)))
+        return LA_ERR_INVALID_ARGUMENT;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void *rk = ws + L.off_rk, *rq = ws + L.off_rq, *rdo = ws + L.off_rdo, *rv = ws + L.off_rv, *rout = ws + L.off_rout;
+    float* s0t = reinterpret_cast<float*>(ws + L.off_s0t);
+    void* pws = ws + L.off_pws;
+
+    // dQ = prefill(dO, V, K) from S0^T
+    if (init_state) {
+        const dim3 grid((unsigned)(num_seqs * heads), (unsigned)((d + 31) / 32), (unsigned)((d + 31) / 32));
+        la::transpose_states_kernel<<<grid, dim3(32, 8), 0, st>>>(init_state, s0t, d);
+        note_launch();
+        if ((s = cuda_check()) != LA_OK) return s;
+    }
+    if ((s = la_prefill(dout, v, k, dq, cu_seqlens, num_seqs, T, heads, d, B, dtype, init_state ? s0t : nullptr, pws,
+                        L.pws, stream)) != LA_OK)
+        return s;
+    // dV and dK: forward prefills over the reversed sequences, reversed back
+    if ((s = launch_reverse(k, rk, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
+        (s = launch_reverse(q, rq, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
+        (s = launch_reverse(dout, rdo, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
+        (s = launch_reverse(v, rv, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK)
+        return s;
+    if ((s = la_prefill(rk, rq, rdo, rout, cu_seqlens, num_seqs, T, heads, d, B, dtype, nullptr, pws, L.pws, stream)) !=
+            LA_OK ||
+        (s = launch_reverse(rout, dv, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK)
+        return s;
+    if ((s = la_prefill(rv, rdo, rq, rout, cu_seqlens, num_seqs, T, heads, d, B, dtype, nullptr, pws, L.pws, stream)) !=
+            LA_OK ||
+        (s = launch_reverse(rout, dk, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK)
+        return s;
+    // dS0 = state of (Q, dO)
+    if (dinit_state)
+        return la_state_from_prefill(q, dout, cu_seqlens, num_seqs, T, heads, d, dtype, nullptr, dinit_state,
+                                     ws + L.off_sws, L.sws, stream);
+    return LA_OK;
 }
 
 la_status la_get_device_status(void* stream) {

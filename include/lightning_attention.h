@@ -132,6 +132,36 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass of la_prefill (the training pass; the pages give the forward
+ * only, so this is the calculus of its definition). With
+ * S_t = S0 + sum_{s <= t, same sequence} k_s^T v_s, O_t = q_t S_t and
+ * L = sum_t dout_t . O_t:
+ *   dq_t = dout_t S_t^T
+ *   dk_s = v_s R_s^T,  dv_s = k_s R_s,  R_s = sum_{t >= s, same sequence} q_t^T dout_t
+ *   dinit_state = R at each sequence's first token (= sum_t q_t^T dout_t)
+ * Computed with the forward kernels: dq is a prefill of (dout, v, k) from
+ * init_state^T; dv and dk are prefills of (k, q, dout) and (v, dout, q) over
+ * every sequence reversed, reversed back; dinit_state is la_state_from_prefill
+ * of (q, dout). Rounding is that of those prefills (bf16 operands, fp32
+ * accumulation; bf16 outputs for bf16 inputs).
+ *   q, k, v, dout     in   [total_tokens][heads][d], dtype (device)
+ *   init_state        in   fp32 [num_seqs][heads][d][d] or NULL (the forward's S0)
+ *   dq, dk, dv        out  [total_tokens][heads][d], dtype; no overlap with the
+ *                          inputs, each other or the workspace
+ *   dinit_state       out  fp32 [num_seqs][heads][d][d], or NULL (not computed)
+ * Shapes, dtypes and errors as la_prefill; the workspace is
+ * la_prefill_backward_workspace_size bytes (five [T][H][d] tensors plus the
+ * prefill's and the state pass's workspaces), 256-byte aligned, caller-owned.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+size_t la_prefill_backward_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                          la_dtype dtype);
+la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout,
+                              const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d, int B,
+                              la_dtype dtype, const float* init_state, void* dq, void* dk, void* dv,
+                              float* dinit_state, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Sequence parallelism (LASP+): each of `world` ranks holds a contiguous
  * segment of the same sequences, computes its segments' states from a zero
  * state (la_state_from_prefill with init_state = NULL), exchanges them with

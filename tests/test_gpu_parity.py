@@ -408,3 +408,51 @@ def test_lasp_segments_on_one_gpu(W, B):
     assert_close(f64(o), ref, TOL[torch.bfloat16], "LASP+ output")
     ref_state = oracle.state(f64(k), f64(v), cu_all, init=init.cpu().double().numpy())
     assert_close(final.cpu().double().numpy(), ref_state, 1e-5, "LASP+ final state")
+
+
+# ---------------------------------------------------------------- backward (training pass)
+@pytest.mark.parametrize("dtype,d,B", [(torch.bfloat16, 128, 256), (torch.bfloat16, 128, 128),
+                                       (torch.float32, 64, 64)], ids=["bf16-256", "bf16-128", "fp32-64"])
+@pytest.mark.parametrize("with_init", [False, True], ids=["zero-S0", "S0"])
+def test_prefill_backward(dtype, d, B, with_init, tc_path):
+    """dq, dk, dv, dS0 of L = sum dO . O against the oracle's gradients."""
+    if dtype == torch.float32 and tc_path == 2:
+        pytest.skip("fp32 has one path")
+    lengths, H = [700, 0, 1, 1300, 255], 2
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, dtype, seed=80 + d)
+    dout = wl.normal_scaled((T, H, d), d, dtype, 81 + d, device=DEV)
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, d, seed=8, device=DEV) if with_init else None
+    dq, dk, dv, dinit = la.prefill_backward(q, k, v, dout, cu, B=B, init_state=init, need_init_grad=True)
+    status_ok()
+    ref = oracle.backward(f64(q), f64(k), f64(v), f64(dout), cu.cpu().numpy(),
+                          init=None if init is None else init.cpu().double().numpy())
+    for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
+        assert_close(f64(got), want, TOL[dtype], name)
+    assert_close(dinit.cpu().double().numpy(), ref[3], 1e-5, "dS0")
+
+
+@pytest.mark.gpu
+def test_prefill_backward_arguments():
+    T, H, d, B = 300, 2, 128, 256
+    q, k, v = inputs(T, H, d, torch.bfloat16, seed=90)
+    dout = wl.normal_scaled((T, H, d), d, torch.bfloat16, 91, device=DEV)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    sh = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
+    wsb = la.la_prefill_backward_workspace_size(T, 1, H, d, B, la.LA_BF16)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=DEV)
+    call = lambda dq_, ws_bytes=wsb: la.la_prefill_backward(P(q), P(k), P(v), P(dout), None, 1, T, H, d, B,
+                                                             la.LA_BF16, None, P(dq_), P(dk), P(dv), None, P(ws),
+                                                             ws_bytes, sh)
+    assert call(q) == 1                       # dq aliases q
+    assert call(dk) == 1                      # dq aliases dk
+    assert call(dq, wsb - 256) == 4           # workspace too small
+    assert call(dq) == 0
+    status_ok()
+    # no tokens: dS0 = 0
+    z = torch.empty(0, H, d, dtype=torch.bfloat16, device=DEV)
+    _, _, _, dinit = la.prefill_backward(z, z, z, z, need_init_grad=True)
+    status_ok()
+    assert torch.count_nonzero(dinit) == 0
