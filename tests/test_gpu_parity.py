@@ -456,3 +456,23 @@ def test_prefill_backward_arguments():
     _, _, _, dinit = la.prefill_backward(z, z, z, z, need_init_grad=True)
     status_ok()
     assert torch.count_nonzero(dinit) == 0
+
+
+@pytest.mark.gpu
+def test_autograd_function_matches_backward():
+    from causal_linear_attention_02_b200.autograd import lightning_attention
+    lengths, H, d = [513, 300], 2, 128
+    T = sum(lengths)
+    q, k, v = (x.requires_grad_(True) for x in inputs(T, H, d, torch.bfloat16, seed=95))
+    init = wl.state_init(len(lengths), H, d, seed=3, device=DEV).requires_grad_(True)
+    cu = cu_of(lengths)
+    dout = wl.normal_scaled((T, H, d), d, torch.bfloat16, 96, device=DEV)
+    o = lightning_attention(q, k, v, cu, 256, init)
+    o.backward(dout)
+    status_ok()
+    ref = oracle.backward(f64(q), f64(k), f64(v), f64(dout), cu.cpu().numpy(), init=init.detach().cpu().double().numpy())
+    for name, got, want in zip(("dq", "dk", "dv"), (q.grad, k.grad, v.grad), ref[:3]):
+        assert_close(f64(got), want, TOL[torch.bfloat16], name)
+    assert_close(init.grad.cpu().double().numpy(), ref[3], 1e-5, "dS0")
+    assert_close(f64(o.detach()), oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy(),
+                                                   init=init.detach().cpu().double().numpy()), TOL[torch.bfloat16], "O")
