@@ -25,9 +25,10 @@ __all__ = [
     "la_prefill_workspace_size", "la_prefill", "la_prefill_noalloc", "LA_NOALLOC_SCRATCH_BYTES",
     "la_state_workspace_size", "la_state_from_prefill", "la_state_exclusive_prefix",
     "la_prefill_backward_workspace_size", "la_prefill_backward",
+    "la_prefill_with_state_workspace_size", "la_prefill_with_state",
     "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
     "la_launch_count",
-    "prefill", "prefill_backward", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status",
+    "prefill", "prefill_with_state", "prefill_backward", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status",
     "uses_tensor_cores",
 ]
 
@@ -77,6 +78,10 @@ def load_library():
         lib.la_state_workspace_size.restype = sz
         lib.la_state_from_prefill.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, sz, vp]
         lib.la_state_from_prefill.restype = i32
+        lib.la_prefill_with_state_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+        lib.la_prefill_with_state_workspace_size.restype = sz
+        lib.la_prefill_with_state.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        lib.la_prefill_with_state.restype = i32
         lib.la_prefill_backward_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
         lib.la_prefill_backward_workspace_size.restype = sz
         lib.la_prefill_backward.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
@@ -135,6 +140,16 @@ def la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dt
                           workspace, workspace_bytes, stream) -> int:
     return int(load_library().la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype,
                                                     init_state, state_out, workspace, workspace_bytes, stream))
+
+
+def la_prefill_with_state_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) -> int:
+    return int(load_library().la_prefill_with_state_workspace_size(total_tokens, num_seqs, heads, d, B, dtype))
+
+
+def la_prefill_with_state(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state, state_out,
+                          workspace, workspace_bytes, stream) -> int:
+    return int(load_library().la_prefill_with_state(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B,
+                                                    dtype, init_state, state_out, workspace, workspace_bytes, stream))
 
 
 def la_prefill_backward_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) -> int:
@@ -259,6 +274,38 @@ def prefill(q, k, v, cu_seqlens=None, B: int = 256, init_state=None, out=None, w
                         _stream_handle(stream, q.device))
     _raise(status, "la_prefill")
     return out
+
+
+def prefill_with_state(q, k, v, cu_seqlens=None, B: int = 256, init_state=None, out=None, state_out=None,
+                       workspace=None, stream=None):
+    """(O, final state) of packed [T, H, d] q, k, v (see la_prefill_with_state); state_out may be
+    init_state itself to update it in place."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise LightningError("q, k, v must share one [T, H, d] shape and dtype", 1)
+    T, H, d = q.shape
+    nseq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", q.device)
+    if init_state is not None:
+        _need(init_state, "init_state", q.device)
+    code = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    if state_out is None:
+        state_out = torch.empty((nseq, H, d, d), dtype=torch.float32, device=q.device)
+    _need(state_out, "state_out", q.device)
+    ws_bytes = la_prefill_with_state_workspace_size(T, nseq, H, d, B, code)
+    if ws_bytes == 0:
+        raise LightningError(f"unsupported prefill shape T={T} H={H} d={d} B={B}", 2)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    status = la_prefill_with_state(_p(q), _p(k), _p(v), _p(out), _p(cu_seqlens), nseq, T, H, d, B, code,
+                                   _p(init_state), _p(state_out), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
+    _raise(status, "la_prefill_with_state")
+    return out, state_out
 
 
 def prefill_backward(q, k, v, dout, cu_seqlens=None, B: int = 256, init_state=None, need_init_grad=False,

@@ -129,6 +129,9 @@ struct Params {
     const int32_t* order;     // [nseq] sequences, longest first
     const Control* ctrl;
     const float* init;        // [nseq][H][D][D] carried-in state, or nullptr
+    float* state_out;         // [nseq][H][D][D] final states (the state-output instance only)
+    const __nv_bfloat16* k;   // K and V, [T][H][D]: the few tokens of a ragged last chunk past its
+    const __nv_bfloat16* v;   // last full 16-key MMA step (state-output instance only)
     int H, B, log2B, nseq;
     uint64_t wait_ns;
     long long suppress_item;  // test hook: this work item never hands over its second block's prefix (-1: none)
@@ -287,6 +290,11 @@ struct Cursor {
     __device__ __forceinline__ uint32_t ouse(int rr) const { return rr == Rb - 1 ? (n >> 1) : o0; }
 };
 
+// kStateOut: also write each sequence's final state S0 + sum_t k_t^T v_t to
+// p.state_out (the last block runs its state MMAs too; the copy-out group reads
+// the accumulator after them). A separate instance, so the plain prefill's code
+// is unchanged.
+template <bool kStateOut>
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -465,13 +473,18 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                             else ready = false;
                         }
                         if (ready) {
-                            if (dc.add_state) {
+                            if (dc.add_state || kStateOut) {
                                 tc_fence_after();
                                 const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4), b = dv + (((kc % NV) * V_BYTES) >> 4);
+                                // a ragged last chunk: its full 16-key steps only (the copy-out
+                                // group adds the rest); the rows past the sequence end belong to
+                                // the next sequence
+                                const int nsteps = dc.add_state ? KC / 16 : min(KC, dc.rows - KC * dc.j) >> 4;
 #pragma unroll
                                 for (int s = 0; s < KC / 16; ++s)
-                                    mma_ss(tmem + TM_KV, a + ((s * 2048) >> 4), b + ((s * 2048) >> 4), IDESC_KV,
-                                           (dc.b > 0 || dc.j > 0 || s > 0 || p.init != nullptr));
+                                    if (s < nsteps)
+                                        mma_ss(tmem + TM_KV, a + ((s * 2048) >> 4), b + ((s * 2048) >> 4), IDESC_KV,
+                                               (dc.b > 0 || dc.j > 0 || s > 0 || p.init != nullptr));
                                 if (dc.j == dc.Rb - 1) {
                                     tc_commit(&bars->kv_ready);
                                     LA_CTRACE(dc.n, TR_KVR);
@@ -650,6 +663,41 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             fence_proxy_async_smem();
             if (!(c.w == p.suppress_item && c.b == 1)) mbar_arrive(&bars->sb_full);
             if (wt == 0) LA_CTRACE(c.n, TR_SB);
+            if (kStateOut && !c.add_state) {
+                // the work item's last block: its state MMAs complete the final state
+                if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
+                ++kvc;
+                tc_fence_after();
+                float x[DV];
+                // with no carried-in state and fewer than 16 tokens no MMA ever ran
+                const bool none = p.init == nullptr && c.bk.len < 16;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a[32];
+                    tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) x[32 * hh + q] = none ? 0.f : __uint_as_float(a[q]);
+                }
+                // the tokens past the last full 16-key step, on CUDA cores
+                for (int t = c.tok0 + (c.rows & ~15); t < c.tok0 + c.rows; ++t) {
+                    const float ki = __bfloat162float(p.k[((int64_t)t * p.H + c.h) * D + m]);
+                    const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + c.h) * D + DV * c.half);
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const uint4 u = __ldg(vr + g);
+                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            x[8 * g + 2 * e] += ki * __uint_as_float(w[e] << 16);
+                            x[8 * g + 2 * e + 1] += ki * __uint_as_float(w[e] & 0xffff0000u);
+                        }
+                    }
+                }
+                float4* dst = reinterpret_cast<float4*>(p.state_out + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half);
+#pragma unroll
+                for (int q = 0; q < DV / 4; ++q) dst[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            }
             c.next_block(p);
         }
     } else if (warp >= 16) {

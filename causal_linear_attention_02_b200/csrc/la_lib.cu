@@ -299,6 +299,66 @@ la_status check_tokens(int64_t T, int nseq, int H, int d, la_dtype dt, const int
     return LA_OK;
 }
 
+// The on-chip-state prefill (bf16, d = 128): sequence table, then the kernel;
+// with state_out, the instance that also writes the final states.
+la_status launch_chain(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens, int num_seqs,
+                       int64_t total_tokens, int heads, int d, int B, const float* init_state, float* state_out,
+                       uint8_t* ws, const Layout& L, cudaStream_t st) {
+    la_status s;
+    const Control* ctrl = reinterpret_cast<const Control*>(ws);
+    la::SeqEntry* seqs = reinterpret_cast<la::SeqEntry*>(ws + L.off_seqs);
+    int32_t* order = reinterpret_cast<int32_t*>(ws + L.off_order);
+    la::seq_table_kernel<<<1, 1024, 0, st>>>(cu_seqlens, num_seqs, total_tokens, seqs, order,
+                                             reinterpret_cast<Control*>(ws));
+    note_launch();
+    if ((s = cuda_check()) != LA_OK) return s;
+    if (state_out && init_state != state_out) {
+        const int64_t per_seq4 = (int64_t)heads * d * d / 4;
+        const int sms = num_sms();
+        if (sms <= 0) return LA_ERR_CUDA;
+        const int64_t want = ((int64_t)num_seqs * per_seq4 + 255) / 256;
+        la::empty_states_kernel<<<(unsigned)std::min<int64_t>(want, (int64_t)sms * 4), 256, 0, st>>>(
+            seqs, num_seqs, per_seq4, reinterpret_cast<const float4*>(init_state), reinterpret_cast<float4*>(state_out));
+        note_launch();
+        if ((s = cuda_check()) != LA_OK) return s;
+    }
+    CUtensorMap tq, tk, tv;
+    if (!map_tokens(&tq, q, total_tokens, heads, d, la::chain::UM) ||
+        !map_tokens(&tk, k, total_tokens, heads, d, la::chain::KC) ||
+        !map_tokens(&tv, v, total_tokens, heads, d, la::chain::KC))
+        return LA_ERR_CUDA;
+    la::chain::Params prm;
+    prm.out = static_cast<__nv_bfloat16*>(o);
+    prm.seqs = seqs;
+    prm.order = order;
+    prm.ctrl = ctrl;
+    prm.init = init_state;
+    prm.state_out = state_out;
+    prm.k = static_cast<const __nv_bfloat16*>(k);
+    prm.v = static_cast<const __nv_bfloat16*>(v);
+    prm.H = heads;
+    prm.B = B;
+    prm.log2B = B == 256 ? 8 : 7;
+    prm.nseq = num_seqs;
+    prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
+    prm.suppress_item = t_suppress_tile;
+    const int64_t items = 2 * (int64_t)num_seqs * heads;
+    const int sms = num_sms();
+    if (sms <= 0) return LA_ERR_CUDA;
+    const unsigned grid = (unsigned)(items < sms ? items : sms);
+    const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
+    prm.trace = (t_trace && t_trace_bytes >= per_block) ? t_trace : nullptr;
+    prm.trace_blocks = prm.trace ? (int)std::min<size_t>(t_trace_bytes / per_block, 1 << 30) : 0;
+    auto kernel = state_out ? la::chain::prefill_chain_kernel<true> : la::chain::prefill_chain_kernel<false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)la::chain::SMEM_BYTES) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    MainKernelTimer timer(st);
+    kernel<<<grid, la::chain::NTHREADS, la::chain::SMEM_BYTES, st>>>(tq, tk, tv, prm);
+    note_launch();
+    return cuda_check();
+}
+
 // Workspace of la_prefill_backward: four reversed inputs, one reversed output,
 // S0^T, and the workspaces of the prefill and of the state pass.
 struct BackwardLayout {
@@ -336,6 +396,23 @@ la_status launch_reverse(const void* in, void* out, const int32_t* cu, int nseq,
     return cuda_check();
 }
 
+// The host checks of la_prefill's arguments (workspace excluded).
+la_status check_prefill(const void* q, const void* k, const void* v, const void* o, const int32_t* cu_seqlens,
+                        int num_seqs, int64_t total_tokens, int heads, int d, int B, la_dtype dtype,
+                        const float* init_state) {
+    la_status s = check_tokens(total_tokens, num_seqs, heads, d, dtype, cu_seqlens);
+    if (s != LA_OK) return s;
+    if (!supported_B(B)) return LA_ERR_UNSUPPORTED;
+    const size_t tensor_bytes = (size_t)total_tokens * heads * d * esize(dtype);
+    if (total_tokens > 0 && (!q || !k || !v || !o)) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return LA_ERR_MISALIGNED;
+    if (init_state && !aligned(init_state, 16)) return LA_ERR_MISALIGNED;
+    if (overlaps(o, tensor_bytes, q, tensor_bytes) || overlaps(o, tensor_bytes, k, tensor_bytes) ||
+        overlaps(o, tensor_bytes, v, tensor_bytes))
+        return LA_ERR_INVALID_ARGUMENT;
+    return LA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -356,16 +433,9 @@ size_t la_state_workspace_size(int64_t total_tokens, int num_seqs, int heads, in
 la_status la_prefill(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
                      int num_seqs, int64_t total_tokens, int heads, int d, int B, la_dtype dtype,
                      const float* init_state, void* workspace, size_t workspace_bytes, void* stream) {
-    la_status s = check_tokens(total_tokens, num_seqs, heads, d, dtype, cu_seqlens);
+    la_status s = check_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state);
     if (s != LA_OK) return s;
-    if (!supported_B(B)) return LA_ERR_UNSUPPORTED;
     const size_t tensor_bytes = (size_t)total_tokens * heads * d * esize(dtype);
-    if (total_tokens > 0 && (!q || !k || !v || !o)) return LA_ERR_INVALID_ARGUMENT;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return LA_ERR_MISALIGNED;
-    if (init_state && !aligned(init_state, 16)) return LA_ERR_MISALIGNED;
-    if (overlaps(o, tensor_bytes, q, tensor_bytes) || overlaps(o, tensor_bytes, k, tensor_bytes) ||
-        overlaps(o, tensor_bytes, v, tensor_bytes))
-        return LA_ERR_INVALID_ARGUMENT;
     if (total_tokens == 0) return LA_OK;
     const Layout L = prefill_layout(total_tokens, num_seqs, heads, d, B, dtype);
     if (!workspace) return LA_ERR_INVALID_ARGUMENT;
@@ -378,45 +448,8 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     const Control* ctrl = reinterpret_cast<const Control*>(ws);
     const Path path = prefill_path(dtype, d, B, num_seqs, heads);
 
-    if (path == Path::chain) {
-        la::SeqEntry* seqs = reinterpret_cast<la::SeqEntry*>(ws + L.off_seqs);
-        int32_t* order = reinterpret_cast<int32_t*>(ws + L.off_order);
-        la::seq_table_kernel<<<1, 1024, 0, st>>>(cu_seqlens, num_seqs, total_tokens, seqs, order,
-                                                 reinterpret_cast<Control*>(ws));
-        note_launch();
-        if ((s = cuda_check()) != LA_OK) return s;
-        CUtensorMap tq, tk, tv;
-        if (!map_tokens(&tq, q, total_tokens, heads, d, la::chain::UM) ||
-            !map_tokens(&tk, k, total_tokens, heads, d, la::chain::KC) ||
-            !map_tokens(&tv, v, total_tokens, heads, d, la::chain::KC))
-            return LA_ERR_CUDA;
-        la::chain::Params prm;
-        prm.out = static_cast<__nv_bfloat16*>(o);
-        prm.seqs = seqs;
-        prm.order = order;
-        prm.ctrl = ctrl;
-        prm.init = init_state;
-        prm.H = heads;
-        prm.B = B;
-        prm.log2B = B == 256 ? 8 : 7;
-        prm.nseq = num_seqs;
-        prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
-        prm.suppress_item = t_suppress_tile;
-        const int64_t items = 2 * (int64_t)num_seqs * heads;
-        const int sms = num_sms();
-        if (sms <= 0) return LA_ERR_CUDA;
-        const unsigned grid = (unsigned)(items < sms ? items : sms);
-        const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
-        prm.trace = (t_trace && t_trace_bytes >= per_block) ? t_trace : nullptr;
-        prm.trace_blocks = prm.trace ? (int)std::min<size_t>(t_trace_bytes / per_block, 1 << 30) : 0;
-        if (cudaFuncSetAttribute(la::chain::prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)la::chain::SMEM_BYTES) != cudaSuccess)
-            return LA_ERR_CUDA;
-        MainKernelTimer timer(st);
-        la::chain::prefill_chain_kernel<<<grid, la::chain::NTHREADS, la::chain::SMEM_BYTES, st>>>(tq, tk, tv, prm);
-        note_launch();
-        return cuda_check();
-    }
+    if (path == Path::chain)
+        return launch_chain(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, init_state, nullptr, ws, L, st);
 
     const int32_t* seq_blk = reinterpret_cast<const int32_t*>(ws + L.off_seq_blk);
     const BlockEntry* table = reinterpret_cast<const BlockEntry*>(ws + L.off_table);
@@ -575,6 +608,55 @@ la_status la_state_exclusive_prefix(const float* gathered, int world, int rank, 
         reinterpret_cast<float4*>(out));
     note_launch();
     return cuda_check();
+}
+
+size_t la_prefill_with_state_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                            la_dtype dtype) {
+    const size_t a = la_prefill_workspace_size(total_tokens, num_seqs, heads, d, B, dtype);
+    const size_t b = la_state_workspace_size(total_tokens, num_seqs, heads, d, dtype);
+    return (a == 0 || b == 0) ? 0 : std::max(a, b);
+}
+
+la_status la_prefill_with_state(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                                int num_seqs, int64_t total_tokens, int heads, int d, int B, la_dtype dtype,
+                                const float* init_state, float* state_out, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+    la_status s = check_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state);
+    if (s != LA_OK) return s;
+    if (!state_out) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(state_out, 16)) return LA_ERR_MISALIGNED;
+    const size_t tb = (size_t)total_tokens * heads * d * esize(dtype);
+    const size_t sb = (size_t)num_seqs * heads * d * d * 4;
+    // state_out may be init_state itself (the state is read before it is written, per slice)
+    if (init_state && init_state != state_out && overlaps(state_out, sb, init_state, sb)) return LA_ERR_INVALID_ARGUMENT;
+    if (overlaps(state_out, sb, o, tb) || overlaps(state_out, sb, q, tb) || overlaps(state_out, sb, k, tb) ||
+        overlaps(state_out, sb, v, tb))
+        return LA_ERR_INVALID_ARGUMENT;
+    if (workspace && overlaps(workspace, workspace_bytes, state_out, sb)) return LA_ERR_INVALID_ARGUMENT;
+    if (total_tokens > 0 && prefill_path(dtype, d, B, num_seqs, heads) == Path::chain) {
+        // one pass: the prefill kernel's state-output instance
+        const Layout L = prefill_layout(total_tokens, num_seqs, heads, d, B, dtype);
+        if (!workspace) return LA_ERR_INVALID_ARGUMENT;
+        if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
+        if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
+        if (overlaps(workspace, L.total, o, tb)) return LA_ERR_INVALID_ARGUMENT;
+        return launch_chain(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, init_state, state_out,
+                            static_cast<uint8_t*>(workspace), L, reinterpret_cast<cudaStream_t>(stream));
+    }
+    // other paths: the prefill, then the state pass (stream order keeps init_state valid until both read it)
+    if (init_state == state_out && init_state) {
+        // the state pass accumulates in place; the prefill reads S0 first
+        if ((s = la_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state, workspace,
+                            workspace_bytes, stream)) != LA_OK)
+            return s;
+        return la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype, state_out, state_out,
+                                     workspace, workspace_bytes, stream);
+    }
+    if ((s = la_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state, workspace,
+                        workspace_bytes, stream)) != LA_OK)
+        return s;
+    return la_state_from_prefill(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype, init_state, state_out,
+                                 workspace, workspace_bytes, stream);
 }
 
 size_t la_prefill_backward_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,

@@ -237,4 +237,16 @@ __global__ void __launch_bounds__(256) chain_scan_kernel(const float* __restrict
     if (state_out) *reinterpret_cast<float4*>(state_out + ((int64_t)s * H + h) * dd + e) = run;
 }
 
+// Final states of the empty sequences for la_prefill_with_state (the prefill
+// kernel visits only sequences with tokens): S0, or zero without one. One
+// 16-byte group per thread and iteration over [nseq][H][d][d].
+__global__ void __launch_bounds__(256)
+empty_states_kernel(const SeqEntry* seqs, int nseq, int64_t per_seq4, const float4* init, float4* out) {
+    const int64_t total = (int64_t)nseq * per_seq4;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        if (seqs[i / per_seq4].len > 0) continue;
+        out[i] = init ? init[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
 }  // namespace la

@@ -132,6 +132,27 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * la_prefill that also returns each sequence's final state, the state a decode
+ * (or the next chunk of a chunked prefill) continues from:
+ *   o          as la_prefill
+ *   state_out  fp32 [num_seqs][heads][d][d] = init_state + sum_{t in seq} k_t^T v_t
+ * On the on-chip-state path (bf16, d = 128, B in {128, 256}, at least 64
+ * (sequence, head, value-half) work items) this is one pass: the prefill
+ * kernel's accumulator already holds the running state, and the kernel writes
+ * it out after each sequence's last block. Elsewhere it is la_prefill followed
+ * by la_state_from_prefill. state_out may be init_state itself (in-place
+ * update); it must not overlap q, k, v, o or the workspace otherwise. The
+ * workspace is la_prefill_with_state_workspace_size bytes. Errors as
+ * la_prefill, plus LA_ERR_INVALID_ARGUMENT for a NULL state_out.
+ */
+size_t la_prefill_with_state_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                            la_dtype dtype);
+la_status la_prefill_with_state(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                                int num_seqs, int64_t total_tokens, int heads, int d, int B, la_dtype dtype,
+                                const float* init_state, float* state_out, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
  * Backward pass of la_prefill (the training pass; the pages give the forward
  * only, so this is the calculus of its definition). With
  * S_t = S0 + sum_{s <= t, same sequence} k_s^T v_s, O_t = q_t S_t and

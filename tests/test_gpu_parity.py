@@ -476,3 +476,32 @@ def test_autograd_function_matches_backward():
     assert_close(init.grad.cpu().double().numpy(), ref[3], 1e-5, "dS0")
     assert_close(f64(o.detach()), oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy(),
                                                    init=init.detach().cpu().double().numpy()), TOL[torch.bfloat16], "O")
+
+
+# ---------------------------------------------------------------- prefill with the final state
+@pytest.mark.parametrize("lengths,H,B,dtype", [
+    ([5000, 1, 15, 16, 17, 300, 0, 2049], 8, 256, torch.bfloat16),   # on-chip-state path, ragged tails
+    ([1, 7, 130, 255, 256, 257], 16, 128, torch.bfloat16),
+    ([700, 33], 2, 256, torch.bfloat16),                              # block-parallel path (few work items)
+    ([300, 45], 2, 64, torch.float32),                                # SIMT path
+], ids=["onchip-256", "onchip-128", "lookback", "fp32"])
+@pytest.mark.parametrize("with_init", [False, True], ids=["zero-S0", "S0"])
+def test_prefill_with_state(lengths, H, B, dtype, with_init):
+    d = 128 if dtype == torch.bfloat16 else 64
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, dtype, seed=110 + len(lengths))
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, d, seed=11, device=DEV) if with_init else None
+    o, st = la.prefill_with_state(q, k, v, cu, B=B, init_state=init)
+    status_ok()
+    init64 = None if init is None else init.cpu().double().numpy()
+    ref_o, ref_s = oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy(), init=init64, return_state=True)
+    assert_close(f64(o), ref_o, TOL[dtype], "O")
+    assert_close(st.cpu().double().numpy(), ref_s, 1e-5, "final state")
+    if with_init:
+        # in place: the state is updated from itself
+        st2 = init.clone()
+        o2, _ = la.prefill_with_state(q, k, v, cu, B=B, init_state=st2, state_out=st2)
+        status_ok()
+        assert_close(st2.cpu().double().numpy(), ref_s, 1e-5, "final state, in place")
+        assert torch.equal(o2, o)
