@@ -24,6 +24,16 @@ L = sum_t dO_t . O_t, the training pass; the pages give the forward only) is
 pinned by central differences through the pinned forward, which are exact
 because O is linear in each input taken alone, by a one-token closed form and
 by the independence of packed sequences.
+
+``decay_*`` (a per-head decay rate on the state, S_t = lambda S_{t-1} + k_t^T v_t;
+not on the pages, the Lightning Attention-2 form taken in its plainest reading)
+are pinned by reduction to the pinned no-decay functions through an exact
+change of variables (q_t -> lambda^(t+1) q_t, k_s -> lambda^-(s+1) k_s), by
+lambda = 1 and lambda = 0 closed forms, by a discounted cumulative sum computed
+with scipy's IIR filter, and by the splitting of a sequence at any token.
+``feature_map`` (phi(x) = ELU(x) + alpha x, page "MiniMax-M2.5语言模型：Linear
+Attention架构解析与实践", section 2.2) is pinned by torch's ELU and by values
+worked by hand.
 """
 from __future__ import annotations
 
@@ -46,7 +56,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp]
+               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB)
     return _LIB
@@ -66,6 +76,12 @@ def _load():
             lib.oracle_state.argtypes = [dp, dp, ip, i, i, i, dp, dp]
             lib.oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, i, i, i]
             lib.oracle_backward.argtypes = [dp, dp, dp, dp, ip, i, i, i, dp, dp, dp, dp, dp]
+            lib.oracle_decay_quadratic.argtypes = [dp, dp, dp, dp, ip, i, i, i, dp, dp]
+            lib.oracle_decay_recurrent.argtypes = [dp, dp, dp, dp, ip, i, i, i, dp, dp, dp]
+            lib.oracle_decay_blocked.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, dp, dp, dp]
+            lib.oracle_decay_state.argtypes = [dp, dp, ip, i, i, i, dp, dp, dp]
+            lib.oracle_decay_decode_step.argtypes = [dp, dp, dp, dp, dp, i, i, i, dp]
+            lib.oracle_feature_map.argtypes = [dp, dp, ctypes.c_int64, ctypes.c_double]
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -190,6 +206,101 @@ def backward(q, k, v, dout, cu_seqlens=None, init=None):
     _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), cup, nseq, H, d, _ptr(init),
                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dinit))
     return dq, dk, dv, dinit
+
+
+# ---------------------------------------------------------------- decay variant
+# S_t = lambda_h S_{t-1} + k_t^T v_t, o_t = q_t S_t (lambda = 1: the functions above).
+
+def _lam(decay, H):
+    lam = _f64(decay)
+    if lam.shape != (H,):
+        raise ValueError("decay must be [H]")
+    if np.any(~np.isfinite(lam)) or np.any(lam < 0) or np.any(lam > 1):
+        raise ValueError("decay rates must lie in [0, 1]")
+    return lam
+
+
+def decay_quadratic(q, k, v, decay, cu_seqlens=None, init=None):
+    """O_t = lambda^(t-start+1) q_t S0 + sum_{s<=t} lambda^(t-s) (q_t . k_s) v_s, term by term."""
+    q, k, v = _check_qkv(q, k, v)
+    T, H, d = q.shape
+    cu, cup = _cu(cu_seqlens, T)
+    init = _init(init, cu.size - 1, H, d)
+    lam = _lam(decay, H)
+    o = np.zeros_like(q)
+    _load().oracle_decay_quadratic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), cup, cu.size - 1, H, d,
+                                   _ptr(init), _ptr(lam))
+    return o
+
+
+def decay_recurrent(q, k, v, decay, cu_seqlens=None, init=None, return_state=False):
+    """S = lambda S + k^T v; o = q S, token by token. Optionally returns the final state."""
+    q, k, v = _check_qkv(q, k, v)
+    T, H, d = q.shape
+    cu, cup = _cu(cu_seqlens, T)
+    nseq = cu.size - 1
+    init = _init(init, nseq, H, d)
+    lam = _lam(decay, H)
+    o = np.zeros_like(q)
+    st = np.zeros((nseq, H, d, d)) if return_state else None
+    _load().oracle_decay_recurrent(_ptr(q), _ptr(k), _ptr(v), _ptr(o), cup, nseq, H, d,
+                                   _ptr(init), _ptr(lam), _ptr(st))
+    return (o, st) if return_state else o
+
+
+def decay_blocked(q, k, v, decay, B, cu_seqlens=None, init=None, return_state=False):
+    """Block decomposition with decay mask, lambda^(r+1)-scaled inter term and decayed prefix."""
+    q, k, v = _check_qkv(q, k, v)
+    T, H, d = q.shape
+    if int(B) < 1:
+        raise ValueError("B must be >= 1")
+    cu, cup = _cu(cu_seqlens, T)
+    nseq = cu.size - 1
+    init = _init(init, nseq, H, d)
+    lam = _lam(decay, H)
+    o = np.zeros_like(q)
+    st = np.zeros((nseq, H, d, d)) if return_state else None
+    _load().oracle_decay_blocked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), cup, nseq, H, d, int(B),
+                                 _ptr(init), _ptr(lam), _ptr(st))
+    return (o, st) if return_state else o
+
+
+def decay_state(k, v, decay, cu_seqlens=None, init=None):
+    """Final state per (sequence, head): lambda^n S0 + sum_t lambda^(end-1-t) k_t^T v_t."""
+    k, v = _f64(k), _f64(v)
+    if k.ndim != 3 or k.shape != v.shape:
+        raise ValueError("k, v must share one shape [T, H, d]")
+    T, H, d = k.shape
+    cu, cup = _cu(cu_seqlens, T)
+    nseq = cu.size - 1
+    init = _init(init, nseq, H, d)
+    lam = _lam(decay, H)
+    st = np.zeros((nseq, H, d, d))
+    _load().oracle_decay_state(_ptr(k), _ptr(v), cup, nseq, H, d, _ptr(init), _ptr(lam), _ptr(st))
+    return st
+
+
+def decay_decode_step(q, k, v, state_in, decay):
+    """One step S = lambda S + k^T v; o = q S on [batch, H, d]; returns (o, new_state)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    if q.ndim != 3 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one shape [batch, H, d]")
+    batch, H, d = q.shape
+    st = np.array(state_in, dtype=np.float64, copy=True, order="C")
+    if st.shape != (batch, H, d, d):
+        raise ValueError("state must be [batch, H, d, d]")
+    lam = _lam(decay, H)
+    o = np.zeros_like(q)
+    _load().oracle_decay_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(st), _ptr(o), batch, H, d, _ptr(lam))
+    return o, st
+
+
+def feature_map(x, alpha=0.3):
+    """phi(x) = ELU(x) + alpha x elementwise, same shape as x."""
+    x = _f64(x)
+    y = np.zeros_like(x)
+    _load().oracle_feature_map(_ptr(x.reshape(-1)), _ptr(y.reshape(-1)), x.size, float(alpha))
+    return y
 
 
 def num_threads() -> int:

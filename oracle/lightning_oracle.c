@@ -7,7 +7,7 @@
  * helper with the CUDA library.
  *
  * What is computed (the plain definition, no decay, no feature map, no
- * normaliser):
+ * normaliser; the decay variant and the feature map are at the end):
  *
  *     O_t = q_t . S0  +  sum_{s in seq(t), s <= t} (q_t . k_s) v_s
  *
@@ -32,7 +32,10 @@
  *   oracle_backward   - the gradients of L = sum_t dO_t . O_t with respect to
  *                       q, k, v and S0 (the training pass; the pages give the
  *                       forward only, so this is the calculus of the forward
- *                       definition above, written out).
+ *                       definition above, written out);
+ *   oracle_decay_*    - the same forms with a per-head decay on the state (an
+ *                       extension the pages do not give; defined further down);
+ *   oracle_feature_map- the feature map phi one page gives, elementwise.
  *
  * Layout (all row-major, innermost index fastest):
  *   q, k, v, o   : [T][H][d]      tokens of all sequences packed back to back
@@ -46,6 +49,7 @@
  * Parallelism: OpenMP over independent (sequence, head) pairs only; the order
  * of every floating-point sum inside a pair is the plain left-to-right order.
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -265,6 +269,195 @@ void oracle_backward(const double* q, const double* k, const double* v, const do
         }
         if (dinit) memcpy((double*)state_ptr(dinit, s, h, H, d), R, sizeof(double) * d * d);
         free(S);
+    }
+}
+
+/*
+ * ---------------------------------------------------------------- decay variant
+ * Not on the pages: a per-head decay rate lambda_h in [0, 1] on the state, the
+ * Lightning Attention-2 form of the same method, taken in its plainest reading
+ * (lambda = 1 is the method above):
+ *
+ *     S_t = lambda_h S_{t-1} + k_t^T v_t,   S_{start-1} = S0,   o_t = q_t S_t
+ *
+ * so that, written out over a sequence starting at `start`,
+ *
+ *     O_t = lambda^(t-start+1) q_t . S0 + sum_{s in seq(t), s <= t} lambda^(t-s) (q_t . k_s) v_s.
+ *
+ * lam: [H]. Powers are pow(lambda, n) with n >= 0 an integer, pow(0, 0) = 1.
+ */
+
+/* The written-out sum above, term by term. */
+void oracle_decay_quadratic(const double* q, const double* k, const double* v, double* o,
+                            const int32_t* cu_seqlens, int nseq, int H, int d,
+                            const double* init, const double* lam)
+{
+    int64_t npairs = (int64_t)nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int s = (int)(p / H), h = (int)(p % H);
+        int64_t start = cu_seqlens[s], end = cu_seqlens[s + 1];
+        const double* S0 = init ? state_ptr(init, s, h, H, d) : NULL;
+        for (int64_t t = start; t < end; ++t) {
+            double* ot = o + at3(t, h, 0, H, d);
+            for (int j = 0; j < d; ++j) ot[j] = 0.0;
+            if (S0) {
+                double w = pow(lam[h], (double)(t - start + 1));
+                for (int i = 0; i < d; ++i) {
+                    double qi = q[at3(t, h, i, H, d)];
+                    for (int j = 0; j < d; ++j) ot[j] += w * qi * S0[(int64_t)i * d + j];
+                }
+            }
+            for (int64_t u = start; u <= t; ++u) {
+                double score = 0.0;
+                for (int i = 0; i < d; ++i)
+                    score += q[at3(t, h, i, H, d)] * k[at3(u, h, i, H, d)];
+                double w = pow(lam[h], (double)(t - u)) * score;
+                const double* vu = v + at3(u, h, 0, H, d);
+                for (int j = 0; j < d; ++j) ot[j] += w * vu[j];
+            }
+        }
+    }
+}
+
+/* The recurrence itself: S = lambda S + k^T v, then o = q S. */
+void oracle_decay_recurrent(const double* q, const double* k, const double* v, double* o,
+                            const int32_t* cu_seqlens, int nseq, int H, int d,
+                            const double* init, const double* lam, double* state_out)
+{
+    int64_t npairs = (int64_t)nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int s = (int)(p / H), h = (int)(p % H);
+        int64_t start = cu_seqlens[s], end = cu_seqlens[s + 1];
+        double* S = (double*)calloc((size_t)d * d, sizeof(double));
+        if (init) memcpy(S, state_ptr(init, s, h, H, d), sizeof(double) * d * d);
+        for (int64_t t = start; t < end; ++t) {
+            const double* kt = k + at3(t, h, 0, H, d);
+            const double* vt = v + at3(t, h, 0, H, d);
+            const double* qt = q + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j)
+                    S[(int64_t)i * d + j] = lam[h] * S[(int64_t)i * d + j] + kt[i] * vt[j];
+            double* ot = o + at3(t, h, 0, H, d);
+            for (int j = 0; j < d; ++j) ot[j] = 0.0;
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j) ot[j] += qt[i] * S[(int64_t)i * d + j];
+        }
+        if (state_out)
+            memcpy((double*)state_ptr(state_out, s, h, H, d), S, sizeof(double) * d * d);
+        free(S);
+    }
+}
+
+/*
+ * The block decomposition with decay (Lightning Attention-2). For a block of
+ * n tokens starting at b0, with KV the state just before b0 and r = t - b0:
+ *   intra: O_t  = sum_{u=b0..t} lambda^(t-u) (q_t . k_u) v_u       (decay mask)
+ *   inter: O_t += lambda^(r+1) q_t KV
+ *   then   KV   = lambda^n KV + sum_u lambda^(b0+n-1-u) k_u^T v_u
+ */
+void oracle_decay_blocked(const double* q, const double* k, const double* v, double* o,
+                          const int32_t* cu_seqlens, int nseq, int H, int d, int B,
+                          const double* init, const double* lam, double* state_out)
+{
+    int64_t npairs = (int64_t)nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int s = (int)(p / H), h = (int)(p % H);
+        int64_t start = cu_seqlens[s], end = cu_seqlens[s + 1];
+        double* KV = (double*)calloc((size_t)d * d, sizeof(double));
+        if (init) memcpy(KV, state_ptr(init, s, h, H, d), sizeof(double) * d * d);
+        for (int64_t b0 = start; b0 < end; b0 += B) {
+            int64_t b1 = b0 + B < end ? b0 + B : end;
+            for (int64_t t = b0; t < b1; ++t) {
+                double* ot = o + at3(t, h, 0, H, d);
+                for (int j = 0; j < d; ++j) ot[j] = 0.0;
+                for (int64_t u = b0; u <= t; ++u) {
+                    double score = 0.0;
+                    for (int i = 0; i < d; ++i)
+                        score += q[at3(t, h, i, H, d)] * k[at3(u, h, i, H, d)];
+                    double w = pow(lam[h], (double)(t - u)) * score;
+                    for (int j = 0; j < d; ++j) ot[j] += w * v[at3(u, h, j, H, d)];
+                }
+                double w = pow(lam[h], (double)(t - b0 + 1));
+                for (int i = 0; i < d; ++i) {
+                    double qi = w * q[at3(t, h, i, H, d)];
+                    for (int j = 0; j < d; ++j) ot[j] += qi * KV[(int64_t)i * d + j];
+                }
+            }
+            double wn = pow(lam[h], (double)(b1 - b0));
+            for (int64_t x = 0; x < (int64_t)d * d; ++x) KV[x] *= wn;
+            for (int64_t u = b0; u < b1; ++u) {
+                double w = pow(lam[h], (double)(b1 - 1 - u));
+                for (int i = 0; i < d; ++i)
+                    for (int j = 0; j < d; ++j)
+                        KV[(int64_t)i * d + j] += w * k[at3(u, h, i, H, d)] * v[at3(u, h, j, H, d)];
+            }
+        }
+        if (state_out)
+            memcpy((double*)state_ptr(state_out, s, h, H, d), KV, sizeof(double) * d * d);
+        free(KV);
+    }
+}
+
+/* Final state per (sequence, head): lambda^n S0 + sum_t lambda^(end-1-t) k_t^T v_t. */
+void oracle_decay_state(const double* k, const double* v, const int32_t* cu_seqlens,
+                        int nseq, int H, int d, const double* init, const double* lam,
+                        double* state_out)
+{
+    int64_t npairs = (int64_t)nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int s = (int)(p / H), h = (int)(p % H);
+        int64_t start = cu_seqlens[s], end = cu_seqlens[s + 1];
+        double* S = (double*)state_ptr(state_out, s, h, H, d);
+        double w0 = pow(lam[h], (double)(end - start));
+        for (int64_t x = 0; x < (int64_t)d * d; ++x)
+            S[x] = init ? w0 * state_ptr(init, s, h, H, d)[x] : 0.0;
+        for (int64_t t = start; t < end; ++t) {
+            double w = pow(lam[h], (double)(end - 1 - t));
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j)
+                    S[(int64_t)i * d + j] += w * k[at3(t, h, i, H, d)] * v[at3(t, h, j, H, d)];
+        }
+    }
+}
+
+/* One decode step with decay: S <- lambda_h S + k^T v ; o = q S. */
+void oracle_decay_decode_step(const double* q, const double* k, const double* v,
+                              double* state, double* o, int batch, int H, int d,
+                              const double* lam)
+{
+    int64_t npairs = (int64_t)batch * H;
+#pragma omp parallel for schedule(static)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int h = (int)(p % H);
+        double* S = state + p * (int64_t)d * d;
+        const double* qp = q + p * d;
+        const double* kp = k + p * d;
+        const double* vp = v + p * d;
+        double* op = o + p * d;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j)
+                S[(int64_t)i * d + j] = lam[h] * S[(int64_t)i * d + j] + kp[i] * vp[j];
+        for (int j = 0; j < d; ++j) op[j] = 0.0;
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) op[j] += qp[i] * S[(int64_t)i * d + j];
+    }
+}
+
+/*
+ * Feature map of the page "MiniMax-M2.5语言模型：Linear Attention架构解析与实践",
+ * section "2.2 Linear Attention的数学原理" (alpha = 0.3 there):
+ * phi(x) = ELU(x) + alpha x, ELU(x) = x for x > 0 and e^x - 1 otherwise,
+ * applied elementwise to n values.
+ */
+void oracle_feature_map(const double* x, double* y, int64_t n, double alpha)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        double e = x[i] > 0.0 ? x[i] : expm1(x[i]);
+        y[i] = e + alpha * x[i];
     }
 }
 

@@ -349,3 +349,162 @@ def pin_backward_varlen(impl):
 
 
 BACKWARD_PINS = [pin_backward_finite_differences, pin_backward_single_token, pin_backward_varlen]
+
+
+# --------------------------------------------------------------------------- decay variant
+# Pins for ``decay_*``: a per-head decay rate lambda_h on the state,
+#   S_t = lambda_h S_{t-1} + k_t^T v_t,  S_{start-1} = S0,  o_t = q_t S_t.
+# The pages give no decay; this is the Lightning Attention-2 form of the same
+# method in its plainest reading. The pins tie it to the pinned no-decay
+# functions (``quadratic``, ``state``, ``decode_step``) of the same object, to
+# closed forms and to a library IIR filter.
+def _decay_case(seed, lengths=(13, 1, 0, 22), H=3, d=4):
+    r = _rng(seed)
+    T = sum(lengths)
+    q, k, v = (r.standard_normal((T, H, d)) for _ in range(3))
+    init = r.standard_normal((len(lengths), H, d, d))
+    cu = np.cumsum([0, *lengths])
+    return q, k, v, init, cu
+
+
+def _reweight(q, k, cu, lam):
+    """q_t -> lambda^(r+1) q_t and k_s -> lambda^-(r+1) k_s, r the position in the sequence.
+    Then (q'_t . k'_s) = lambda^(t-s) (q_t . k_s) and q'_t S0 = lambda^(t-start+1) q_t S0:
+    the no-decay method on (q', k', v) is the decay method on (q, k, v)."""
+    qw, kw = q.copy(), k.copy()
+    for s in range(len(cu) - 1):
+        for t in range(cu[s], cu[s + 1]):
+            e = t - cu[s] + 1
+            qw[t] *= (lam ** e)[:, None]
+            kw[t] *= (lam ** (-e))[:, None]
+    return qw, kw
+
+
+def pin_decay_change_of_variables(impl):
+    """Every decay form equals the pinned no-decay quadratic form on reweighted q, k."""
+    lam = np.array([0.5, 0.8, 0.97])
+    q, k, v, init, cu = _decay_case(40)
+    qw, kw = _reweight(q, k, cu, lam)
+    want = impl.quadratic(qw, kw, v, cu, init=init)
+    _close(impl.decay_quadratic(q, k, v, lam, cu, init=init), want, 1e-11, "decay quadratic")
+    _close(impl.decay_recurrent(q, k, v, lam, cu, init=init), want, 1e-11, "decay recurrent")
+    for B in (1, 2, 5, 8, 64):
+        _close(impl.decay_blocked(q, k, v, lam, B, cu, init=init), want, 1e-11, f"decay blocked B={B}")
+    # final state: lambda^n (S0 + sum_s lambda^-(r_s+1) k_s^T v_s) = lambda^n state(k', v, S0)
+    n = np.diff(cu)
+    st_want = impl.state(kw, v, cu, init=init) * (lam[None, :] ** n[:, None])[:, :, None, None]
+    _close(impl.decay_state(k, v, lam, cu, init=init), st_want, 1e-11, "decay state")
+    _, st_r = impl.decay_recurrent(q, k, v, lam, cu, init=init, return_state=True)
+    _, st_b = impl.decay_blocked(q, k, v, lam, 4, cu, init=init, return_state=True)
+    _close(st_r, st_want, 1e-11, "decay recurrent final state")
+    _close(st_b, st_want, 1e-11, "decay blocked final state")
+    # decode: lambda S + k^T v = lambda (S + (k / lambda)^T v), o = (lambda q)(S + (k / lambda)^T v)
+    r = _rng(41)
+    dq, dk, dv = (r.standard_normal((2, 3, 4)) for _ in range(3))
+    S = r.standard_normal((2, 3, 4, 4))
+    o_w, s_w = impl.decode_step(dq * lam[None, :, None], dk / lam[None, :, None], dv, S)
+    o, s_new = impl.decay_decode_step(dq, dk, dv, S, lam)
+    _close(o, o_w, 1e-13, "decay decode o")
+    _close(s_new, s_w * lam[None, :, None, None], 1e-13, "decay decode state")
+
+
+def pin_decay_one(impl):
+    """lambda = 1 is the method without decay."""
+    lam = np.ones(3)
+    q, k, v, init, cu = _decay_case(42)
+    want = impl.quadratic(q, k, v, cu, init=init)
+    _close(impl.decay_quadratic(q, k, v, lam, cu, init=init), want, 1e-12, "lambda=1 quadratic")
+    _close(impl.decay_recurrent(q, k, v, lam, cu, init=init), want, 1e-12, "lambda=1 recurrent")
+    _close(impl.decay_blocked(q, k, v, lam, 4, cu, init=init), want, 1e-12, "lambda=1 blocked")
+    _close(impl.decay_state(k, v, lam, cu, init=init), impl.state(k, v, cu, init=init), 1e-12, "lambda=1 state")
+
+
+def pin_decay_zero(impl):
+    """lambda = 0 keeps only the current token: O_t = (q_t . k_t) v_t, S0 unseen even at t = start;
+    the final state is k_last^T v_last (S0 for an empty sequence)."""
+    lam = np.zeros(3)
+    q, k, v, init, cu = _decay_case(43)
+    want = np.einsum("thi,thi->th", q, k)[:, :, None] * v
+    for name, o in (("quadratic", impl.decay_quadratic(q, k, v, lam, cu, init=init)),
+                    ("recurrent", impl.decay_recurrent(q, k, v, lam, cu, init=init)),
+                    ("blocked", impl.decay_blocked(q, k, v, lam, 4, cu, init=init))):
+        _close(o, want, 1e-14, f"lambda=0 {name}")
+    st = impl.decay_state(k, v, lam, cu, init=init)
+    for s in range(len(cu) - 1):
+        for h in range(3):
+            last = cu[s + 1] - 1
+            exp = init[s, h] if cu[s + 1] == cu[s] else np.outer(k[last, h], v[last, h])
+            _close(st[s, h], exp, 1e-14, f"lambda=0 state of sequence {s}")
+    o, sn = impl.decay_decode_step(q[:2], k[:2], v[:2], init[:2], lam)
+    _close(o, want[:2], 1e-14, "lambda=0 decode o")
+    _close(sn, np.einsum("bhi,bhj->bhij", k[:2], v[:2]), 1e-14, "lambda=0 decode state")
+
+
+def pin_decay_discounted_cumsum(impl):
+    """All scores one (q = k = e_0): O_t = sum_{s<=t} lambda^(t-s) v_s + lambda^(t-start+1) S0[0, :],
+    the first-order IIR filter y_t = v_t + lambda y_{t-1}, y_{start-1} = S0[0, :] (scipy's lfilter)."""
+    from scipy.signal import lfilter
+    lam = np.array([0.3, 0.9])
+    lengths = (9, 14)
+    T, H, d = sum(lengths), 2, 3
+    r = _rng(44)
+    q = np.zeros((T, H, d)); q[:, :, 0] = 1.0
+    k = q.copy()
+    v = r.standard_normal((T, H, d))
+    init = r.standard_normal((2, H, d, d))
+    cu = np.cumsum([0, *lengths])
+    want = np.zeros_like(v)
+    for s in range(2):
+        for h in range(H):
+            a, b = cu[s], cu[s + 1]
+            want[a:b, h], _ = lfilter([1.0], [1.0, -lam[h]], v[a:b, h], axis=0, zi=lam[h] * init[s, h, 0][None, :])
+    for name, o in (("quadratic", impl.decay_quadratic(q, k, v, lam, cu, init=init)),
+                    ("recurrent", impl.decay_recurrent(q, k, v, lam, cu, init=init)),
+                    ("blocked B=4", impl.decay_blocked(q, k, v, lam, 4, cu, init=init)),
+                    ("blocked B=16", impl.decay_blocked(q, k, v, lam, 16, cu, init=init))):
+        _close(o, want, 1e-12, f"discounted cumsum ({name})")
+
+
+def pin_decay_split(impl):
+    """Splitting a sequence anywhere: the tail run from the head's final state reproduces the
+    tail rows, and decode steps from the state of a prefix reproduce the following rows."""
+    lam = np.array([0.6, 0.95])
+    r = _rng(45)
+    T, H, d = 21, 2, 4
+    q, k, v = (r.standard_normal((T, H, d)) for _ in range(3))
+    S0 = r.standard_normal((1, H, d, d))
+    full = impl.decay_quadratic(q, k, v, lam, init=S0)
+    for m in (1, 8, 20):
+        st = impl.decay_state(k[:m], v[:m], lam, init=S0)
+        _close(impl.decay_recurrent(q[m:], k[m:], v[m:], lam, init=st), full[m:], 1e-11, f"resume at {m}")
+        _close(impl.decay_blocked(q[m:], k[m:], v[m:], lam, 3, init=st), full[m:], 1e-11, f"resume blocked at {m}")
+    st = impl.decay_state(k[:12], v[:12], lam, init=S0)
+    for t in range(12, T):
+        o, st = impl.decay_decode_step(q[t:t + 1], k[t:t + 1], v[t:t + 1], st, lam)
+        _close(o[0], full[t], 1e-11, f"decay decode at t={t}")
+    _close(st, impl.decay_state(k, v, lam, init=S0), 1e-11, "decay decode final state")
+
+
+DECAY_PINS = [pin_decay_change_of_variables, pin_decay_one, pin_decay_zero, pin_decay_discounted_cumsum,
+              pin_decay_split]
+
+
+# --------------------------------------------------------------------------- feature map
+def pin_feature_map(impl):
+    """phi(x) = ELU(x) + 0.3 x (page "MiniMax-M2.5语言模型：Linear Attention架构解析与实践",
+    section 2.2): torch's ELU plus 0.3 x, and values worked by hand."""
+    import math
+    import torch
+    x = np.concatenate([np.linspace(-30, 30, 601), [-1e-12, 0.0, 1e-12, -700.0, 5e3]])
+    want = torch.nn.functional.elu(torch.from_numpy(x)).numpy() + 0.3 * x
+    _close(impl.feature_map(x), want, 1e-15, "phi against torch ELU")
+    got = impl.feature_map(np.array([0.0, 1.0, 2.0, -1.0, -2.0]))
+    hand = [0.0, 1.3, 2.6, math.exp(-1.0) - 1.0 - 0.3, math.exp(-2.0) - 1.0 - 0.6]
+    np.testing.assert_allclose(got, hand, rtol=1e-15, atol=1e-16, err_msg="phi by hand")
+    tiny = impl.feature_map(np.array([-1e-20]))[0]          # e^x - 1 without cancellation
+    assert abs(tiny + 1.3e-20) <= 1e-15 * 1.3e-20, "phi near zero keeps relative precision"
+    y = impl.feature_map(np.ones((2, 3)) * -0.5, alpha=0.0)
+    _close(y, np.full((2, 3), math.expm1(-0.5)), 1e-15, "alpha = 0 is ELU")
+
+
+FEATURE_PINS = [pin_feature_map]

@@ -203,3 +203,168 @@ def test_clean_twin_passes_every_backward_pin():
 def test_planted_backward_bug_is_caught(bug):
     failed = _failing_backward_pins(Twin(bug))
     assert failed, f"no backward pin catches the planted bug {bug!r}"
+
+
+class DecayTwin(Twin):
+    """numpy restatement of the decay functions, with an optional planted bug; the
+    no-decay functions it inherits are the clean twin's."""
+
+    def __init__(self, bug=None):
+        super().__init__(None)
+        self.dbug = bug
+
+    def _lam(self, lam, h):
+        return lam[0] if self.dbug == "decay_head0" else lam[h]
+
+    def _inter_pow(self, r):
+        return r if self.dbug == "decay_inter_pow_r" else r + 1
+
+    def _intra_pow(self, t, u):
+        return t - u + 1 if self.dbug == "decay_intra_pow_plus1" else t - u
+
+    def decay_quadratic(self, q, k, v, decay, cu_seqlens=None, init=None):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        o = np.zeros_like(q)
+        for s in range(len(cu) - 1):
+            a, b = cu[s], cu[s + 1]
+            for h in range(H):
+                lam = self._lam(decay, h)
+                S0 = self._init(init, s, h, d)
+                for t in range(a, b):
+                    acc = lam ** self._inter_pow(t - a) * (q[t, h] @ S0)
+                    for u in range(a, t + 1):
+                        acc = acc + lam ** self._intra_pow(t, u) * (q[t, h] @ k[u, h]) * v[u, h]
+                    o[t, h] = acc
+        return o
+
+    def decay_recurrent(self, q, k, v, decay, cu_seqlens=None, init=None, return_state=False):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        o = np.zeros_like(q)
+        st = np.zeros((len(cu) - 1, H, d, d))
+        for s in range(len(cu) - 1):
+            for h in range(H):
+                lam = self._lam(decay, h)
+                S = self._init(init, s, h, d)
+                for t in range(cu[s], cu[s + 1]):
+                    if self.dbug == "decay_after_add":
+                        S = lam * (S + np.outer(k[t, h], v[t, h]))
+                    else:
+                        S = lam * S + np.outer(k[t, h], v[t, h])
+                    o[t, h] = q[t, h] @ S
+                st[s, h] = S
+        return (o, st) if return_state else o
+
+    def decay_blocked(self, q, k, v, decay, B, cu_seqlens=None, init=None, return_state=False):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        o = np.zeros_like(q)
+        st = np.zeros((len(cu) - 1, H, d, d))
+        for s in range(len(cu) - 1):
+            a, e = cu[s], cu[s + 1]
+            for h in range(H):
+                lam = self._lam(decay, h)
+                KV = self._init(init, s, h, d)
+                for b0 in range(a, e, B):
+                    b1 = min(b0 + B, e)
+                    n = b1 - b0
+                    r = np.arange(n)
+                    M = np.tril(lam ** np.maximum(self._intra_pow(r[:, None], r[None, :]), 0))
+                    Q, K, V = q[b0:b1, h], k[b0:b1, h], v[b0:b1, h]
+                    o[b0:b1, h] = ((Q @ K.T) * M) @ V + (lam ** self._inter_pow(r))[:, None] * (Q @ KV)
+                    kpow = n - r if self.dbug == "decay_key_pow" else n - 1 - r
+                    blk = (K * (lam ** kpow)[:, None]).T @ V
+                    KV = blk + (KV if self.dbug == "decay_prefix_undecayed" else lam ** n * KV)
+                st[s, h] = KV
+        return (o, st) if return_state else o
+
+    def decay_state(self, k, v, decay, cu_seqlens=None, init=None):
+        k, v = (np.asarray(x, dtype=np.float64) for x in (k, v))
+        T, H, d = k.shape
+        cu = self._cu(T, cu_seqlens)
+        st = np.zeros((len(cu) - 1, H, d, d))
+        for s in range(len(cu) - 1):
+            a, b = cu[s], cu[s + 1]
+            for h in range(H):
+                lam = self._lam(decay, h)
+                n = b - a
+                S = (lam ** (n if self.dbug != "decay_state_init_undecayed" else 0)) * self._init(init, s, h, d)
+                for t in range(a, b):
+                    S = S + lam ** (b - 1 - t) * np.outer(k[t, h], v[t, h])
+                st[s, h] = S
+        return st
+
+    def decay_decode_step(self, q, k, v, state_in, decay):
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        Bt, H, d = q.shape
+        st = np.array(state_in, dtype=np.float64, copy=True)
+        o = np.zeros_like(q)
+        for b in range(Bt):
+            for h in range(H):
+                lam = self._lam(decay, h)
+                if self.dbug == "decay_decode_output_first":
+                    o[b, h] = q[b, h] @ st[b, h]
+                    st[b, h] = lam * st[b, h] + np.outer(k[b, h], v[b, h])
+                else:
+                    st[b, h] = lam * st[b, h] + np.outer(k[b, h], v[b, h])
+                    o[b, h] = q[b, h] @ st[b, h]
+        return o, st
+
+
+DECAY_BUGS = ["decay_head0", "decay_inter_pow_r", "decay_intra_pow_plus1", "decay_after_add", "decay_key_pow",
+              "decay_prefix_undecayed", "decay_state_init_undecayed", "decay_decode_output_first"]
+
+
+def _failing_decay_pins(impl):
+    failed = []
+    for pin in pins.DECAY_PINS:
+        try:
+            pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+def test_clean_decay_twin_passes_every_decay_pin():
+    assert _failing_decay_pins(DecayTwin()) == []
+
+
+@pytest.mark.parametrize("bug", DECAY_BUGS)
+def test_planted_decay_bug_is_caught(bug):
+    failed = _failing_decay_pins(DecayTwin(bug))
+    assert failed, f"no decay pin catches the planted bug {bug!r}"
+
+
+class FeatureTwin:
+    def __init__(self, bug=None):
+        self.bug = bug
+
+    def feature_map(self, x, alpha=0.3):
+        x = np.asarray(x, dtype=np.float64)
+        with np.errstate(over="ignore"):
+            return self._phi(x, alpha)
+
+    def _phi(self, x, alpha):
+        if self.bug == "elu_exp_not_expm1":
+            e = np.where(x > 0, x, np.exp(x) - 1.0)
+        elif self.bug == "elu_plus_one":
+            e = np.where(x > 0, x, np.expm1(x)) + 1.0
+        elif self.bug == "alpha_on_negative_only":
+            return np.where(x > 0, x, np.expm1(x) + alpha * x)
+        else:
+            e = np.where(x > 0, x, np.expm1(np.minimum(x, 0.0)))
+        return e + alpha * x
+
+
+@pytest.mark.parametrize("bug", [None, "elu_exp_not_expm1", "elu_plus_one", "alpha_on_negative_only"])
+def test_feature_map_pin_is_sharp(bug):
+    try:
+        pins.pin_feature_map(FeatureTwin(bug))
+        caught = False
+    except AssertionError:
+        caught = True
+    assert caught == (bug is not None)

@@ -15,6 +15,11 @@ def test_oracle_backward_pin(pin):
     pin(oracle)
 
 
+@pytest.mark.parametrize("pin", pins.DECAY_PINS + pins.FEATURE_PINS, ids=lambda p: p.__name__)
+def test_oracle_decay_and_feature_pin(pin):
+    pin(oracle)
+
+
 def test_oracle_validates_arguments():
     import numpy as np
     q = np.zeros((4, 1, 2))
@@ -24,3 +29,7 @@ def test_oracle_validates_arguments():
         oracle.recurrent(q, q, q, cu_seqlens=[0, 3, 2, 4])  # decreasing
     with pytest.raises(ValueError):
         oracle.blocked(q, q, q, 0)
+    with pytest.raises(ValueError):
+        oracle.decay_recurrent(q, q, q, np.array([1.5]))   # decay rate above 1
+    with pytest.raises(ValueError):
+        oracle.decay_state(q, q, np.array([0.5, 0.5]))     # one rate per head
