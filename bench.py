@@ -59,6 +59,7 @@ def flops_per_token_head(B, d):
 # only while those sources are unchanged; otherwise traffic is null.
 KERNEL_SOURCES = {
     "prefill_chain_kernel": ("chain.cuh", "pipe.cuh", "sm100.cuh", "common.cuh"),
+    "prefill_chain_kernel_decay": ("chain.cuh", "pipe.cuh", "sm100.cuh", "common.cuh", "decay.cuh"),
     "prefill_fused_kernel": ("fused.cuh", "pipe.cuh", "sm100.cuh", "common.cuh"),
     "decode_step_kernel": ("decode.cuh", "common.cuh"),
 }
@@ -280,6 +281,11 @@ def run_cuda(args):
     if not args.no_decode:
         dec = run_decode(la, dev, stream, args, pk, pg, local)
 
+    # ---- decay variant on the same inputs (CUDA-core path), per-head rates of the decay recipe
+    dcy = None
+    if not args.no_decay:
+        dcy = run_decay(la, dev, stream, args, pk, pg, local, q, k, v, o, w)
+
     # ---- end to end through host buffers: H2D q,k,v (pinned) + la_prefill + D2H o, per step
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
@@ -325,6 +331,7 @@ def run_cuda(args):
                          "kernel_ms": kernel_ms,
                          "algorithmic_bytes": alg_bytes},
             "decode": dec,
+            "decay": dcy,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
@@ -382,12 +389,86 @@ def run_decode(la, dev, stream, args, pk, pg, local):
     gbs = (state_bytes + io_bytes) / (kms / 1e3) / 1e9
     if la.device_status() != 0:
         raise RuntimeError("device status after decode")
+    # the same steps with the decay recipe's per-head rates (la_decode_step_decay)
+    decay = wl.decay_rates(H, device=dev)
+    dtimers = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_steps)]
+    for a, b in dtimers:
+        a.record(); b.record()
+    for i in range(3):
+        la.la_decode_step_decay(P(qs[i]), P(ks[i]), P(vs[i]), P(state), P(o), Bt, H, d, la.LA_BF16, P(decay), sh)
+    torch.cuda.synchronize(dev)
+    for i in range(n_steps):
+        la.la_set_kernel_timer(ctypes.c_void_p(dtimers[i][0].cuda_event), ctypes.c_void_p(dtimers[i][1].cuda_event))
+        s = la.la_decode_step_decay(P(qs[i]), P(ks[i]), P(vs[i]), P(state), P(o), Bt, H, d, la.LA_BF16, P(decay), sh)
+        if s != 0:
+            raise RuntimeError(f"la_decode_step_decay failed: {la.STATUS.get(s, s)}")
+    torch.cuda.synchronize(dev)
+    if la.device_status() != 0:
+        raise RuntimeError("device status after decode with decay")
+    dkms = max_over_ranks(pg, statistics.mean(a.elapsed_time(b) for a, b in dtimers))
+    dgbs = (state_bytes + io_bytes) / (dkms / 1e3) / 1e9
     return {"workload": w.name, "steps": n_steps, "ms_per_step": ms, "kernel_ms": kms,
             "value": gbs, "unit": "GB/s", "hbm_frac": gbs / pk["hbm_gbs"],
             "tokens_per_s": Bt / (ms / 1e3),
+            "decay": {"kernel_ms": dkms, "value": dgbs, "unit": "GB/s", "hbm_frac": dgbs / pk["hbm_gbs"]},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": captured_traffic("decode_step_kernel"),
                          "algorithmic_bytes": state_bytes + io_bytes}}
+
+
+def run_decay(la, dev, stream, args, pk, pg, local, q, k, v, o, w):
+    """la_prefill_decay on the 32k workload's inputs with the decay recipe's per-head rates
+    (lambda_h = exp(-2^(-8 (h+1) / H))): the decay instance of the on-chip-state tensor-core
+    kernel. Same algorithmic bytes and counted FLOPs as the prefill without decay."""
+    import ctypes
+    T, H, d, B = w.total_tokens, w.heads, w.d, w.B
+    decay = wl.decay_rates(H, device=dev)
+    ws_bytes = la.la_prefill_decay_workspace_size(T, 1, H, d, B, la.LA_BF16)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    n = max(10, min(args.steps, 100))
+
+    def step(timer=None):
+        if timer is not None:
+            la.la_set_kernel_timer(ctypes.c_void_p(timer[0].cuda_event), ctypes.c_void_p(timer[1].cuda_event))
+        s = la.la_prefill_decay(P(q), P(k), P(v), P(o), None, 1, T, H, d, B, la.LA_BF16, None, P(decay), None,
+                                P(ws), ws_bytes, sh)
+        if s != 0:
+            raise RuntimeError(f"la_prefill_decay failed: {la.STATUS.get(s, s)}")
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    timers = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in timers:
+        a.record(); b.record()
+    torch.cuda.synchronize(dev)
+    barrier(pg, local)
+    launches0 = la.la_launch_count()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for i in range(n):
+        step(timers[i])
+    a1.record(stream)
+    launches = la.la_launch_count() - launches0
+    torch.cuda.synchronize(dev)
+    barrier(pg, local)
+    ms = max_over_ranks(pg, a0.elapsed_time(a1)) / n
+    kms = max_over_ranks(pg, statistics.mean(a.elapsed_time(b) for a, b in timers))
+    if la.device_status() != 0:
+        raise RuntimeError("device status after decay prefill")
+    del ws
+    alg_bytes = 8 * d * T * H
+    gbs = alg_bytes / (kms / 1e3) / 1e9
+    tflops = flops_per_token_head(B, d) * T * H / (ms / 1e3) / 1e12
+    return {"workload": f"bf16 prefill with per-head decay T={T} H={H} d={d} B={B}",
+            "rates": "lambda_h = exp(-2^(-8 (h+1) / H)), 0.40 .. 0.996",
+            "steps": n, "ms_per_step": ms, "kernel_ms": kms, "tokens_per_s": T / (ms / 1e3),
+            "tflops": tflops, "tc_peak_frac": tflops / pk["bf16_tflops"], "launches_per_step": launches / n,
+            "roofline": {"bound": "hbm", "kernel": "prefill_chain_kernel (decay instance)", "achieved": gbs,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                         "traffic": captured_traffic("prefill_chain_kernel_decay"),
+                         "algorithmic_bytes": alg_bytes}}
 
 
 # ---------------------------------------------------------------------------- reference arm
@@ -438,6 +519,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-decay", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

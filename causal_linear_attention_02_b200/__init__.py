@@ -26,9 +26,11 @@ __all__ = [
     "la_state_workspace_size", "la_state_from_prefill", "la_state_exclusive_prefix",
     "la_prefill_backward_workspace_size", "la_prefill_backward",
     "la_prefill_with_state_workspace_size", "la_prefill_with_state",
-    "la_decode_step", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
+    "la_decode_step", "la_prefill_decay_workspace_size", "la_prefill_decay", "la_state_decay_workspace_size",
+    "la_state_decay", "la_decode_step_decay", "la_feature_map", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
     "la_launch_count",
     "prefill", "prefill_with_state", "prefill_backward", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status",
+    "prefill_decay", "state_decay", "decode_step_decay", "feature_map",
     "uses_tensor_cores",
 ]
 
@@ -37,6 +39,7 @@ LA_FP32 = 1
 STATUS = {
     0: "LA_OK", 1: "LA_ERR_INVALID_ARGUMENT", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_MISALIGNED",
     4: "LA_ERR_WORKSPACE_TOO_SMALL", 5: "LA_ERR_CUDA", 6: "LA_ERR_TIMEOUT", 7: "LA_ERR_BAD_SEQLENS",
+    8: "LA_ERR_BAD_DECAY",
 }
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +94,18 @@ def load_library():
         lib.la_state_exclusive_prefix.restype = i32
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         lib.la_decode_step.restype = i32
+        lib.la_prefill_decay_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+        lib.la_prefill_decay_workspace_size.restype = sz
+        lib.la_prefill_decay.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        lib.la_prefill_decay.restype = i32
+        lib.la_state_decay_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+        lib.la_state_decay_workspace_size.restype = sz
+        lib.la_state_decay.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+        lib.la_state_decay.restype = i32
+        lib.la_decode_step_decay.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]
+        lib.la_decode_step_decay.restype = i32
+        lib.la_feature_map.argtypes = [vp, vp, i64, i32, ctypes.c_float, vp]
+        lib.la_feature_map.restype = i32
         lib.la_get_device_status.argtypes = [vp]
         lib.la_get_device_status.restype = i32
         lib.la_status_string.argtypes = [i32]
@@ -169,6 +184,34 @@ def la_state_exclusive_prefix(gathered, world, rank, n, d, init, out, stream) ->
 
 def la_decode_step(q, k, v, state, o, batch, heads, d, dtype, stream) -> int:
     return int(load_library().la_decode_step(q, k, v, state, o, batch, heads, d, dtype, stream))
+
+
+def la_prefill_decay_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) -> int:
+    return int(load_library().la_prefill_decay_workspace_size(total_tokens, num_seqs, heads, d, B, dtype))
+
+
+def la_prefill_decay(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state, decay,
+                     state_out, workspace, workspace_bytes, stream) -> int:
+    return int(load_library().la_prefill_decay(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype,
+                                               init_state, decay, state_out, workspace, workspace_bytes, stream))
+
+
+def la_state_decay_workspace_size(total_tokens, num_seqs, heads, d, dtype) -> int:
+    return int(load_library().la_state_decay_workspace_size(total_tokens, num_seqs, heads, d, dtype))
+
+
+def la_state_decay(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype, init_state, decay, state_out,
+                   workspace, workspace_bytes, stream) -> int:
+    return int(load_library().la_state_decay(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype, init_state,
+                                             decay, state_out, workspace, workspace_bytes, stream))
+
+
+def la_decode_step_decay(q, k, v, state, o, batch, heads, d, dtype, decay, stream) -> int:
+    return int(load_library().la_decode_step_decay(q, k, v, state, o, batch, heads, d, dtype, decay, stream))
+
+
+def la_feature_map(x, y, n, dtype, alpha, stream) -> int:
+    return int(load_library().la_feature_map(x, y, n, dtype, alpha, stream))
 
 
 def la_get_device_status(stream) -> int:
@@ -404,6 +447,113 @@ def decode_step(q, k, v, state, out=None, stream=None):
     status = la_decode_step(_p(q), _p(k), _p(v), _p(state), _p(out), batch, H, d, code,
                             _stream_handle(stream, q.device))
     _raise(status, "la_decode_step")
+    return out
+
+
+def _decay_rates(decay, H, device):
+    _need(decay, "decay", device)
+    if decay.dtype != torch.float32 or tuple(decay.shape) != (H,):
+        raise LightningError("decay must be fp32 [H]", 1)
+
+
+def prefill_decay(q, k, v, decay, cu_seqlens=None, B: int = 256, init_state=None, return_state=False, out=None,
+                  state_out=None, workspace=None, stream=None):
+    """O (and optionally the final states) of causal linear attention with a per-head decay rate on the state,
+    S_t = decay[h] S_{t-1} + k_t^T v_t, o_t = q_t S_t (see la_prefill_decay)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise LightningError("q, k, v must share one [T, H, d] shape and dtype", 1)
+    T, H, d = q.shape
+    _decay_rates(decay, H, q.device)
+    nseq = 1
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", q.device)
+        if cu_seqlens.dtype != torch.int32:
+            raise LightningError("cu_seqlens must be int32", 1)
+        nseq = cu_seqlens.numel() - 1
+    if init_state is not None:
+        _need(init_state, "init_state", q.device)
+        if init_state.dtype != torch.float32 or tuple(init_state.shape) != (nseq, H, d, d):
+            raise LightningError("init_state must be fp32 [num_seqs, H, d, d]", 1)
+    code = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.device)
+    if return_state and state_out is None:
+        state_out = torch.empty((nseq, H, d, d), dtype=torch.float32, device=q.device)
+    if state_out is not None:
+        _need(state_out, "state_out", q.device)
+    ws_bytes = la_prefill_decay_workspace_size(T, nseq, H, d, B, code)
+    if ws_bytes == 0:
+        raise LightningError(f"unsupported prefill shape T={T} H={H} d={d} B={B}", 2)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    status = la_prefill_decay(_p(q), _p(k), _p(v), _p(out), _p(cu_seqlens), nseq, T, H, d, B, code, _p(init_state),
+                              _p(decay), _p(state_out), _p(workspace), workspace.numel() * workspace.element_size(),
+                              _stream_handle(stream, q.device))
+    _raise(status, "la_prefill_decay")
+    return (out, state_out) if (return_state or state_out is not None) else out
+
+
+def state_decay(k, v, decay, cu_seqlens=None, init_state=None, out=None, workspace=None, stream=None):
+    """fp32 [num_seqs, H, d, d] final states with decay (see la_state_decay)."""
+    _need(k, "k"); _need(v, "v", k.device)
+    if k.dim() != 3 or v.shape != k.shape or v.dtype != k.dtype:
+        raise LightningError("k, v must share one [T, H, d] shape and dtype", 1)
+    T, H, d = k.shape
+    _decay_rates(decay, H, k.device)
+    nseq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", k.device)
+    if out is None:
+        out = torch.empty((nseq, H, d, d), dtype=torch.float32, device=k.device)
+    _need(out, "out", k.device)
+    if init_state is not None:
+        _need(init_state, "init_state", k.device)
+    code = _dtype_code(k.dtype)
+    ws_bytes = la_state_decay_workspace_size(T, nseq, H, d, code)
+    if ws_bytes == 0:
+        raise LightningError(f"unsupported state shape T={T} H={H} d={d}", 2)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device)
+    status = la_state_decay(_p(k), _p(v), _p(cu_seqlens), nseq, T, H, d, code, _p(init_state), _p(decay), _p(out),
+                            _p(workspace), workspace.numel() * workspace.element_size(),
+                            _stream_handle(stream, k.device))
+    _raise(status, "la_state_decay")
+    return out
+
+
+def decode_step_decay(q, k, v, state, decay, out=None, stream=None):
+    """One step S <- decay[h] S + k^T v, o = q S on [batch, H, d] inputs; state updated in place."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("state", state)):
+        _need(t, n, q.device)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise LightningError("q, k, v must share one [batch, H, d] shape", 1)
+    batch, H, d = q.shape
+    _decay_rates(decay, H, q.device)
+    if state.dtype != torch.float32 or tuple(state.shape) != (batch, H, d, d):
+        raise LightningError("state must be fp32 [batch, H, d, d]", 1)
+    code = _dtype_code(q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    status = la_decode_step_decay(_p(q), _p(k), _p(v), _p(state), _p(out), batch, H, d, code, _p(decay),
+                                  _stream_handle(stream, q.device))
+    _raise(status, "la_decode_step_decay")
+    return out
+
+
+def feature_map(x, alpha: float = 0.3, out=None, stream=None):
+    """phi(x) = ELU(x) + alpha x elementwise (see la_feature_map); out may be x for in place."""
+    _need(x, "x")
+    code = _dtype_code(x.dtype)
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", x.device)
+    if out.dtype != x.dtype or out.numel() != x.numel():
+        raise LightningError("out must match x in dtype and size", 1)
+    status = la_feature_map(_p(x), _p(out), x.numel(), code, float(alpha), _stream_handle(stream, x.device))
+    _raise(status, "la_feature_map")
     return out
 
 

@@ -59,6 +59,7 @@
 #include "common.cuh"
 #include "sm100.cuh"
 #include "pipe.cuh"
+#include "decay.cuh"
 
 namespace la {
 namespace chain {
@@ -79,7 +80,7 @@ constexpr int KC = 128;                    // keys per chunk
 #define LA_CHAIN_NV 2
 #endif
 constexpr int NQ = LA_CHAIN_NQ;            // Q sub-unit stages
-constexpr int NK = LA_CHAIN_NK;            // K chunk stages
+constexpr int NK_MAX = LA_CHAIN_NK > 2 ? LA_CHAIN_NK : 2;   // K chunk stages, either instance
 constexpr int NV = LA_CHAIN_NV;            // V chunk stages
 constexpr int NS = 2;                      // score buffers in TMEM
 constexpr int NTHREADS = 640;
@@ -91,13 +92,22 @@ constexpr uint32_t K_BYTES = 2 * KH_BYTES;       // 32 KB
 constexpr uint32_t V_BYTES = KC * DV * 2;        // 16 KB
 constexpr uint32_t SB_BYTES = D * DV * 2;        // 16 KB: bf16 KV_b, 128 rows x 64 columns
 
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + NQ * Q_BYTES;
-constexpr uint32_t OFF_V = OFF_K + NK * K_BYTES;
-constexpr uint32_t OFF_SB = OFF_V + NV * V_BYTES;
-constexpr uint32_t OFF_BAR = OFF_SB + SB_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;   // + barriers + 1 KB alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+// Shared-memory layout. The decay instance (a rate per head on the state) also
+// keeps a ring of decay-weighted V chunks, the B operand of its state MMAs, and
+// gives up one K stage for it.
+template <bool kDecay>
+struct Smem {
+    static constexpr int NK = kDecay ? 2 : LA_CHAIN_NK;    // K chunk stages
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_K = OFF_Q + NQ * Q_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + NK * K_BYTES;
+    static constexpr uint32_t OFF_VW = OFF_V + NV * V_BYTES;               // weighted V (decay only)
+    static constexpr uint32_t OFF_SB = OFF_VW + (kDecay ? NV * V_BYTES : 0);
+    static constexpr uint32_t OFF_BAR = OFF_SB + SB_BYTES;
+    static constexpr uint32_t BYTES = OFF_BAR + 512 + 1024;   // + barriers + 1 KB alignment slack
+    static_assert(BYTES <= 232448, "shared memory per CTA");
+    static_assert(NK <= NK_MAX, "barrier arrays");
+};
 
 // TMEM columns (512 x 32-bit, 128 lanes): three O slots, the state, NS score buffers.
 constexpr uint32_t TM_O = 0, TM_KV = 192, TM_S = 256, TM_COLS = 512;
@@ -110,8 +120,11 @@ constexpr uint32_t IDESC_C = idesc_bf16(UM, DV, false, true);    // Q (K-major) 
 
 struct Bars {
     uint64_t q_full[NQ], q_empty[NQ];
-    uint64_t k_full[NK], k_empty[NK];     // k_empty: two arrivals, the chunk's scores and its state MMA
-    uint64_t v_full[NV], v_empty[NV];     // v_empty: two arrivals, the chunk's PVs and its state MMA
+    uint64_t k_full[NK_MAX], k_empty[NK_MAX]; // k_empty: two arrivals, the chunk's scores and its state MMA
+    uint64_t v_full[NV], v_empty[NV];     // v_empty: two arrivals, the chunk's PVs and its state MMA (decay
+                                          // instance: the weighting warp, which reads it for the state MMA)
+    uint64_t vw_full[NV], vw_empty[NV];   // decay instance: weighted V chunk written / read by its state MMA
+    uint64_t c_full[3], c_scaled[3];      // decay instance: inter-block MMA done / its rows scaled, per O slot
     uint64_t s_full[NS], p_full[NS], s_free[NS];
     uint64_t o_full[3], o_empty[3];
     uint64_t kv_ready;        // issuer -> state group: KV accumulator holds the next block's prefix
@@ -132,6 +145,7 @@ struct Params {
     float* state_out;         // [nseq][H][D][D] final states (the state-output instance only)
     const __nv_bfloat16* k;   // K and V, [T][H][D]: the few tokens of a ragged last chunk past its
     const __nv_bfloat16* v;   // last full 16-key MMA step (state-output instance only)
+    const float* decay;       // [H] decay rates (the decay instance only)
     int H, B, log2B, nseq;
     uint64_t wait_ns;
     long long suppress_item;  // test hook: this work item never hands over its second block's prefix (-1: none)
@@ -294,10 +308,27 @@ struct Cursor {
 // p.state_out (the last block runs its state MMAs too; the copy-out group reads
 // the accumulator after them). A separate instance, so the plain prefill's code
 // is unchanged.
-template <bool kStateOut>
+//
+// kDecay: a decay rate lambda_h in [0, 1] per head on the state (decay.cuh):
+// S_t = lambda S_{t-1} + k_t^T v_t. For a block of n rows, row r (in the block)
+// and key c (in the block):
+//   P[r][c]   = lambda^(r-c) S[r][c]                 (P groups, c <= r)
+//   O_r      += lambda^(r+1) q_r bf16(KV_b)          (copy-out group scales the
+//               rows of the inter-block accumulator in TMEM before the first PV)
+//   KV_{b+1}  = lambda^n KV_b + sum_c K_c^T (lambda^(n-1-c) v_c)
+//               (copy-out group rescales the accumulator when it reads KV_b;
+//               warp 2 writes the weighted V chunk, the state MMA's B operand)
+// The weighted V is rounded to bf16 once, so the state's increments carry one
+// extra bf16 rounding (relative 2^-9 per term). Rates are checked before the
+// launch (a bad rate leaves the launch with no work).
+template <bool kStateOut, bool kDecay>
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
+    using SM = Smem<kDecay>;
+    constexpr int NK = SM::NK;
+    constexpr uint32_t OFF_Q = SM::OFF_Q, OFF_K = SM::OFF_K, OFF_V = SM::OFF_V, OFF_SB = SM::OFF_SB,
+                       OFF_BAR = SM::OFF_BAR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BAR);
@@ -320,6 +351,10 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars->sb_empty, 1);
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->drain_b, 1);
+        if constexpr (kDecay) {
+            for (int i = 0; i < NV; ++i) { mbar_init(&bars->vw_full[i], 32); mbar_init(&bars->vw_empty[i], 1); }
+            for (int i = 0; i < 3; ++i) { mbar_init(&bars->c_full[i], 1); mbar_init(&bars->c_scaled[i], 128); }
+        }
         bars->abort_flag = 0;
         fence_mbar_init();
     }
@@ -424,6 +459,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const uint64_t dkt = sdesc_sw128(smem_u32(smem + OFF_K), KH_BYTES, 1024);      // MN-major (state)
         const uint64_t dv = sdesc_sw128(smem_u32(smem + OFF_V), V_BYTES, 1024);
         const uint64_t dsb = sdesc_sw128(smem_u32(smem + OFF_SB), SB_BYTES, 1024);
+        const uint64_t dvs = kDecay ? sdesc_sw128(smem_u32(smem + SM::OFF_VW), V_BYTES, 1024) : dv;   // state MMA's V
         if (warp == 1 && lane == 0) {
             // ============================================================ issuer A: scores, state MMAs
             // Event loop over two cursors; every step is taken only when its inputs are
@@ -467,7 +503,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         dc.next_item(p);
                     } else {
                         const uint32_t kc = dc.kc0 + dc.j;
-                        bool ready = mbar_test_wait(&bars->v_full[kc % NV], (kc / NV) & 1);
+                        bool ready = mbar_test_wait(kDecay ? &bars->vw_full[kc % NV] : &bars->v_full[kc % NV],
+                                                    (kc / NV) & 1);
                         if (ready && dc.add_state && dc.j == 0 && kvr_blk != dc.n) {
                             if (mbar_test_wait(&bars->kv_read[dc.n & 3], (dc.n >> 2) & 1)) kvr_blk = dc.n;
                             else ready = false;
@@ -475,7 +512,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         if (ready) {
                             if (dc.add_state || kStateOut) {
                                 tc_fence_after();
-                                const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4), b = dv + (((kc % NV) * V_BYTES) >> 4);
+                                const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4), b = dvs + (((kc % NV) * V_BYTES) >> 4);
                                 // a ragged last chunk: its full 16-key steps only (the copy-out
                                 // group adds the rest); the rows past the sequence end belong to
                                 // the next sequence
@@ -491,7 +528,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                                 }
                             }
                             tc_commit(&bars->k_empty[kc % NK]);          // the state MMA's shares
-                            tc_commit(&bars->v_empty[kc % NV]);
+                            tc_commit(kDecay ? &bars->vw_empty[kc % NV] : &bars->v_empty[kc % NV]);
                             dc.next_item(p);
                             prog = true;
                         }
@@ -536,6 +573,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (c.r == c.Rb - 1) tc_commit(&bars->sb_empty);
                     tc_commit(&bars->q_empty[qc % NQ]);                  // the inter-block MMA's share
                     LA_CTRACE(c.n, c.r == 0 ? TR_C0 : TR_CL);
+                    if constexpr (kDecay) {
+                        // lambda^(r+1) on its rows before the PVs add onto it
+                        tc_commit(&bars->c_full[slot]);
+                        if (!wait_bar(&bars->c_scaled[slot], c.ouse(c.r) & 1, ab)) { ok = false; break; }
+                    }
                 }
                 // O_r += P V_j; P of keys 0-63 in columns 0-31, of keys 64-127 in 64-95
                 if (!wait_bar(&bars->p_full[sbuf], (c.i / NS) & 1, ab)) { ok = false; break; }
@@ -557,6 +599,53 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&bars->drain_b, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
         }
+    } else if (warp == 2) {
+        if constexpr (kDecay) {
+            // ============================================================ weighted V (decay instance)
+            // Every V chunk in ring order: the copy lambda^(rows-1-c) v_c (c the key in the block,
+            // zero past the block's end) that the state MMA reads, then the chunk's second V
+            // release, which in this instance is this warp's (the state MMA reads the copy).
+            // A chunk whose state MMA does not run passes through the ring unwritten. A line of
+            // the swizzled chunk is one key's 64 columns, so lines are scaled whole; the 32
+            // lanes take 512 contiguous bytes (4 lines) per step.
+            bool ok = true;
+            Cursor c;
+            c.init(p);
+            while (ok && c.valid) {
+                const float l2 = log2f(__ldg(p.decay + c.h));
+                for (int j = 0; j < c.Rb; ++j) {
+                    const uint32_t kc = c.kc0 + j, st = kc % NV;
+                    if (!warp_all(wait_bar(&bars->v_full[st], (kc / NV) & 1, ab)) ||
+                        !warp_all(wait_bar(&bars->vw_empty[st], ((kc / NV) & 1) ^ 1, ab))) {
+                        ok = false;
+                        break;
+                    }
+                    if (c.add_state || kStateOut) {
+                        const uint8_t* src = smem + OFF_V + st * V_BYTES;
+                        uint8_t* dst = smem + SM::OFF_VW + st * V_BYTES;
+#pragma unroll 4
+                        for (int it = 0; it < KC / 4; ++it) {
+                            const int line = 4 * it + (lane >> 3);                 // key KC*j + line
+                            const int t = KC * j + line;
+                            const float w = t < c.rows ? decay_pow(l2, c.rows - 1 - t) : 0.f;
+                            const uint32_t off = line * 128 + (lane & 7) * 16;
+                            uint4 u = *reinterpret_cast<const uint4*>(src + off);
+                            uint32_t* e = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+                            for (int x = 0; x < 4; ++x)
+                                e[x] = pack_bf16x2(__uint_as_float(e[x] << 16) * w,
+                                                   __uint_as_float(e[x] & 0xffff0000u) * w);
+                            *reinterpret_cast<uint4*>(dst + off) = u;
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    mbar_arrive(&bars->vw_full[st]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->v_empty[st]);      // done reading the V chunk
+                }
+                c.next_block(p);
+            }
+        }
     } else if (warp >= 4 && warp < 12) {
         // ================================================================ scores -> P
         const int hk = warp >= 8 ? 1 : 0;                // keys 0-63 or 64-127 of the chunk
@@ -573,16 +662,36 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint32_t ts = tmem + lane_base + TM_S + sbuf * KC + 64 * hk;
             const int lim = UM * (c.r - c.j) + m - 64 * hk;    // key column kept when col <= lim
             uint32_t pk[32];
+            float lam = 1.f, l2 = 0.f;
+            if constexpr (kDecay) {
+                lam = __ldg(p.decay + c.h);
+                l2 = log2f(lam);
+            }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t a[32];
                 tmem_ld_x32(ts + 32 * hh, a);
                 tmem_wait_ld();
+                if constexpr (kDecay) {
+                    // lambda^(lim - col) for col <= lim (lim - col = row - key in the block), from the
+                    // highest column of this half down: one power, then a product per kept column
+                    float f = decay_pow(l2, max(lim - (32 * hh + 31), 0));
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int c0 = 32 * hh + 2 * q;
-                    pk[16 * hh + q] = pack_bf16x2(c0 <= lim ? __uint_as_float(a[2 * q]) : 0.f,
-                                                  c0 + 1 <= lim ? __uint_as_float(a[2 * q + 1]) : 0.f);
+                    for (int q = 15; q >= 0; --q) {
+                        const int c1 = 32 * hh + 2 * q + 1, c0 = c1 - 1;
+                        const float x1 = c1 <= lim ? __uint_as_float(a[2 * q + 1]) * f : 0.f;
+                        f = c1 <= lim ? f * lam : f;
+                        const float x0 = c0 <= lim ? __uint_as_float(a[2 * q]) * f : 0.f;
+                        f = c0 <= lim ? f * lam : f;
+                        pk[16 * hh + q] = pack_bf16x2(x0, x1);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int c0 = 32 * hh + 2 * q;
+                        pk[16 * hh + q] = pack_bf16x2(c0 <= lim ? __uint_as_float(a[2 * q]) : 0.f,
+                                                      c0 + 1 <= lim ? __uint_as_float(a[2 * q + 1]) : 0.f);
+                    }
                 }
             }
             tmem_st_x32(ts, pk);             // P of these 64 keys over the first 32 of their columns
@@ -607,6 +716,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         while (ok && c.valid) {
             // KV_b -> bf16 operand of the inter-block product (row m, 64 columns)
             uint32_t pk[32];
+            float l2 = 0.f, wn = 1.f;                   // decay: log2 of the rate, lambda^rows
+            if constexpr (kDecay) {
+                l2 = log2f(__ldg(p.decay + c.h));
+                wn = decay_pow(l2, c.rows);
+            }
             if (c.b > 0) {
                 if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
                 ++kvc;
@@ -617,13 +731,28 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     uint32_t a[32];
                     tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
                     tmem_wait_ld();
-                    if (hh == 1) {
-                        tc_fence_before();
-                        mbar_arrive(&bars->kv_read[c.n & 3]);    // the accumulator may take this block's keys
-                    }
+                    if constexpr (kDecay) {
+                        // the accumulator carries lambda^rows KV_b into this block's keys
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                        for (int q = 0; q < 16; ++q)
+                            pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__uint_as_float(a[q]) * wn);
+                        tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                        if (hh == 1) {
+                            tmem_wait_st();
+                            tc_fence_before();
+                            mbar_arrive(&bars->kv_read[c.n & 3]);
+                        }
+                    } else {
+                        if (hh == 1) {
+                            tc_fence_before();
+                            mbar_arrive(&bars->kv_read[c.n & 3]);    // the accumulator may take this block's keys
+                        }
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                    }
                 }
             } else {
                 // A work item's first block: KV_0 = S0 (zero without a carried-in state).
@@ -642,10 +771,19 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                             a[4 * q + 2] = __float_as_uint(v.z);
                             a[4 * q + 3] = __float_as_uint(v.w);
                         }
-                        tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                        if constexpr (kDecay) {   // seeded as lambda^rows S0
 #pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                            for (int q = 0; q < 16; ++q)
+                                pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__uint_as_float(a[q]) * wn);
+                            tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                        } else {
+                            tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+#pragma unroll
+                            for (int q = 0; q < 16; ++q)
+                                pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                        }
                     }
                     tmem_wait_st();
                 } else {
@@ -663,6 +801,28 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             fence_proxy_async_smem();
             if (!(c.w == p.suppress_item && c.b == 1)) mbar_arrive(&bars->sb_full);
             if (wt == 0) LA_CTRACE(c.n, TR_SB);
+            if constexpr (kDecay) {
+                // lambda^(r+1) on row r of each sub-unit's inter-block accumulator (r in the block)
+                for (int r = 0; r < c.Rb; ++r) {
+                    const uint32_t slot = c.oslot(r);
+                    if (!warp_all(wait_bar(&bars->c_full[slot], c.ouse(r) & 1, ab))) { ok = false; break; }
+                    tc_fence_after();
+                    const float wr = decay_pow(l2, UM * r + m + 1);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t a[32];
+                        tmem_ld_x32(tmem + lane_base + TM_O + slot * 64 + 32 * hh, a);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__uint_as_float(a[q]) * wr);
+                        tmem_st_x32(tmem + lane_base + TM_O + slot * 64 + 32 * hh, a);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&bars->c_scaled[slot]);
+                }
+                if (!ok) break;
+            }
             if (kStateOut && !c.add_state) {
                 // the work item's last block: its state MMAs complete the final state
                 if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
@@ -681,7 +841,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
                 // the tokens past the last full 16-key step, on CUDA cores
                 for (int t = c.tok0 + (c.rows & ~15); t < c.tok0 + c.rows; ++t) {
-                    const float ki = __bfloat162float(p.k[((int64_t)t * p.H + c.h) * D + m]);
+                    float ki = __bfloat162float(p.k[((int64_t)t * p.H + c.h) * D + m]);
+                    if constexpr (kDecay) ki *= decay_pow(l2, c.tok0 + c.rows - 1 - t);
                     const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + c.h) * D + DV * c.half);
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {

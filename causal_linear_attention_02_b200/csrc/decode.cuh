@@ -8,9 +8,13 @@
 // re-read. One CTA per (sequence, head): a warp covers whole rows with 16-byte
 // coalesced streaming loads/stores; the partial outputs of the row groups are
 // reduced through shared memory.
+//
+// The kDecay instance takes a per-head decay rate (decay.cuh):
+// S <- lambda_h S + k^T v, o = lambda_h (q S_old) + (q . k) v.
 #pragma once
 
 #include "common.cuh"
+#include "decay.cuh"
 
 namespace la {
 
@@ -23,10 +27,10 @@ __host__ __device__ constexpr int decode_row_groups(int D) {
     return best;
 }
 
-template <typename Tin, int D>
+template <typename Tin, int D, bool kDecay = false>
 __global__ void __launch_bounds__((D / 4) * decode_row_groups(D))
 decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
-                   float* __restrict__ state, Tin* __restrict__ o) {
+                   float* __restrict__ state, Tin* __restrict__ o, const float* decay, int H) {
     constexpr int CG = D / 4;                 // float4 column groups per row
     constexpr int RG = decode_row_groups(D);  // row groups (threads sharing a column group)
     constexpr int NT = CG * RG;
@@ -36,6 +40,14 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const T
     __shared__ float4 red[RG][CG];
     const int64_t p = blockIdx.x;             // (sequence, head) pair
     const int tid = threadIdx.x;
+    float lam = 1.f;
+    if constexpr (kDecay) {
+        lam = decay[p % H];
+        if (!(lam >= 0.f && lam <= 1.f)) {
+            if (tid == 0) record_status(LA_ERR_BAD_DECAY);
+            return;
+        }
+    }
     if (tid < D) {
         qs[tid] = io<Tin>::ld(q + p * D + tid);
         ks[tid] = io<Tin>::ld(k + p * D + tid);
@@ -56,8 +68,13 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const T
         float4 s = rows[a];
         acc.x = fmaf(qi, s.x, acc.x); acc.y = fmaf(qi, s.y, acc.y);
         acc.z = fmaf(qi, s.z, acc.z); acc.w = fmaf(qi, s.w, acc.w);
-        s.x = fmaf(ki, vv.x, s.x); s.y = fmaf(ki, vv.y, s.y);
-        s.z = fmaf(ki, vv.z, s.z); s.w = fmaf(ki, vv.w, s.w);
+        if constexpr (kDecay) {
+            s.x = fmaf(ki, vv.x, lam * s.x); s.y = fmaf(ki, vv.y, lam * s.y);
+            s.z = fmaf(ki, vv.z, lam * s.z); s.w = fmaf(ki, vv.w, lam * s.w);
+        } else {
+            s.x = fmaf(ki, vv.x, s.x); s.y = fmaf(ki, vv.y, s.y);
+            s.z = fmaf(ki, vv.z, s.z); s.w = fmaf(ki, vv.w, s.w);
+        }
         __stcs(S + (int64_t)i * CG + cg, s);
     }
     red[rg][cg] = acc;
@@ -72,6 +89,7 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const T
             const float4 x = red[r][c];
             sum += lane4 == 0 ? x.x : lane4 == 1 ? x.y : lane4 == 2 ? x.z : x.w;
         }
+        if constexpr (kDecay) sum *= lam;
         io<Tin>::st(o + p * D + tid, fmaf(qk, vs[tid], sum));
     }
 }

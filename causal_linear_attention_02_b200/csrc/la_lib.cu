@@ -21,6 +21,7 @@
 #include "state.cuh"
 #include "lasp.cuh"
 #include "backward.cuh"
+#include "decay.cuh"
 
 namespace {
 
@@ -107,6 +108,21 @@ Layout prefill_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt) {
     return L;
 }
 
+// The CUDA-core three-kernel prefill (block states, scan, prefill) whatever the
+// dtype and shape: it also carries the decay variant.
+Layout simt_layout(int64_t T, int nseq, int H, int d, int B) {
+    Layout L;
+    size_t off = layout_head(L, T, nseq, B);
+    const size_t dd = (size_t)d * d;
+    L.off_U = off;      off = align_up(off + 4 * dd * (size_t)H * (size_t)L.max_blocks, 256);
+    L.off_prefix = off; off = align_up(off + 4 * dd * (size_t)H * (size_t)L.max_blocks, 256);
+    L.total = off;
+    return L;
+}
+
+// Block states of kStateBlock tokens and their scan (the CUDA-core state pass).
+Layout simt_state_layout(int64_t T, int nseq, int H, int d);
+
 Layout state_layout(int64_t T, int nseq, int H, int d, la_dtype dt) {
     Layout L;
     if (dt == LA_BF16 && d == 128) {
@@ -117,6 +133,11 @@ Layout state_layout(int64_t T, int nseq, int H, int d, la_dtype dt) {
         L.total = off;
         return L;
     }
+    return simt_state_layout(T, nseq, H, d);
+}
+
+Layout simt_state_layout(int64_t T, int nseq, int H, int d) {
+    Layout L;
     size_t off = layout_head(L, T, nseq, kStateBlock);
     L.off_U = off; off = align_up(off + 4 * (size_t)d * d * (size_t)H * (size_t)L.max_blocks, 256);
     L.total = off;
@@ -206,30 +227,31 @@ la_status launch_block_table(const int32_t* cu, int nseq, int64_t T, int B, int 
     return cuda_check();
 }
 
-template <typename Tin, int D>
+template <typename Tin, int D, bool kDecay>
 la_status prefill_simt_main(const void* q, const void* k, const void* v, void* o, int H, int B,
-                            const Layout& L, uint8_t* ws, cudaStream_t st) {
+                            const Layout& L, uint8_t* ws, const float* decay, cudaStream_t st) {
     const Control* ctrl = reinterpret_cast<const Control*>(ws);
     const BlockEntry* table = reinterpret_cast<const BlockEntry*>(ws + L.off_table);
     const float* prefix = reinterpret_cast<const float*>(ws + L.off_prefix);
     constexpr size_t smem = la::simt::prefill_simt_smem<D>();
-    if (cudaFuncSetAttribute(la::simt::prefill_simt<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(la::simt::prefill_simt<Tin, D, kDecay>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return LA_ERR_CUDA;
     const int64_t grid = L.max_blocks * H * (B / 64);
-    la::simt::prefill_simt<Tin, D><<<(unsigned)grid, la::simt::THREADS, smem, st>>>(
-        (const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, prefix, table, ctrl, H, B);
+    la::simt::prefill_simt<Tin, D, kDecay><<<(unsigned)grid, la::simt::THREADS, smem, st>>>(
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, prefix, table, ctrl, H, B, decay);
     note_launch();
     return cuda_check();
 }
 
-template <typename Tin, int D>
-la_status state_simt_launch(const void* k, const void* v, int H, const Layout& L, uint8_t* ws, cudaStream_t st) {
+template <typename Tin, int D, bool kDecay>
+la_status state_simt_launch(const void* k, const void* v, int H, const Layout& L, uint8_t* ws, const float* decay,
+                            cudaStream_t st) {
     const Control* ctrl = reinterpret_cast<const Control*>(ws);
     const BlockEntry* table = reinterpret_cast<const BlockEntry*>(ws + L.off_table);
     float* U = reinterpret_cast<float*>(ws + L.off_U);
-    la::simt::block_state_simt<Tin, D><<<(unsigned)(L.max_blocks * H), la::simt::THREADS, 0, st>>>(
-        (const Tin*)k, (const Tin*)v, table, ctrl, H, U);
+    la::simt::block_state_simt<Tin, D, kDecay><<<(unsigned)(L.max_blocks * H), la::simt::THREADS, 0, st>>>(
+        (const Tin*)k, (const Tin*)v, table, ctrl, H, U, decay);
     note_launch();
     return cuda_check();
 }
@@ -247,45 +269,59 @@ la_status state_simt_launch(const void* k, const void* v, int H, const Layout& L
         default: return LA_ERR_UNSUPPORTED;                \
     }
 
+// The instances with a decay rate per head (decay.cuh) are chosen by decay != nullptr.
 template <int D>
 la_status simt_states(la_dtype dt, const void* k, const void* v, int H, const Layout& L, uint8_t* ws,
-                      cudaStream_t st) {
-    return dt == LA_BF16 ? state_simt_launch<__nv_bfloat16, D>(k, v, H, L, ws, st)
-                         : state_simt_launch<float, D>(k, v, H, L, ws, st);
+                      const float* decay, cudaStream_t st) {
+    if (decay)
+        return dt == LA_BF16 ? state_simt_launch<__nv_bfloat16, D, true>(k, v, H, L, ws, decay, st)
+                             : state_simt_launch<float, D, true>(k, v, H, L, ws, decay, st);
+    return dt == LA_BF16 ? state_simt_launch<__nv_bfloat16, D, false>(k, v, H, L, ws, nullptr, st)
+                         : state_simt_launch<float, D, false>(k, v, H, L, ws, nullptr, st);
 }
 
 template <int D>
 la_status simt_prefill(la_dtype dt, const void* q, const void* k, const void* v, void* o, int H, int B,
-                       const Layout& L, uint8_t* ws, cudaStream_t st) {
-    return dt == LA_BF16 ? prefill_simt_main<__nv_bfloat16, D>(q, k, v, o, H, B, L, ws, st)
-                         : prefill_simt_main<float, D>(q, k, v, o, H, B, L, ws, st);
+                       const Layout& L, uint8_t* ws, const float* decay, cudaStream_t st) {
+    if (decay)
+        return dt == LA_BF16 ? prefill_simt_main<__nv_bfloat16, D, true>(q, k, v, o, H, B, L, ws, decay, st)
+                             : prefill_simt_main<float, D, true>(q, k, v, o, H, B, L, ws, decay, st);
+    return dt == LA_BF16 ? prefill_simt_main<__nv_bfloat16, D, false>(q, k, v, o, H, B, L, ws, nullptr, st)
+                         : prefill_simt_main<float, D, false>(q, k, v, o, H, B, L, ws, nullptr, st);
+}
+
+template <typename Tin, int D, bool kDecay>
+void decode_instance(const void* q, const void* k, const void* v, float* state, void* o, int64_t pairs,
+                     const float* decay, int H, cudaStream_t st) {
+    constexpr int nt = (D / 4) * la::decode_row_groups(D);
+    la::decode_step_kernel<Tin, D, kDecay><<<(unsigned)pairs, nt, 0, st>>>(
+        (const Tin*)q, (const Tin*)k, (const Tin*)v, state, (Tin*)o, decay, H);
 }
 
 template <int D>
 la_status decode_launch(la_dtype dt, const void* q, const void* k, const void* v, float* state, void* o,
-                        int64_t pairs, cudaStream_t st) {
-    constexpr int nt = (D / 4) * la::decode_row_groups(D);
+                        int64_t pairs, const float* decay, int H, cudaStream_t st) {
     if (dt == LA_BF16)
-        la::decode_step_kernel<__nv_bfloat16, D><<<(unsigned)pairs, nt, 0, st>>>(
-            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, state, (__nv_bfloat16*)o);
+        decay ? decode_instance<__nv_bfloat16, D, true>(q, k, v, state, o, pairs, decay, H, st)
+              : decode_instance<__nv_bfloat16, D, false>(q, k, v, state, o, pairs, nullptr, H, st);
     else
-        la::decode_step_kernel<float, D><<<(unsigned)pairs, nt, 0, st>>>(
-            (const float*)q, (const float*)k, (const float*)v, state, (float*)o);
+        decay ? decode_instance<float, D, true>(q, k, v, state, o, pairs, decay, H, st)
+              : decode_instance<float, D, false>(q, k, v, state, o, pairs, nullptr, H, st);
     note_launch();
     return cuda_check();
 }
 
 la_status simt_states_d(int d, la_dtype dt, const void* k, const void* v, int H, const Layout& L, uint8_t* ws,
-                        cudaStream_t st) {
-    LA_DISPATCH_D(d, simt_states, dt, k, v, H, L, ws, st);
+                        const float* decay, cudaStream_t st) {
+    LA_DISPATCH_D(d, simt_states, dt, k, v, H, L, ws, decay, st);
 }
 la_status simt_prefill_d(int d, la_dtype dt, const void* q, const void* k, const void* v, void* o, int H, int B,
-                         const Layout& L, uint8_t* ws, cudaStream_t st) {
-    LA_DISPATCH_D(d, simt_prefill, dt, q, k, v, o, H, B, L, ws, st);
+                         const Layout& L, uint8_t* ws, const float* decay, cudaStream_t st) {
+    LA_DISPATCH_D(d, simt_prefill, dt, q, k, v, o, H, B, L, ws, decay, st);
 }
 la_status decode_d(int d, la_dtype dt, const void* q, const void* k, const void* v, float* state, void* o,
-                   int64_t pairs, cudaStream_t st) {
-    LA_DISPATCH_D(d, decode_launch, dt, q, k, v, state, o, pairs, st);
+                   int64_t pairs, const float* decay, int H, cudaStream_t st) {
+    LA_DISPATCH_D(d, decode_launch, dt, q, k, v, state, o, pairs, decay, H, st);
 }
 
 // Common argument checks of the token-major entry points.
@@ -301,9 +337,16 @@ la_status check_tokens(int64_t T, int nseq, int H, int d, la_dtype dt, const int
 
 // The on-chip-state prefill (bf16, d = 128): sequence table, then the kernel;
 // with state_out, the instance that also writes the final states.
+// Rates of the decay variant (nullptr: none) are checked on the device first.
+la_status launch_decay_check(const float* decay, int heads, uint8_t* ws, cudaStream_t st) {
+    la::decay_check_kernel<<<1, 256, 0, st>>>(decay, heads, reinterpret_cast<Control*>(ws));
+    note_launch();
+    return cuda_check();
+}
+
 la_status launch_chain(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens, int num_seqs,
                        int64_t total_tokens, int heads, int d, int B, const float* init_state, float* state_out,
-                       uint8_t* ws, const Layout& L, cudaStream_t st) {
+                       uint8_t* ws, const Layout& L, cudaStream_t st, const float* decay = nullptr) {
     la_status s;
     const Control* ctrl = reinterpret_cast<const Control*>(ws);
     la::SeqEntry* seqs = reinterpret_cast<la::SeqEntry*>(ws + L.off_seqs);
@@ -312,13 +355,15 @@ la_status launch_chain(const void* q, const void* k, const void* v, void* o, con
                                              reinterpret_cast<Control*>(ws));
     note_launch();
     if ((s = cuda_check()) != LA_OK) return s;
+    if (decay && (s = launch_decay_check(decay, heads, ws, st)) != LA_OK) return s;
     if (state_out && init_state != state_out) {
         const int64_t per_seq4 = (int64_t)heads * d * d / 4;
         const int sms = num_sms();
         if (sms <= 0) return LA_ERR_CUDA;
         const int64_t want = ((int64_t)num_seqs * per_seq4 + 255) / 256;
         la::empty_states_kernel<<<(unsigned)std::min<int64_t>(want, (int64_t)sms * 4), 256, 0, st>>>(
-            seqs, num_seqs, per_seq4, reinterpret_cast<const float4*>(init_state), reinterpret_cast<float4*>(state_out));
+            seqs, num_seqs, per_seq4, reinterpret_cast<const float4*>(init_state), reinterpret_cast<float4*>(state_out),
+            ctrl);
         note_launch();
         if ((s = cuda_check()) != LA_OK) return s;
     }
@@ -342,6 +387,7 @@ la_status launch_chain(const void* q, const void* k, const void* v, void* o, con
     prm.nseq = num_seqs;
     prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
     prm.suppress_item = t_suppress_tile;
+    prm.decay = decay;
     const int64_t items = 2 * (int64_t)num_seqs * heads;
     const int sms = num_sms();
     if (sms <= 0) return LA_ERR_CUDA;
@@ -349,12 +395,15 @@ la_status launch_chain(const void* q, const void* k, const void* v, void* o, con
     const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
     prm.trace = (t_trace && t_trace_bytes >= per_block) ? t_trace : nullptr;
     prm.trace_blocks = prm.trace ? (int)std::min<size_t>(t_trace_bytes / per_block, 1 << 30) : 0;
-    auto kernel = state_out ? la::chain::prefill_chain_kernel<true> : la::chain::prefill_chain_kernel<false>;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)la::chain::SMEM_BYTES) !=
-        cudaSuccess)
+    auto kernel = decay ? (state_out ? la::chain::prefill_chain_kernel<true, true>
+                                     : la::chain::prefill_chain_kernel<false, true>)
+                        : (state_out ? la::chain::prefill_chain_kernel<true, false>
+                                     : la::chain::prefill_chain_kernel<false, false>);
+    const uint32_t smem = decay ? la::chain::Smem<true>::BYTES : la::chain::Smem<false>::BYTES;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return LA_ERR_CUDA;
     MainKernelTimer timer(st);
-    kernel<<<grid, la::chain::NTHREADS, la::chain::SMEM_BYTES, st>>>(tq, tk, tv, prm);
+    kernel<<<grid, la::chain::NTHREADS, smem, st>>>(tq, tk, tv, prm);
     note_launch();
     return cuda_check();
 }
@@ -495,14 +544,15 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o, const
     }
 
     // CUDA-core path
-    if ((s = simt_states_d(d, dtype, k, v, heads, L, ws, st)) != LA_OK) return s;
+    if ((s = simt_states_d(d, dtype, k, v, heads, L, ws, nullptr, st)) != LA_OK) return s;
     dim3 sg((dd + 1023) / 1024, num_seqs * heads);
     la::chain_scan_kernel<float><<<sg, 256, 0, st>>>(U, reinterpret_cast<float*>(ws + L.off_prefix), init_state,
-                                                     nullptr, seq_blk, ctrl, num_seqs, heads, dd, true);
+                                                     nullptr, seq_blk, ctrl, num_seqs, heads, dd, true, table,
+                                                     nullptr);
     note_launch();
     if ((s = cuda_check()) != LA_OK) return s;
     MainKernelTimer timer(st);
-    return simt_prefill_d(d, dtype, q, k, v, o, heads, B, L, ws, st);
+    return simt_prefill_d(d, dtype, q, k, v, o, heads, B, L, ws, nullptr, st);
 }
 
 la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_seqlens, int num_seqs,
@@ -555,13 +605,13 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
         return cuda_check();
     }
     if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, kStateBlock, heads, L, ws, st)) != LA_OK) return s;
-    if (total_tokens > 0 && (s = simt_states_d(d, dtype, k, v, heads, L, ws, st)) != LA_OK) return s;
+    if (total_tokens > 0 && (s = simt_states_d(d, dtype, k, v, heads, L, ws, nullptr, st)) != LA_OK) return s;
     const int dd = d * d;
     dim3 sg((dd + 1023) / 1024, num_seqs * heads);
     la::chain_scan_kernel<float><<<sg, 256, 0, st>>>(
         reinterpret_cast<const float*>(ws + L.off_U), static_cast<float*>(nullptr), init_state, state_out,
         reinterpret_cast<const int32_t*>(ws + L.off_seq_blk), reinterpret_cast<const Control*>(ws), num_seqs,
-        heads, dd, false);
+        heads, dd, false, reinterpret_cast<const BlockEntry*>(ws + L.off_table), nullptr);
     note_launch();
     return cuda_check();
 }
@@ -584,7 +634,7 @@ la_status la_decode_step(const void* q, const void* k, const void* v, float* sta
         return LA_ERR_INVALID_ARGUMENT;
     if (pairs >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;
     MainKernelTimer timer(reinterpret_cast<cudaStream_t>(stream));
-    return decode_d(d, dtype, q, k, v, state, o, pairs, reinterpret_cast<cudaStream_t>(stream));
+    return decode_d(d, dtype, q, k, v, state, o, pairs, nullptr, heads, reinterpret_cast<cudaStream_t>(stream));
 }
 
 la_status la_state_exclusive_prefix(const float* gathered, int world, int rank, int64_t n, int d, const float* init,
@@ -738,6 +788,157 @@ la_status la_prefill_backward(const void* q, const void* k, const void* v, const
     return LA_OK;
 }
 
+// ---------------------------------------------------------------- decay variant
+size_t la_prefill_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B, la_dtype dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || heads < 1 || !supported_d(d) || !supported_B(B) ||
+        (dtype != LA_BF16 && dtype != LA_FP32))
+        return 0;
+    if (total_tokens > 0 && prefill_path(dtype, d, B, num_seqs, heads) == Path::chain)
+        return prefill_layout(total_tokens, num_seqs, heads, d, B, dtype).total;
+    return simt_layout(total_tokens, num_seqs, heads, d, B).total;
+}
+
+la_status la_prefill_decay(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                           int num_seqs, int64_t total_tokens, int heads, int d, int B, la_dtype dtype,
+                           const float* init_state, const float* decay, float* state_out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    la_status s = check_prefill(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state);
+    if (s != LA_OK) return s;
+    if (!decay) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(decay, 4)) return LA_ERR_MISALIGNED;
+    const size_t tb = (size_t)total_tokens * heads * d * esize(dtype);
+    const size_t sb = (size_t)num_seqs * heads * d * d * 4;
+    const size_t db = (size_t)heads * 4;
+    if (overlaps(decay, db, o, tb)) return LA_ERR_INVALID_ARGUMENT;
+    if (state_out) {
+        if (!aligned(state_out, 16)) return LA_ERR_MISALIGNED;
+        // state_out may be init_state itself: the scan reads each element of S0 before it writes it
+        if (init_state && init_state != state_out && overlaps(state_out, sb, init_state, sb))
+            return LA_ERR_INVALID_ARGUMENT;
+        if (overlaps(state_out, sb, o, tb) || overlaps(state_out, sb, q, tb) || overlaps(state_out, sb, k, tb) ||
+            overlaps(state_out, sb, v, tb) || overlaps(state_out, sb, decay, db))
+            return LA_ERR_INVALID_ARGUMENT;
+    }
+    if (total_tokens == 0 && !state_out) return LA_OK;
+    // the on-chip-state tensor-core kernel where la_prefill would use it, else CUDA cores
+    const bool chain = total_tokens > 0 && prefill_path(dtype, d, B, num_seqs, heads) == Path::chain;
+    const Layout L = chain ? prefill_layout(total_tokens, num_seqs, heads, d, B, dtype)
+                           : simt_layout(total_tokens, num_seqs, heads, d, B);
+    if (!workspace) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
+    if (overlaps(workspace, L.total, o, tb) || overlaps(workspace, L.total, decay, db) ||
+        (state_out && overlaps(workspace, L.total, state_out, sb)))
+        return LA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (chain)
+        return launch_chain(q, k, v, o, cu_seqlens, num_seqs, total_tokens, heads, d, B, init_state, state_out, ws, L,
+                            st, decay);
+    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, B, heads, L, ws, st)) != LA_OK) return s;
+    if ((s = launch_decay_check(decay, heads, ws, st)) != LA_OK) return s;
+    if (total_tokens > 0 && (s = simt_states_d(d, dtype, k, v, heads, L, ws, decay, st)) != LA_OK) return s;
+    const int dd = d * d;
+    dim3 sg((dd + 1023) / 1024, num_seqs * heads);
+    la::chain_scan_kernel<float><<<sg, 256, 0, st>>>(
+        reinterpret_cast<const float*>(ws + L.off_U), reinterpret_cast<float*>(ws + L.off_prefix), init_state,
+        state_out, reinterpret_cast<const int32_t*>(ws + L.off_seq_blk), reinterpret_cast<const Control*>(ws),
+        num_seqs, heads, dd, state_out == nullptr, reinterpret_cast<const BlockEntry*>(ws + L.off_table), decay);
+    note_launch();
+    if ((s = cuda_check()) != LA_OK) return s;
+    if (total_tokens == 0) return LA_OK;
+    MainKernelTimer timer(st);
+    return simt_prefill_d(d, dtype, q, k, v, o, heads, B, L, ws, decay, st);
+}
+
+size_t la_state_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, la_dtype dtype) {
+    if (total_tokens < 0 || num_seqs < 1 || heads < 1 || !supported_d(d) || (dtype != LA_BF16 && dtype != LA_FP32))
+        return 0;
+    return simt_state_layout(total_tokens, num_seqs, heads, d).total;
+}
+
+la_status la_state_decay(const void* k, const void* v, const int32_t* cu_seqlens, int num_seqs,
+                         int64_t total_tokens, int heads, int d, la_dtype dtype, const float* init_state,
+                         const float* decay, float* state_out, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    la_status s = check_tokens(total_tokens, num_seqs, heads, d, dtype, cu_seqlens);
+    if (s != LA_OK) return s;
+    if (!state_out || !decay || (total_tokens > 0 && (!k || !v))) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(state_out, 16) || !aligned(decay, 4)) return LA_ERR_MISALIGNED;
+    if (init_state && !aligned(init_state, 16)) return LA_ERR_MISALIGNED;
+    const size_t sb = (size_t)num_seqs * heads * d * d * 4;
+    const size_t tb = (size_t)total_tokens * heads * d * esize(dtype);
+    if (init_state && init_state != state_out && overlaps(init_state, sb, state_out, sb)) return LA_ERR_INVALID_ARGUMENT;
+    if (overlaps(state_out, sb, k, tb) || overlaps(state_out, sb, v, tb) || overlaps(state_out, sb, decay, heads * 4))
+        return LA_ERR_INVALID_ARGUMENT;
+    const Layout L = simt_state_layout(total_tokens, num_seqs, heads, d);
+    if (!workspace) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
+    if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
+    if (overlaps(workspace, L.total, state_out, sb)) return LA_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if ((s = launch_block_table(cu_seqlens, num_seqs, total_tokens, kStateBlock, heads, L, ws, st)) != LA_OK) return s;
+    if ((s = launch_decay_check(decay, heads, ws, st)) != LA_OK) return s;
+    if (total_tokens > 0 && (s = simt_states_d(d, dtype, k, v, heads, L, ws, decay, st)) != LA_OK) return s;
+    const int dd = d * d;
+    dim3 sg((dd + 1023) / 1024, num_seqs * heads);
+    la::chain_scan_kernel<float><<<sg, 256, 0, st>>>(
+        reinterpret_cast<const float*>(ws + L.off_U), static_cast<float*>(nullptr), init_state, state_out,
+        reinterpret_cast<const int32_t*>(ws + L.off_seq_blk), reinterpret_cast<const Control*>(ws), num_seqs,
+        heads, dd, false, reinterpret_cast<const BlockEntry*>(ws + L.off_table), decay);
+    note_launch();
+    return cuda_check();
+}
+
+la_status la_decode_step_decay(const void* q, const void* k, const void* v, float* state, void* o, int batch,
+                               int heads, int d, la_dtype dtype, const float* decay, void* stream) {
+    if (batch < 0 || heads < 1) return LA_ERR_INVALID_ARGUMENT;
+    if (dtype != LA_BF16 && dtype != LA_FP32) return LA_ERR_UNSUPPORTED;
+    if (!supported_d(d)) return LA_ERR_UNSUPPORTED;
+    if (batch == 0) return LA_OK;
+    if (!q || !k || !v || !state || !o || !decay) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(state, 16) ||
+        !aligned(decay, 4))
+        return LA_ERR_MISALIGNED;
+    const int64_t pairs = (int64_t)batch * heads;
+    const size_t vec = (size_t)pairs * d * esize(dtype);
+    const size_t sbytes = (size_t)pairs * d * d * 4;
+    const size_t db = (size_t)heads * 4;
+    if (overlaps(o, vec, q, vec) || overlaps(o, vec, k, vec) || overlaps(o, vec, v, vec) ||
+        overlaps(o, vec, state, sbytes) || overlaps(state, sbytes, q, vec) || overlaps(state, sbytes, k, vec) ||
+        overlaps(state, sbytes, v, vec) || overlaps(decay, db, state, sbytes) || overlaps(decay, db, o, vec))
+        return LA_ERR_INVALID_ARGUMENT;
+    if (pairs >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;
+    MainKernelTimer timer(reinterpret_cast<cudaStream_t>(stream));
+    return decode_d(d, dtype, q, k, v, state, o, pairs, decay, heads, reinterpret_cast<cudaStream_t>(stream));
+}
+
+la_status la_feature_map(const void* x, void* y, int64_t n, la_dtype dtype, float alpha, void* stream) {
+    if (n < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (dtype != LA_BF16 && dtype != LA_FP32) return LA_ERR_UNSUPPORTED;
+    if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) return LA_ERR_INVALID_ARGUMENT;
+    if (n == 0) return LA_OK;
+    if (!x || !y) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(x, 16) || !aligned(y, 16)) return LA_ERR_MISALIGNED;
+    const size_t bytes = (size_t)n * esize(dtype);
+    if (x != y && overlaps(x, bytes, y, bytes)) return LA_ERR_INVALID_ARGUMENT;
+    const int sms = num_sms();
+    if (sms <= 0) return LA_ERR_CUDA;
+    const int64_t groups = n / (16 / (int64_t)esize(dtype));
+    const int64_t want = std::max<int64_t>(1, (groups + 255) / 256);
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)sms * 8);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == LA_BF16)
+        la::feature_map_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), n, alpha);
+    else
+        la::feature_map_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), static_cast<float*>(y), n,
+                                                             alpha);
+    note_launch();
+    return cuda_check();
+}
+
 la_status la_get_device_status(void* stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return LA_ERR_CUDA;
     int v = 0, zero = 0;
@@ -786,6 +987,7 @@ const char* la_status_string(la_status s) {
         case LA_ERR_CUDA: return "CUDA error";
         case LA_ERR_TIMEOUT: return "device-side wait timed out";
         case LA_ERR_BAD_SEQLENS: return "cu_seqlens inconsistent with total_tokens";
+        case LA_ERR_BAD_DECAY: return "a decay rate outside [0, 1]";
     }
     return "unknown status";
 }

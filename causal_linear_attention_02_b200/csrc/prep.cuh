@@ -8,6 +8,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "decay.cuh"
 
 namespace la {
 
@@ -194,7 +195,9 @@ __global__ void __launch_bounds__(1024) seq_table_kernel(const int32_t* __restri
 
 // Exclusive prefix over the blocks of every (sequence, head) chain:
 //   prefix[g] = S0 + sum_{blocks c of the same sequence before g} U[c]
-// and, optionally, the chain total S0 + sum_all U into state_out.
+// and, optionally, the chain total S0 + sum_all U into state_out. With a
+// per-head decay rate (decay != nullptr; decay.cuh) the running state is
+// multiplied by lambda^len(g) before U[g] is added.
 // U, prefix: [block][H][d*d]; init, state_out: [nseq][H][d*d].
 // grid = (ceil(d*d / 1024), nseq * H), 256 threads, 4 consecutive elements per thread.
 template <typename OutT>
@@ -203,10 +206,13 @@ __global__ void __launch_bounds__(256) chain_scan_kernel(const float* __restrict
                                                          const float* init, float* state_out,
                                                          const int32_t* __restrict__ seq_blk,
                                                          const Control* __restrict__ ctrl,
-                                                         int nseq, int H, int dd, bool skip_last) {
+                                                         int nseq, int H, int dd, bool skip_last,
+                                                         const BlockEntry* __restrict__ table, const float* decay) {
     if (!ctrl->ok) return;
     const int chain = blockIdx.y;
     const int s = chain / H, h = chain % H;
+    float l2 = 0.f;
+    if (decay && !load_decay(decay, h, l2)) return;
     const int e = (blockIdx.x * 256 + threadIdx.x) * 4;
     if (e >= dd) return;
     const int64_t g0 = seq_blk[s], g1 = seq_blk[s + 1];
@@ -231,7 +237,13 @@ __global__ void __launch_bounds__(256) chain_scan_kernel(const float* __restrict
             const float4 u = nxt;
             if (g + 1 < gend)
                 nxt = __ldcs(reinterpret_cast<const float4*>(U + ((int64_t)(g + 1) * H + h) * dd + e));
-            run.x += u.x; run.y += u.y; run.z += u.z; run.w += u.w;
+            if (decay) {
+                const float w = decay_pow(l2, table[g].len);
+                run.x = fmaf(w, run.x, u.x); run.y = fmaf(w, run.y, u.y);
+                run.z = fmaf(w, run.z, u.z); run.w = fmaf(w, run.w, u.w);
+            } else {
+                run.x += u.x; run.y += u.y; run.z += u.z; run.w += u.w;
+            }
         }
     }
     if (state_out) *reinterpret_cast<float4*>(state_out + ((int64_t)s * H + h) * dd + e) = run;
@@ -239,9 +251,12 @@ __global__ void __launch_bounds__(256) chain_scan_kernel(const float* __restrict
 
 // Final states of the empty sequences for la_prefill_with_state (the prefill
 // kernel visits only sequences with tokens): S0, or zero without one. One
-// 16-byte group per thread and iteration over [nseq][H][d][d].
+// 16-byte group per thread and iteration over [nseq][H][d][d]. Nothing when
+// the call's checks failed (ctrl->ok = 0).
 __global__ void __launch_bounds__(256)
-empty_states_kernel(const SeqEntry* seqs, int nseq, int64_t per_seq4, const float4* init, float4* out) {
+empty_states_kernel(const SeqEntry* seqs, int nseq, int64_t per_seq4, const float4* init, float4* out,
+                    const Control* ctrl) {
+    if (!ctrl->ok) return;
     const int64_t total = (int64_t)nseq * per_seq4;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         if (seqs[i / per_seq4].len > 0) continue;

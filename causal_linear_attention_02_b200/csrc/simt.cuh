@@ -5,9 +5,13 @@
 //   block_state_simt : U_b = K_b^T V_b over the valid rows of block b
 //   (chain_scan_kernel turns U into per-block prefix states)
 //   prefill_simt     : O_b = (Q_b K_b^T masked) V_b + Q_b . prefix_b
+// The kDecay instances add a per-head decay rate on the state (decay.cuh): key
+// rows weighted lambda^(n-1-r) in U_b, the decay mask lambda^(t-u) on the
+// scores and lambda^(r+1) on the inter-block product.
 #pragma once
 
 #include "common.cuh"
+#include "decay.cuh"
 
 namespace la {
 namespace simt {
@@ -18,11 +22,11 @@ constexpr int THREADS = 256;
 // One CTA per (block, head); tokens staged through shared memory 32 at a time.
 // Thread (ti, tj) of a 16 x 16 grid owns the (D/16) x (D/16) micro-tile
 // rows ti*(D/16).., cols tj*(D/16)...
-template <typename Tin, int D>
+template <typename Tin, int D, bool kDecay = false>
 __global__ void __launch_bounds__(THREADS) block_state_simt(const Tin* __restrict__ k, const Tin* __restrict__ v,
                                                             const BlockEntry* __restrict__ table,
                                                             const Control* __restrict__ ctrl, int H,
-                                                            float* __restrict__ U) {
+                                                            float* __restrict__ U, const float* decay) {
     constexpr int MT = D / 16;
     constexpr int CH = 32;
     __shared__ float ks[CH][D];
@@ -31,6 +35,10 @@ __global__ void __launch_bounds__(THREADS) block_state_simt(const Tin* __restric
     const int h = blockIdx.x % H;
     if (g >= ctrl->nblocks) return;
     const BlockEntry e = table[g];
+    float l2 = 0.f;
+    if constexpr (kDecay) {
+        if (!load_decay(decay, h, l2)) return;
+    }
     const int tid = threadIdx.x, ti = tid / 16, tj = tid % 16;
     float acc[MT][MT];
 #pragma unroll
@@ -46,6 +54,7 @@ __global__ void __launch_bounds__(THREADS) block_state_simt(const Tin* __restric
                 const int64_t off = ((int64_t)(e.tok0 + t0 + r) * H + h) * D + c;
                 kv = io<Tin>::ld(k + off);
                 vv = io<Tin>::ld(v + off);
+                if constexpr (kDecay) kv *= decay_pow(l2, e.len - 1 - (t0 + r));
             }
             ks[r][c] = kv;
             vs[r][c] = vv;
@@ -76,12 +85,13 @@ __global__ void __launch_bounds__(THREADS) block_state_simt(const Tin* __restric
 //   acc += sum over 64-key tiles kt <= qt of (Q_tile K_kt^T masked) V_kt  (intra left product)
 // prefix is fp32 [block][H][D][D]. Thread (ti, tj) of 16 x 16 owns rows
 // ti*4..ti*4+3 and columns tj*(D/16)...
-template <typename Tin, int D>
+template <typename Tin, int D, bool kDecay = false>
 __global__ void __launch_bounds__(THREADS) prefill_simt(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                         const Tin* __restrict__ v, Tin* __restrict__ o,
                                                         const float* __restrict__ prefix,
                                                         const BlockEntry* __restrict__ table,
-                                                        const Control* __restrict__ ctrl, int H, int B) {
+                                                        const Control* __restrict__ ctrl, int H, int B,
+                                                        const float* decay) {
     constexpr int MT = D / 16;
     constexpr int QT = 64;
     extern __shared__ float4 smem_f4[];
@@ -99,6 +109,10 @@ __global__ void __launch_bounds__(THREADS) prefill_simt(const Tin* __restrict__ 
     const int r0 = qt * QT;
     if (r0 >= e.len) return;
     const int nq = min(QT, e.len - r0);
+    float l2 = 0.f;
+    if constexpr (kDecay) {
+        if (!load_decay(decay, h, l2)) return;
+    }
     const int tid = threadIdx.x, ti = tid / 16, tj = tid % 16;
 
     for (int x = tid; x < QT * D; x += THREADS) {
@@ -128,6 +142,14 @@ __global__ void __launch_bounds__(THREADS) prefill_simt(const Tin* __restrict__ 
 #pragma unroll
                 for (int b = 0; b < MT; ++b) acc[a][b] = fmaf(qa, pr[b], acc[a][b]);
             }
+        }
+    }
+    if constexpr (kDecay) {   // lambda^(r+1) on the inter-block product of row r of the block
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const float w = decay_pow(l2, r0 + ti * 4 + a + 1);
+#pragma unroll
+            for (int b = 0; b < MT; ++b) acc[a][b] *= w;
         }
     }
     // intra-block: key tiles up to and including the diagonal tile
@@ -170,7 +192,9 @@ __global__ void __launch_bounds__(THREADS) prefill_simt(const Tin* __restrict__ 
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
                     const int qi = r0 + ti * 4 + a, kj = k0 + tj * 4 + b;   // positions in the block
-                    ss[(ti * 4 + a) * (QT + 1) + tj * 4 + b] = (kj <= qi && kj < e.len) ? sc[a][b] : 0.f;
+                    float x = (kj <= qi && kj < e.len) ? sc[a][b] : 0.f;
+                    if constexpr (kDecay) x *= decay_pow(l2, max(qi - kj, 0));
+                    ss[(ti * 4 + a) * (QT + 1) + tj * 4 + b] = x;
                 }
         }
         __syncthreads();

@@ -59,7 +59,8 @@ typedef enum {
     LA_ERR_WORKSPACE_TOO_SMALL = 4, /* workspace_bytes below the *_workspace_size() result     */
     LA_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed                   */
     LA_ERR_TIMEOUT = 6,             /* device: a bounded wait ran out (reported by status)    */
-    LA_ERR_BAD_SEQLENS = 7          /* device: cu_seqlens not 0..total_tokens non-decreasing  */
+    LA_ERR_BAD_SEQLENS = 7,         /* device: cu_seqlens not 0..total_tokens non-decreasing  */
+    LA_ERR_BAD_DECAY = 8            /* device: a decay rate outside [0, 1] (or NaN)            */
 } la_status;
 
 typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
@@ -217,11 +218,92 @@ la_status la_state_exclusive_prefix(const float* gathered, int world, int rank, 
 la_status la_decode_step(const void* q, const void* k, const void* v, float* state, void* o,
                          int batch, int heads, int d, la_dtype dtype, void* stream);
 
+/* ------------------------------------------------------------------ decay variant
+ * Not on the pages: Lightning Attention with a decay rate per head on the
+ * state, the Lightning Attention-2 form of the same method taken in its
+ * plainest reading (a rate of 1 is the method without decay):
+ *
+ *     S_t = lambda_h S_{t-1} + k_t^T v_t,   S_{start-1} = S0,   o_t = q_t S_t
+ *     O_t = lambda^(t-start+1) q_t . S0 + sum_{s in seq(t), s <= t} lambda^(t-s) (q_t . k_s) v_s
+ *
+ * `decay` is fp32 [heads] in device memory, 4-byte aligned, read only, each
+ * rate in [0, 1]; lambda^0 = 1 also for lambda = 0. A rate outside [0, 1] or
+ * NaN is a device-side condition: la_get_device_status reports
+ * LA_ERR_BAD_DECAY; la_prefill_decay and la_state_decay then write nothing at
+ * all, la_decode_step_decay nothing for that head.
+ * la_prefill_decay runs on the on-chip-state tensor-core kernel where
+ * la_prefill would (bf16, d = 128, B in {128, 256}, at least 64 work items of
+ * (sequence, head, value half)); there the state's increments read
+ * lambda^(n-1-c) v_c rounded to bf16. Every other shape, and la_state_decay,
+ * runs on CUDA cores in fp32.
+ */
+
+/* Workspace for la_prefill_decay; 0 for an unsupported shape. */
+size_t la_prefill_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                       la_dtype dtype);
+
+/*
+ * Prefill with decay. Arguments, layouts and errors as la_prefill, plus:
+ *   decay      in   fp32 [heads] (see above); may not overlap o, state_out or the workspace
+ *   state_out  out  fp32 [num_seqs][heads][d][d], each sequence's final state
+ *                   lambda^n S0 + sum_t lambda^(end-1-t) k_t^T v_t, or NULL for none. It may
+ *                   be init_state itself (updated in place); it may not overlap any other
+ *                   argument. Empty sequences get S0 (or zero).
+ * Block decomposition (block of n tokens from b0, KV the state before b0, r = t - b0):
+ *   O_t = sum_{u=b0..t} lambda^(t-u) (q_t . k_u) v_u + lambda^(r+1) q_t KV,
+ *   KV' = lambda^n KV + sum_u lambda^(b0+n-1-u) k_u^T v_u;
+ * the result does not depend on B beyond rounding. Launches: tensor-core path:
+ * sequence table, rate check, (empty-sequence states,) prefill; CUDA cores:
+ * block table (2), rate check, block states, scan, prefill.
+ */
+la_status la_prefill_decay(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens,
+                           int num_seqs, int64_t total_tokens, int heads, int d, int B, la_dtype dtype,
+                           const float* init_state, const float* decay, float* state_out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Workspace for la_state_decay; 0 for an unsupported shape. */
+size_t la_state_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, la_dtype dtype);
+
+/*
+ * Final state with decay of each sequence, without the output:
+ *   state_out[s][h] = lambda_h^n S0 + sum_t lambda_h^(end-1-t) k_t^T v_t  (n tokens).
+ * Arguments and errors as la_state_from_prefill, plus `decay` as above.
+ */
+la_status la_state_decay(const void* k, const void* v, const int32_t* cu_seqlens, int num_seqs,
+                         int64_t total_tokens, int heads, int d, la_dtype dtype, const float* init_state,
+                         const float* decay, float* state_out, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * One decode step with decay: S <- lambda_h S + k^T v ; o = q S.
+ * Arguments and errors as la_decode_step, plus `decay` as above (it may not
+ * overlap state or o). Same bandwidth as la_decode_step: one read and one
+ * write of the fp32 state.
+ */
+la_status la_decode_step_decay(const void* q, const void* k, const void* v, float* state, void* o, int batch,
+                               int heads, int d, la_dtype dtype, const float* decay, void* stream);
+
+/*
+ * Feature map phi(x) = ELU(x) + alpha x, elementwise over n values (page
+ * "MiniMax-M2.5语言模型：Linear Attention架构解析与实践", section "2.2 Linear
+ * Attention的数学原理", which takes alpha = 0.3; ELU(x) = x for x > 0,
+ * e^x - 1 otherwise). A pre-pass for q and k before a prefill or decode step,
+ * for callers that want the feature map; the prefill itself uses q and k as
+ * given.
+ *   x  in   n values of `dtype`, 16-byte aligned
+ *   y  out  n values of `dtype`, 16-byte aligned; may be x itself (in place),
+ *           may not overlap x otherwise
+ * Computed in fp32, rounded to nearest even for bf16. Errors:
+ * LA_ERR_INVALID_ARGUMENT (n < 0, null pointer, partial overlap, alpha not
+ * finite), LA_ERR_UNSUPPORTED (dtype), LA_ERR_MISALIGNED.
+ */
+la_status la_feature_map(const void* x, void* y, int64_t n, la_dtype dtype, float alpha, void* stream);
+
 /*
  * Synchronises `stream`, then returns and clears the status word of the
- * current device: LA_OK, LA_ERR_BAD_SEQLENS or LA_ERR_TIMEOUT (the first
- * condition recorded since the last call), or LA_ERR_CUDA if the
- * synchronisation itself failed.
+ * current device: LA_OK, LA_ERR_BAD_SEQLENS, LA_ERR_TIMEOUT or
+ * LA_ERR_BAD_DECAY (the first condition recorded since the last call), or
+ * LA_ERR_CUDA if the synchronisation itself failed.
  */
 la_status la_get_device_status(void* stream);
 

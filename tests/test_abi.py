@@ -118,6 +118,62 @@ def test_state_argument_errors(lib):
     assert st(init=4 * P + 1024) == 1                   # partial overlap of init and out
 
 
+def test_decay_argument_errors(lib):
+    """Host checks of the decay entry points (each case fails before any launch)."""
+    def pre(**kw):
+        a = dict(q=P, k=2 * P, v=3 * P, o=4 * P, cu=None, nseq=1, T=64, H=2, d=128, B=256, dt=la.LA_BF16,
+                 init=None, decay=6 * P, out=None, ws=5 * P, wsb=BIG)
+        a.update(kw)
+        return la.la_prefill_decay(a["q"], a["k"], a["v"], a["o"], a["cu"], a["nseq"], a["T"], a["H"], a["d"],
+                                   a["B"], a["dt"], a["init"], a["decay"], a["out"], a["ws"], a["wsb"], None)
+    assert pre(decay=None) == 1
+    assert pre(decay=6 * P + 2) == 3                    # rates are 4-byte aligned fp32
+    assert pre(decay=4 * P) == 1                        # rates inside the output
+    assert pre(d=100) == 2
+    assert pre(B=32) == 2
+    assert pre(out=8 * P + 4) == 3
+    assert pre(out=4 * P) == 1                          # state_out overlaps o
+    assert pre(init=8 * P, out=8 * P + 4096) == 1       # state_out partially overlaps init
+    assert pre(wsb=16) == 4
+    assert pre(ws=None) == 1
+    assert pre(T=0) == 0                                # nothing to compute, no state asked for
+
+    def st(**kw):
+        a = dict(k=P, v=2 * P, cu=None, nseq=1, T=64, H=2, d=64, dt=la.LA_FP32, init=None, decay=6 * P,
+                 out=4 * P, ws=5 * P, wsb=BIG)
+        a.update(kw)
+        return la.la_state_decay(a["k"], a["v"], a["cu"], a["nseq"], a["T"], a["H"], a["d"], a["dt"], a["init"],
+                                 a["decay"], a["out"], a["ws"], a["wsb"], None)
+    assert st(decay=None) == 1
+    assert st(out=None) == 1
+    assert st(decay=4 * P) == 1                         # rates inside the state
+    assert st(wsb=8) == 4
+
+    def dec(**kw):
+        a = dict(q=P, k=2 * P, v=3 * P, s=8 * P, o=4 * P, b=4, H=2, d=128, dt=la.LA_BF16, decay=6 * P)
+        a.update(kw)
+        return la.la_decode_step_decay(a["q"], a["k"], a["v"], a["s"], a["o"], a["b"], a["H"], a["d"], a["dt"],
+                                       a["decay"], None)
+    assert dec(decay=None) == 1
+    assert dec(decay=8 * P) == 1                        # rates inside the state
+    assert dec(decay=6 * P + 1) == 3
+    assert dec(s=2 * P) == 1
+    assert dec(b=0) == 0
+
+    def fm(**kw):
+        a = dict(x=P, y=2 * P, n=100, dt=la.LA_BF16, alpha=0.3)
+        a.update(kw)
+        return la.la_feature_map(a["x"], a["y"], a["n"], a["dt"], a["alpha"], None)
+    assert fm(n=-1) == 1
+    assert fm(dt=3) == 2
+    assert fm(x=None) == 1
+    assert fm(x=P + 8) == 3
+    assert fm(y=P + 64) == 1                            # partial overlap (in place is y == x)
+    assert fm(alpha=float("nan")) == 1
+    assert fm(alpha=float("inf")) == 1
+    assert fm(n=0) == 0
+
+
 def test_workspace_sizes(lib):
     assert la.la_prefill_workspace_size(32768, 1, 64, 128, 256, la.LA_BF16) > 0
     assert la.la_prefill_workspace_size(32768, 1, 64, 100, 256, la.LA_BF16) == 0
@@ -127,6 +183,9 @@ def test_workspace_sizes(lib):
     assert b > a
     assert la.la_state_workspace_size(4096, 2, 4, 64, la.LA_FP32) > 0
     assert la.la_prefill_workspace_size(100, 1, 1, 64, 64, la.LA_FP32) % 256 == 0
+    assert la.la_prefill_decay_workspace_size(32768, 1, 64, 128, 256, la.LA_BF16) > 0
+    assert la.la_prefill_decay_workspace_size(32768, 1, 64, 128, 48, la.LA_BF16) == 0
+    assert la.la_state_decay_workspace_size(4096, 2, 4, 64, la.LA_FP32) > 0
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

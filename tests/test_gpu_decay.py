@@ -1,0 +1,304 @@
+"""GPU parity of the decay variant and of the feature map, through the C ABI,
+against the fp64 oracle.
+
+Decay (not on the pages; the Lightning Attention-2 form of the method):
+S_t = lambda_h S_{t-1} + k_t^T v_t, o_t = q_t S_t. Tolerances as for the
+method without decay: max|O - O_ref| <= 1e-2 max|O_ref| for bf16 inputs and
+1e-4 for fp32; states 1e-4 max|S_ref| on the CUDA-core path (fp32 arithmetic
+on both input types). On the tensor-core path (bf16, d = 128, B in {128, 256},
+the on-chip-state kernel) the state MMAs read lambda^(n-1-c) v_c rounded to
+bf16, one rounding of relative size <= 2^-9 per term, so its states are held
+to 5e-3 max|S_ref|.
+Feature map phi(x) = ELU(x) + alpha x: elementwise, within 2^-8 of |phi| for
+bf16 outputs (one rounding to bf16) and 1e-6 for fp32.
+"""
+import numpy as np
+import pytest
+import torch
+
+import causal_linear_attention_02_b200 as la
+import oracle
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+TOL = {torch.bfloat16: 1e-2, torch.float32: 1e-4}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    from causal_linear_attention_02_b200 import build
+    build.build()
+    la.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.set_device(DEV)
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def assert_close(out, ref, tol, what=""):
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    r = float(np.abs(out - ref).max(initial=0.0) / max(np.abs(ref).max(initial=0.0), 1e-30))
+    assert r <= tol, f"{what}: max|x - x_ref| / max|x_ref| = {r:.3e} > {tol:.0e}"
+
+
+def status_ok():
+    s = la.device_status()
+    assert s == 0, f"device status {la.STATUS.get(s, s)}"
+
+
+STATE_TOL = {"auto": 1e-4, "onchip": 5e-3}
+
+
+@pytest.fixture(params=["auto", "onchip"])
+def path(request):
+    """auto: the path la_prefill_decay picks (CUDA cores below 64 work items); onchip: the
+    on-chip-state tensor-core kernel forced (la_debug_set_path(1), bf16 d = 128 only)."""
+    assert la.la_debug_set_path(1 if request.param == "onchip" else 0) == 0
+    yield request.param
+    la.la_debug_set_path(0)
+
+
+RATES = {  # per-head rates: the edges 0 and 1, and rates in between
+    2: [0.9, 0.999],
+    4: [0.0, 0.5, 0.95, 1.0],
+}
+
+
+@pytest.mark.parametrize("dtype,d,B,lengths,H", [
+    (torch.float32, 64, 64, [1024], 2),               # the small fp32 workload's shape
+    (torch.bfloat16, 128, 256, [1000, 1, 0, 513], 4),
+    (torch.bfloat16, 128, 128, [300, 129], 4),
+    (torch.bfloat16, 32, 64, [77, 200], 2),
+    (torch.float32, 16, 256, [600, 3], 4),
+    (torch.float32, 128, 128, [257], 2),
+], ids=lambda x: str(x).replace(" ", ""))
+@pytest.mark.parametrize("with_init", [False, True], ids=["zero-S0", "S0"])
+def test_prefill_decay(dtype, d, B, lengths, H, with_init, path):
+    if path == "onchip" and not la.uses_tensor_cores(dtype, d, B):
+        pytest.skip("no tensor-core path for this shape")
+    T = sum(lengths)
+    q, k, v = wl.qkv(T, H, d, dtype, seed=T + d, device=DEV)
+    cu = wl.cu_seqlens(lengths, device=DEV)
+    decay = torch.tensor(RATES[H], dtype=torch.float32, device=DEV)
+    init = wl.state_init(len(lengths), H, d, seed=5, device=DEV) if with_init else None
+    o, st = la.prefill_decay(q, k, v, decay, cu, B=B, init_state=init, return_state=True)
+    status_ok()
+    ref_o, ref_st = oracle.decay_recurrent(f64(q), f64(k), f64(v), decay.cpu().double().numpy(), cu.cpu().numpy(),
+                                           init=None if init is None else init.cpu().double().numpy(),
+                                           return_state=True)
+    assert_close(f64(o), ref_o, TOL[dtype], "decay prefill O")
+    assert_close(st.cpu().double().numpy(), ref_st, STATE_TOL[path], "decay prefill final state")
+    # the state output is optional and changes nothing else
+    o2 = la.prefill_decay(q, k, v, decay, cu, B=B, init_state=init)
+    assert torch.equal(o2, o)
+
+
+@pytest.mark.parametrize("lengths,H,B", [
+    ([1000, 1, 15, 16, 17, 0, 300], 8, 256),    # ragged tails of 1, 15, 16, 17 tokens, an empty sequence
+    ([129, 255, 2048], 12, 128),
+    ([4096], 64, 256),
+])
+def test_prefill_decay_onchip(lengths, H, B):
+    """The tensor-core path with enough work items to be the automatic choice, the decay recipe's
+    rates, S0 and the final state."""
+    T = sum(lengths)
+    q, k, v = wl.qkv(T, H, 128, torch.bfloat16, seed=T + H, device=DEV)
+    cu = wl.cu_seqlens(lengths, device=DEV)
+    decay = wl.decay_rates(H, device=DEV)
+    init = wl.state_init(len(lengths), H, 128, seed=11, device=DEV)
+    assert 2 * len(lengths) * H >= 64
+    o, st = la.prefill_decay(q, k, v, decay, cu, B=B, init_state=init, return_state=True)
+    status_ok()
+    lam = decay.cpu().double().numpy()
+    ref_o, ref_st = oracle.decay_recurrent(f64(q), f64(k), f64(v), lam, cu.cpu().numpy(),
+                                           init=init.cpu().double().numpy(), return_state=True)
+    assert_close(f64(o), ref_o, 1e-2, "O")
+    assert_close(st.cpu().double().numpy(), ref_st, 5e-3, "final state")
+    # without the state output (the other instance) the same O
+    o2 = la.prefill_decay(q, k, v, decay, cu, B=B, init_state=init)
+    status_ok()
+    assert_close(f64(o2), ref_o, 1e-2, "O without the state output")
+
+
+def test_prefill_decay_onchip_edge_rates():
+    """Rates 0 and 1 on the tensor-core path: lambda = 1 is the method, lambda = 0 keeps the
+    current token only."""
+    T, H = 700, 32
+    q, k, v = wl.qkv(T, H, 128, torch.bfloat16, seed=78, device=DEV)
+    decay = torch.tensor([0.0, 1.0] * (H // 2), dtype=torch.float32, device=DEV)
+    init = wl.state_init(1, H, 128, seed=12, device=DEV)
+    o, st = la.prefill_decay(q, k, v, decay, B=256, init_state=init, return_state=True)
+    status_ok()
+    ref_o, ref_st = oracle.decay_recurrent(f64(q), f64(k), f64(v), decay.cpu().double().numpy(),
+                                           init=init.cpu().double().numpy(), return_state=True)
+    assert_close(f64(o), ref_o, 1e-2, "O")
+    assert_close(st.cpu().double().numpy(), ref_st, 5e-3, "final state")
+    ref_plain = la.prefill(q[:, 1::2].contiguous(), k[:, 1::2].contiguous(), v[:, 1::2].contiguous(), B=256,
+                           init_state=init[:, 1::2].contiguous())
+    assert_close(f64(o[:, 1::2]), f64(ref_plain), 1e-2, "lambda = 1 against la_prefill")
+
+
+def test_prefill_decay_rate_one_is_the_method():
+    T, H, d = 700, 2, 128
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, seed=71, device=DEV)
+    decay = torch.ones(H, dtype=torch.float32, device=DEV)
+    o = la.prefill_decay(q, k, v, decay, B=256)
+    status_ok()
+    assert_close(f64(o), oracle.recurrent(f64(q), f64(k), f64(v)), 1e-2, "lambda = 1")
+
+
+def test_prefill_decay_block_size_independence():
+    T, H, d = 900, 4, 64
+    q, k, v = wl.qkv(T, H, d, torch.float32, seed=72, device=DEV)
+    decay = torch.tensor(RATES[4], dtype=torch.float32, device=DEV)
+    outs = [la.prefill_decay(q, k, v, decay, B=B) for B in (64, 128, 256)]
+    status_ok()
+    for o in outs[1:]:
+        assert_close(f64(o), f64(outs[0]), 1e-5, "B independence")
+
+
+def test_prefill_decay_state_in_place():
+    lengths, H, d = [400, 0, 90], 4, 128
+    T = sum(lengths)
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, seed=73, device=DEV)
+    cu = wl.cu_seqlens(lengths, device=DEV)
+    decay = torch.tensor(RATES[4], dtype=torch.float32, device=DEV)
+    init = wl.state_init(3, H, d, seed=6, device=DEV)
+    ref_st = oracle.decay_state(f64(k), f64(v), decay.cpu().double().numpy(), cu.cpu().numpy(),
+                                init=init.cpu().double().numpy())
+    ref_o = oracle.decay_recurrent(f64(q), f64(k), f64(v), decay.cpu().double().numpy(), cu.cpu().numpy(),
+                                   init=init.cpu().double().numpy())
+    o, st = la.prefill_decay(q, k, v, decay, cu, B=256, init_state=init, state_out=init)
+    status_ok()
+    assert st.data_ptr() == init.data_ptr()
+    assert_close(f64(o), ref_o, 1e-2, "O with the state updated in place")
+    assert_close(init.cpu().double().numpy(), ref_st, 1e-4, "state updated in place")
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+@pytest.mark.parametrize("with_init", [False, True], ids=["zero-S0", "S0"])
+def test_state_decay(dtype, d, with_init):
+    lengths, H = [5000, 0, 1, 2049], 4            # several 2048-token state blocks, empty and 1-token sequences
+    T = sum(lengths)
+    _, k, v = wl.qkv(T, H, d, dtype, seed=74, device=DEV)
+    cu = wl.cu_seqlens(lengths, device=DEV)
+    decay = torch.tensor(RATES[4], dtype=torch.float32, device=DEV)
+    init = wl.state_init(4, H, d, seed=7, device=DEV) if with_init else None
+    st = la.state_decay(k, v, decay, cu, init_state=init)
+    status_ok()
+    ref = oracle.decay_state(f64(k), f64(v), decay.cpu().double().numpy(), cu.cpu().numpy(),
+                             init=None if init is None else init.cpu().double().numpy())
+    assert_close(st.cpu().double().numpy(), ref, 1e-4, "decay state")
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 48)])
+def test_decode_step_decay(dtype, d):
+    batch, H, steps = 5, 4, 3
+    st = wl.state_init(batch, H, d, seed=d, device=DEV)
+    ref_state = st.cpu().double().numpy()
+    decay = torch.tensor(RATES[4], dtype=torch.float32, device=DEV)
+    q, k, v = wl.decode_inputs(batch, H, d, steps, dtype, seed=9 + d, device=DEV)
+    for t in range(steps):
+        o = la.decode_step_decay(q[t], k[t], v[t], st, decay)
+        ref_o, ref_state = oracle.decay_decode_step(f64(q[t]), f64(k[t]), f64(v[t]), ref_state,
+                                                    decay.cpu().double().numpy())
+        assert_close(f64(o), ref_o, TOL[dtype], f"decay decode o step {t}")
+    status_ok()
+    assert_close(st.cpu().double().numpy(), ref_state, 1e-5, "decay decode state")
+
+
+def test_decay_prefill_then_decode_continuity():
+    """State of the first m tokens from the prefill, then decode steps: the rows of one prefill."""
+    T, m, H, d = 600, 520, 4, 128
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, seed=75, device=DEV)
+    decay = wl.decay_rates(H, device=DEV)
+    full = la.prefill_decay(q, k, v, decay, B=256)
+    _, st = la.prefill_decay(q[:m], k[:m], v[:m], decay, B=256, return_state=True)
+    rows = []
+    for t in range(m, T):
+        rows.append(la.decode_step_decay(q[t:t + 1], k[t:t + 1], v[t:t + 1], st, decay))
+    status_ok()
+    dec = torch.cat(rows)
+    ref = oracle.decay_recurrent(f64(q), f64(k), f64(v), decay.cpu().double().numpy())[m:]
+    assert_close(f64(dec), ref, 1e-2, "decode rows after a prefill")
+    assert_close(f64(full[m:]), ref, 1e-2, "prefill rows")
+
+
+@pytest.mark.parametrize("bad", [1.5, -0.25, float("nan")])
+@pytest.mark.parametrize("dtype,d,H,B", [(torch.float32, 64, 4, 64), (torch.bfloat16, 128, 64, 256)],
+                         ids=["cuda-cores", "tensor-cores"])
+def test_bad_decay_rate_reported_on_device(bad, dtype, d, H, B):
+    T = 300
+    q, k, v = wl.qkv(T, H, d, dtype, seed=76, device=DEV)
+    decay = torch.full((H,), 0.9, dtype=torch.float32, device=DEV)
+    decay[1] = bad
+    o = torch.full_like(q, 7.0)
+    st_out = torch.full((1, H, d, d), 7.0, dtype=torch.float32, device=DEV)
+    la.prefill_decay(q, k, v, decay, B=B, out=o, state_out=st_out)
+    assert la.device_status() == 8                      # LA_ERR_BAD_DECAY
+    assert torch.all(o == 7.0) and torch.all(st_out == 7.0), "a call with a bad rate writes nothing"
+    la.prefill_decay(q, k, v, torch.full((H,), 0.9, dtype=torch.float32, device=DEV), B=B, out=o)
+    status_ok()                                         # the next call with good rates runs
+    assert not torch.any(o == 7.0)
+    q, k, v = q[:, :4].contiguous(), k[:, :4].contiguous(), v[:, :4].contiguous()
+    decay = decay[:4].contiguous()
+    H = 4
+    st = wl.state_init(2, H, d, seed=8, device=DEV)
+    before = st.clone()
+    la.decode_step_decay(q[:2], k[:2], v[:2], st, decay)
+    assert la.device_status() == 8
+    assert torch.equal(st[:, 1], before[:, 1]), "the state of a head with a bad rate is left as it was"
+    assert la.device_status() == 0                      # the status word was cleared
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 1000, 4099, 1 << 20])
+@pytest.mark.parametrize("in_place", [False, True], ids=["out", "in-place"])
+def test_feature_map(dtype, n, in_place):
+    g = torch.Generator(device=DEV).manual_seed(n)
+    x = (torch.randn(n, generator=g, device=DEV) * 4).to(dtype)
+    if n >= 8:
+        x[:6] = torch.tensor([0.0, -0.0, -100.0, 100.0, -1e-30, 1e-30]).to(dtype)
+    ref = oracle.feature_map(f64(x), 0.3)
+    y = la.feature_map(x.clone() if in_place else x, 0.3, out=None)
+    if in_place:
+        xi = x.clone()
+        la.feature_map(xi, 0.3, out=xi)
+        assert torch.equal(xi, y)
+    status_ok()
+    tol = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-6
+    err = np.abs(f64(y) - ref)
+    assert np.all(err <= tol * np.abs(ref) + 1e-38), f"phi: worst relative error {np.max(err / (np.abs(ref) + 1e-38)):.3e}"
+
+
+def test_feature_map_then_prefill_decay():
+    """The pre-pass composes with a prefill: phi on q and k, then the decay prefill."""
+    T, H, d = 333, 2, 64
+    q, k, v = wl.qkv(T, H, d, torch.float32, seed=77, device=DEV)
+    decay = torch.tensor(RATES[2], dtype=torch.float32, device=DEV)
+    o = la.prefill_decay(la.feature_map(q), la.feature_map(k), v, decay, B=64)
+    status_ok()
+    ref = oracle.decay_recurrent(oracle.feature_map(f64(q)), oracle.feature_map(f64(k)), f64(v),
+                                 decay.cpu().double().numpy())
+    assert_close(f64(o), ref, 1e-4, "phi then decay prefill")
+
+
+def test_decay_full_size_sampled_heads():
+    """The bf16 32k workload (T = 32768, H = 64, d = 128, B = 256) with the decay recipe: the
+    heads with the fastest and the slowest decay, in full length, against the oracle."""
+    T, H, d = 32768, 64, 128
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, seed=2, device=DEV)
+    decay = wl.decay_rates(H, device=DEV)
+    o, st = la.prefill_decay(q, k, v, decay, B=256, return_state=True)
+    status_ok()
+    lam = decay.cpu().double().numpy()
+    for h in (0, H - 1):
+        ref_o, ref_st = oracle.decay_recurrent(f64(q[:, h:h + 1]), f64(k[:, h:h + 1]), f64(v[:, h:h + 1]),
+                                               lam[h:h + 1], return_state=True)
+        assert_close(f64(o[:, h:h + 1]), ref_o, 1e-2, f"head {h} (lambda {lam[h]:.4f})")
+        # tensor-core path (64 heads x 2 halves >= 64 work items): the state bound of that path
+        assert_close(st[:, h:h + 1].cpu().double().numpy(), ref_st, 5e-3, f"final state of head {h}")

@@ -143,3 +143,12 @@ def state_init(nseq: int, H: int, d: int, seed: int, device="cpu", scale: float 
     g = _generator(torch.device(device), seed)
     s = torch.randn((nseq, H, d, d), generator=g, dtype=torch.float32, device=device)
     return s.mul_(scale / d)
+
+
+def decay_rates(H: int, device="cpu") -> torch.Tensor:
+    """Per-head decay rates for the decay variant (fp32 [H], deterministic):
+    lambda_h = exp(-2^(-8 (h + 1) / H)), the geometric slopes ALiBi gives its heads,
+    turned into rates in (0, 1): from about 0.40 (h = 0 at H = 64) to 0.996."""
+    h = torch.arange(H, dtype=torch.float64)
+    lam = torch.exp(-torch.pow(2.0, -8.0 * (h + 1) / H))
+    return lam.to(torch.float32).to(device)
