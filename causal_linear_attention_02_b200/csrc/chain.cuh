@@ -81,7 +81,7 @@ constexpr int KC = 128;                    // keys per chunk
 #endif
 constexpr int NQ = LA_CHAIN_NQ;            // Q sub-unit stages
 constexpr int NK_MAX = LA_CHAIN_NK > 2 ? LA_CHAIN_NK : 2;   // K chunk stages, either instance
-constexpr int NV = LA_CHAIN_NV;            // V chunk stages
+constexpr int NV_MAX = 3;                  // V chunk stages, either instance (barrier arrays)
 constexpr int NS = 2;                      // score buffers in TMEM
 constexpr int NTHREADS = 640;
 
@@ -93,20 +93,27 @@ constexpr uint32_t V_BYTES = KC * DV * 2;        // 16 KB
 constexpr uint32_t SB_BYTES = D * DV * 2;        // 16 KB: bf16 KV_b, 128 rows x 64 columns
 
 // Shared-memory layout. The decay instance (a rate per head on the state) also
-// keeps a ring of decay-weighted V chunks, the B operand of its state MMAs, and
-// gives up one K stage for it.
+// keeps a ring of decay-weighted V chunks, the B operand of its state MMAs.
+#ifndef LA_CHAIN_NVW
+#define LA_CHAIN_NVW 2
+#endif
+#ifndef LA_CHAIN_DECAY_NV
+#define LA_CHAIN_DECAY_NV 3
+#endif
 template <bool kDecay>
 struct Smem {
-    static constexpr int NK = kDecay ? 2 : LA_CHAIN_NK;    // K chunk stages
+    static constexpr int NK = kDecay && LA_CHAIN_NVW > 1 ? 2 : LA_CHAIN_NK;   // K chunk stages
+    static constexpr int NV = kDecay ? LA_CHAIN_DECAY_NV : LA_CHAIN_NV;      // V chunk stages
+    static constexpr int NVW = LA_CHAIN_NVW;                               // weighted V stages (decay only)
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + NQ * Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + NK * K_BYTES;
     static constexpr uint32_t OFF_VW = OFF_V + NV * V_BYTES;               // weighted V (decay only)
-    static constexpr uint32_t OFF_SB = OFF_VW + (kDecay ? NV * V_BYTES : 0);
+    static constexpr uint32_t OFF_SB = OFF_VW + (kDecay ? NVW * V_BYTES : 0);
     static constexpr uint32_t OFF_BAR = OFF_SB + SB_BYTES;
     static constexpr uint32_t BYTES = OFF_BAR + 512 + 1024;   // + barriers + 1 KB alignment slack
     static_assert(BYTES <= 232448, "shared memory per CTA");
-    static_assert(NK <= NK_MAX, "barrier arrays");
+    static_assert(NK <= NK_MAX && NV <= NV_MAX && NVW <= NV_MAX, "barrier arrays");
 };
 
 // TMEM columns (512 x 32-bit, 128 lanes): three O slots, the state, NS score buffers.
@@ -121,10 +128,9 @@ constexpr uint32_t IDESC_C = idesc_bf16(UM, DV, false, true);    // Q (K-major) 
 struct Bars {
     uint64_t q_full[NQ], q_empty[NQ];
     uint64_t k_full[NK_MAX], k_empty[NK_MAX]; // k_empty: two arrivals, the chunk's scores and its state MMA
-    uint64_t v_full[NV], v_empty[NV];     // v_empty: two arrivals, the chunk's PVs and its state MMA (decay
+    uint64_t v_full[NV_MAX], v_empty[NV_MAX]; // v_empty: two arrivals, the chunk's PVs and its state MMA (decay
                                           // instance: the weighting warp, which reads it for the state MMA)
-    uint64_t vw_full[NV], vw_empty[NV];   // decay instance: weighted V chunk written / read by its state MMA
-    uint64_t c_full[3], c_scaled[3];      // decay instance: inter-block MMA done / its rows scaled, per O slot
+    uint64_t vw_full[NV_MAX], vw_empty[NV_MAX]; // decay instance: weighted V chunk written / read by its state MMA
     uint64_t s_full[NS], p_full[NS], s_free[NS];
     uint64_t o_full[3], o_empty[3];
     uint64_t kv_ready;        // issuer -> state group: KV accumulator holds the next block's prefix
@@ -313,20 +319,21 @@ struct Cursor {
 // S_t = lambda S_{t-1} + k_t^T v_t. For a block of n rows, row r (in the block)
 // and key c (in the block):
 //   P[r][c]   = lambda^(r-c) S[r][c]                 (P groups, c <= r)
-//   O_r      += lambda^(r+1) q_r bf16(KV_b)          (copy-out group scales the
-//               rows of the inter-block accumulator in TMEM before the first PV)
+//   O_r       = (lambda^(r+1) q_r) bf16(KV_b) + ...  (the P groups write the
+//               scaled Q row into the score buffer's columns that P leaves
+//               free; the inter-block MMA reads its A operand from there)
 //   KV_{b+1}  = lambda^n KV_b + sum_c K_c^T (lambda^(n-1-c) v_c)
 //               (copy-out group rescales the accumulator when it reads KV_b;
 //               warp 2 writes the weighted V chunk, the state MMA's B operand)
-// The weighted V is rounded to bf16 once, so the state's increments carry one
-// extra bf16 rounding (relative 2^-9 per term). Rates are checked before the
-// launch (a bad rate leaves the launch with no work).
+// The weighted V and the scaled Q rows are packed bf16 products (weight and
+// product each rounded to bf16: relative 2^-8 per term). Rates are checked
+// before the launch (a bad rate leaves the launch with no work).
 template <bool kStateOut, bool kDecay>
 __global__ void __launch_bounds__(NTHREADS, 1)
 prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
     using SM = Smem<kDecay>;
-    constexpr int NK = SM::NK;
+    constexpr int NK = SM::NK, NV = SM::NV;
     constexpr uint32_t OFF_Q = SM::OFF_Q, OFF_K = SM::OFF_K, OFF_V = SM::OFF_V, OFF_SB = SM::OFF_SB,
                        OFF_BAR = SM::OFF_BAR;
     extern __shared__ uint8_t smem_raw[];
@@ -352,8 +359,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->drain_b, 1);
         if constexpr (kDecay) {
-            for (int i = 0; i < NV; ++i) { mbar_init(&bars->vw_full[i], 32); mbar_init(&bars->vw_empty[i], 1); }
-            for (int i = 0; i < 3; ++i) { mbar_init(&bars->c_full[i], 1); mbar_init(&bars->c_scaled[i], 128); }
+            for (int i = 0; i < SM::NVW; ++i) { mbar_init(&bars->vw_full[i], 32); mbar_init(&bars->vw_empty[i], 1); }
         }
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -503,8 +509,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         dc.next_item(p);
                     } else {
                         const uint32_t kc = dc.kc0 + dc.j;
-                        bool ready = mbar_test_wait(kDecay ? &bars->vw_full[kc % NV] : &bars->v_full[kc % NV],
-                                                    (kc / NV) & 1);
+                        bool ready = kDecay ? mbar_test_wait(&bars->vw_full[kc % SM::NVW], (kc / SM::NVW) & 1)
+                                            : mbar_test_wait(&bars->v_full[kc % NV], (kc / NV) & 1);
                         if (ready && dc.add_state && dc.j == 0 && kvr_blk != dc.n) {
                             if (mbar_test_wait(&bars->kv_read[dc.n & 3], (dc.n >> 2) & 1)) kvr_blk = dc.n;
                             else ready = false;
@@ -512,7 +518,9 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         if (ready) {
                             if (dc.add_state || kStateOut) {
                                 tc_fence_after();
-                                const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4), b = dvs + (((kc % NV) * V_BYTES) >> 4);
+                                const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4),
+                                               b = kDecay ? dvs + (((kc % SM::NVW) * V_BYTES) >> 4)
+                                                          : dv + (((kc % NV) * V_BYTES) >> 4);
                                 // a ragged last chunk: its full 16-key steps only (the copy-out
                                 // group adds the rest); the rows past the sequence end belong to
                                 // the next sequence
@@ -528,7 +536,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                                 }
                             }
                             tc_commit(&bars->k_empty[kc % NK]);          // the state MMA's shares
-                            tc_commit(kDecay ? &bars->vw_empty[kc % NV] : &bars->v_empty[kc % NV]);
+                            tc_commit(kDecay ? &bars->vw_empty[kc % SM::NVW] : &bars->v_empty[kc % NV]);
                             dc.next_item(p);
                             prog = true;
                         }
@@ -559,7 +567,22 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const uint32_t sbuf = c.i % NS, slot = c.oslot(c.r);
                 const uint32_t kc = c.kc0 + c.j, qc = c.q0 + c.r;
                 const uint32_t d_o = tmem + TM_O + slot * 64;
-                if (c.first_of_sub()) {
+                if (kDecay && c.first_of_sub()) {
+                    // O_r = (Lambda Q_r) . bf16(KV_b) from TMEM: the P groups wrote lambda^(r+1) q_r
+                    // (bf16) into the score buffer's columns that P leaves free
+                    if (!wait_bar(&bars->o_empty[slot], (c.ouse(c.r) & 1) ^ 1, ab)) { ok = false; break; }
+                    if (c.r == 0 && !wait_bar(&bars->sb_full, c.n & 1, ab)) { ok = false; break; }
+                    if (!wait_bar(&bars->p_full[sbuf], (c.i / NS) & 1, ab)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_q = tmem + TM_S + sbuf * KC + 32;
+#pragma unroll
+                    for (int s = 0; s < D / 16; ++s)
+                        mma_ts(d_o, a_q + (s < 4 ? s * 8 : 64 + (s - 4) * 8), dsb + ((s * 2048) >> 4), IDESC_PV,
+                               s > 0);
+                    if (c.r == c.Rb - 1) tc_commit(&bars->sb_empty);
+                    tc_commit(&bars->q_empty[qc % NQ]);                  // the inter-block share (P groups read Q)
+                    LA_CTRACE(c.n, c.r == 0 ? TR_C0 : TR_CL);
+                } else if (c.first_of_sub()) {
                     // O_r = Q_r . bf16(KV_b)
                     if (!wait_bar(&bars->o_empty[slot], (c.ouse(c.r) & 1) ^ 1, ab)) { ok = false; break; }
                     if (c.r == 0 && !wait_bar(&bars->sb_full, c.n & 1, ab)) { ok = false; break; }
@@ -573,11 +596,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (c.r == c.Rb - 1) tc_commit(&bars->sb_empty);
                     tc_commit(&bars->q_empty[qc % NQ]);                  // the inter-block MMA's share
                     LA_CTRACE(c.n, c.r == 0 ? TR_C0 : TR_CL);
-                    if constexpr (kDecay) {
-                        // lambda^(r+1) on its rows before the PVs add onto it
-                        tc_commit(&bars->c_full[slot]);
-                        if (!wait_bar(&bars->c_scaled[slot], c.ouse(c.r) & 1, ab)) { ok = false; break; }
-                    }
                 }
                 // O_r += P V_j; P of keys 0-63 in columns 0-31, of keys 64-127 in 64-95
                 if (!wait_bar(&bars->p_full[sbuf], (c.i / NS) & 1, ab)) { ok = false; break; }
@@ -614,32 +632,32 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             while (ok && c.valid) {
                 const float l2 = log2f(__ldg(p.decay + c.h));
                 for (int j = 0; j < c.Rb; ++j) {
-                    const uint32_t kc = c.kc0 + j, st = kc % NV;
+                    const uint32_t kc = c.kc0 + j, st = kc % NV, sw = kc % SM::NVW;
                     if (!warp_all(wait_bar(&bars->v_full[st], (kc / NV) & 1, ab)) ||
-                        !warp_all(wait_bar(&bars->vw_empty[st], ((kc / NV) & 1) ^ 1, ab))) {
+                        !warp_all(wait_bar(&bars->vw_empty[sw], ((kc / SM::NVW) & 1) ^ 1, ab))) {
                         ok = false;
                         break;
                     }
                     if (c.add_state || kStateOut) {
                         const uint8_t* src = smem + OFF_V + st * V_BYTES;
-                        uint8_t* dst = smem + SM::OFF_VW + st * V_BYTES;
+                        uint8_t* dst = smem + SM::OFF_VW + sw * V_BYTES;
+                        // packed bf16 products: the weight is rounded to bf16 and so is each product
 #pragma unroll 4
                         for (int it = 0; it < KC / 4; ++it) {
                             const int line = 4 * it + (lane >> 3);                 // key KC*j + line
                             const int t = KC * j + line;
-                            const float w = t < c.rows ? decay_pow(l2, c.rows - 1 - t) : 0.f;
+                            const __nv_bfloat162 w2 =
+                                __float2bfloat162_rn(t < c.rows ? decay_pow(l2, c.rows - 1 - t) : 0.f);
                             const uint32_t off = line * 128 + (lane & 7) * 16;
                             uint4 u = *reinterpret_cast<const uint4*>(src + off);
-                            uint32_t* e = reinterpret_cast<uint32_t*>(&u);
+                            __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-                            for (int x = 0; x < 4; ++x)
-                                e[x] = pack_bf16x2(__uint_as_float(e[x] << 16) * w,
-                                                   __uint_as_float(e[x] & 0xffff0000u) * w);
+                            for (int x = 0; x < 4; ++x) e[x] = __hmul2(e[x], w2);
                             *reinterpret_cast<uint4*>(dst + off) = u;
                         }
                         fence_proxy_async_smem();
                     }
-                    mbar_arrive(&bars->vw_full[st]);
+                    mbar_arrive(&bars->vw_full[sw]);
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->v_empty[st]);      // done reading the V chunk
                 }
@@ -695,6 +713,26 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
             }
             tmem_st_x32(ts, pk);             // P of these 64 keys over the first 32 of their columns
+            if constexpr (kDecay) {
+                if (c.first_of_sub()) {
+                    // lambda^(r+1) q_r over the other 32 columns: head dims 64 hk .. 64 hk + 63 of
+                    // query row m (the A operand of the inter-block MMA, read from TMEM)
+                    const uint32_t qc = c.q0 + c.r;
+                    if (!warp_all(wait_bar(&bars->q_full[qc % NQ], (qc / NQ) & 1, ab))) { ok = false; break; }
+                    const uint8_t* qrow = smem + OFF_Q + (qc % NQ) * Q_BYTES + hk * QH_BYTES + m * 128;
+                    const __nv_bfloat162 w2 = __float2bfloat162_rn(decay_pow(l2, UM * c.r + m + 1));
+                    uint32_t qk[32];
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        uint4 u = *reinterpret_cast<const uint4*>(qrow + ((g ^ (m & 7)) << 4));
+                        __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) e[x] = __hmul2(e[x], w2);
+                        qk[4 * g] = u.x; qk[4 * g + 1] = u.y; qk[4 * g + 2] = u.z; qk[4 * g + 3] = u.w;
+                    }
+                    tmem_st_x32(ts + 32, qk);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_full[sbuf]);
@@ -801,28 +839,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             fence_proxy_async_smem();
             if (!(c.w == p.suppress_item && c.b == 1)) mbar_arrive(&bars->sb_full);
             if (wt == 0) LA_CTRACE(c.n, TR_SB);
-            if constexpr (kDecay) {
-                // lambda^(r+1) on row r of each sub-unit's inter-block accumulator (r in the block)
-                for (int r = 0; r < c.Rb; ++r) {
-                    const uint32_t slot = c.oslot(r);
-                    if (!warp_all(wait_bar(&bars->c_full[slot], c.ouse(r) & 1, ab))) { ok = false; break; }
-                    tc_fence_after();
-                    const float wr = decay_pow(l2, UM * r + m + 1);
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t a[32];
-                        tmem_ld_x32(tmem + lane_base + TM_O + slot * 64 + 32 * hh, a);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__uint_as_float(a[q]) * wr);
-                        tmem_st_x32(tmem + lane_base + TM_O + slot * 64 + 32 * hh, a);
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&bars->c_scaled[slot]);
-                }
-                if (!ok) break;
-            }
             if (kStateOut && !c.add_state) {
                 // the work item's last block: its state MMAs complete the final state
                 if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
