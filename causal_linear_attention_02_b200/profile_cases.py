@@ -2,6 +2,7 @@
 
     python -m causal_linear_attention_02_b200.profile_cases prefill [--tokens T] [--calls N]
     python -m causal_linear_attention_02_b200.profile_cases decode [--batch B] [--calls N]
+    python -m causal_linear_attention_02_b200.profile_cases prefill_decay [--tokens T] [--calls N]
 
 Each case builds seeded synthetic inputs on cuda:0 (the generators of the
 `workloads` module), then makes N calls of one entry point through the C ABI
@@ -12,6 +13,8 @@ prefill: bf16, 64 heads, d = 128, B = 256, one sequence of T tokens
          (default 32768: Q, K, V, O of 0.5 GB each, larger than the L2).
 decode:  bf16 inputs, 64 heads, d = 128, fp32 states of `batch` sequences
          (default 256: 1 GiB of state), states drawn iid instead of from a prefill.
+prefill_decay: as prefill, through la_prefill_decay with the per-head rates
+         lambda_h = exp(-2^(-8 (h+1) / H)) of `workloads.decay_rates`.
 """
 from __future__ import annotations
 
@@ -34,23 +37,29 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def prefill_case(tokens: int, calls: int) -> None:
+def prefill_case(tokens: int, calls: int, decay: bool = False) -> None:
     dev = torch.device("cuda", 0)
     H, d, B = 64, 128, 256
     q, k, v = wl.qkv(tokens, H, d, torch.bfloat16, 2, device=dev)
     o = torch.empty_like(q)
-    ws_bytes = la.la_prefill_workspace_size(tokens, 1, H, d, B, la.LA_BF16)
+    rates = wl.decay_rates(H, device=dev) if decay else None
+    size = la.la_prefill_decay_workspace_size if decay else la.la_prefill_workspace_size
+    ws_bytes = size(tokens, 1, H, d, B, la.LA_BF16)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     sh = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     for _ in range(calls):
-        s = la.la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), None, 1, tokens, H, d, B, la.LA_BF16, None,
-                          _ptr(ws), ws_bytes, sh)
+        if decay:
+            s = la.la_prefill_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(o), None, 1, tokens, H, d, B, la.LA_BF16, None,
+                                    _ptr(rates), None, _ptr(ws), ws_bytes, sh)
+        else:
+            s = la.la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(o), None, 1, tokens, H, d, B, la.LA_BF16, None,
+                              _ptr(ws), ws_bytes, sh)
         if s != 0:
-            raise la.LightningError(f"la_prefill: {la.STATUS.get(s, s)}", s)
+            raise la.LightningError(f"prefill: {la.STATUS.get(s, s)}", s)
     torch.cuda.synchronize(dev)
     if la.device_status() != 0:
         raise la.LightningError("device status after prefill")
-    print(f"prefill T={tokens} H={H} d={d} B={B}: {calls} calls ok")
+    print(f"prefill{' with decay' if decay else ''} T={tokens} H={H} d={d} B={B}: {calls} calls ok")
 
 
 def decode_case(batch: int, calls: int) -> None:
@@ -73,14 +82,14 @@ def decode_case(batch: int, calls: int) -> None:
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill", "decode"])
+    ap.add_argument("case", choices=["prefill", "decode", "prefill_decay"])
     ap.add_argument("--tokens", type=int, default=32768)
     ap.add_argument("--batch", type=int, default=256)
     ap.add_argument("--calls", type=int, default=2)
     a = ap.parse_args()
     la.load_library()
-    if a.case == "prefill":
-        prefill_case(a.tokens, a.calls)
+    if a.case in ("prefill", "prefill_decay"):
+        prefill_case(a.tokens, a.calls, decay=a.case == "prefill_decay")
     else:
         decode_case(a.batch, a.calls)
 
