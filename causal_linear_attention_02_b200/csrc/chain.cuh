@@ -310,6 +310,46 @@ struct Cursor {
     __device__ __forceinline__ uint32_t ouse(int rr) const { return rr == Rb - 1 ? (n >> 1) : o0; }
 };
 
+// Decay instance: the weighted copy lambda^(rows-1-c) v_c (c the key in the block, zero past the
+// block's end) of every V chunk of the cursor's block, the B operand of its state MMAs, written by
+// the 128 threads of the epilogue group; then their releases of the V chunk (the state MMA's share
+// of v_empty). A chunk whose state MMA does not run passes through the ring unwritten. A line of
+// the swizzled chunk is one key's 64 columns, so lines are scaled whole; 8 threads per line, each
+// warp 4 lines (512 contiguous bytes) per step. Packed bf16 products: the weight is rounded to bf16
+// and so is each product. Returns false when a wait gave up.
+template <bool kStateOut, class SM>
+__device__ __forceinline__ bool weight_block(const Cursor& c, const Params& p, Bars* bars, uint8_t* smem, int quad,
+                                             int lane, const Abort& ab) {
+    if (!c.valid) return true;
+    const float l2 = log2f(__ldg(p.decay + c.h));
+    for (int j = 0; j < c.Rb; ++j) {
+        const uint32_t kc = c.kc0 + j, st = kc % SM::NV, sw = kc % SM::NVW;
+        if (!warp_all(wait_bar(&bars->v_full[st], (kc / SM::NV) & 1, ab)) ||
+            !warp_all(wait_bar(&bars->vw_empty[sw], ((kc / SM::NVW) & 1) ^ 1, ab)))
+            return false;
+        if (c.add_state || kStateOut) {
+            const uint8_t* src = smem + SM::OFF_V + st * V_BYTES;
+            uint8_t* dst = smem + SM::OFF_VW + sw * V_BYTES;
+#pragma unroll 2
+            for (int it = 0; it < KC / 16; ++it) {
+                const int line = 16 * it + 4 * quad + (lane >> 3);          // key KC*j + line
+                const int t = KC * j + line;
+                const __nv_bfloat162 w2 = __float2bfloat162_rn(t < c.rows ? decay_pow(l2, c.rows - 1 - t) : 0.f);
+                const uint32_t off = line * 128 + (lane & 7) * 16;
+                uint4 u = *reinterpret_cast<const uint4*>(src + off);
+                __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) e[x] = __hmul2(e[x], w2);
+                *reinterpret_cast<uint4*>(dst + off) = u;
+            }
+            fence_proxy_async_smem();
+        }
+        mbar_arrive(&bars->vw_full[sw]);
+        mbar_arrive(&bars->v_empty[st]);                 // done reading the V chunk
+    }
+    return true;
+}
+
 // kStateOut: also write each sequence's final state S0 + sum_t k_t^T v_t to
 // p.state_out (the last block runs its state MMAs too; the copy-out group reads
 // the accumulator after them). A separate instance, so the plain prefill's code
@@ -324,7 +364,8 @@ struct Cursor {
 //               free; the inter-block MMA reads its A operand from there)
 //   KV_{b+1}  = lambda^n KV_b + sum_c K_c^T (lambda^(n-1-c) v_c)
 //               (copy-out group rescales the accumulator when it reads KV_b;
-//               warp 2 writes the weighted V chunk, the state MMA's B operand)
+//               the epilogue group writes the weighted V chunks, the state
+//               MMA's B operand, one block ahead)
 // The weighted V and the scaled Q rows are packed bf16 products (weight and
 // product each rounded to bf16: relative 2^-8 per term). Rates are checked
 // before the launch (a bad rate leaves the launch with no work).
@@ -345,7 +386,9 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     if (threadIdx.x == 0) {
         for (int i = 0; i < NQ; ++i) { mbar_init(&bars->q_full[i], 1); mbar_init(&bars->q_empty[i], 2); }
         for (int i = 0; i < NK; ++i) { mbar_init(&bars->k_full[i], 1); mbar_init(&bars->k_empty[i], 2); }
-        for (int i = 0; i < NV; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], 2); }
+        // v_empty: the PVs' commit, then the state MMA's commit (the epilogue group's 128 threads,
+        // which read V for the weighted copy, in the decay instance)
+        for (int i = 0; i < NV; ++i) { mbar_init(&bars->v_full[i], 1); mbar_init(&bars->v_empty[i], kDecay ? 129 : 2); }
         for (int i = 0; i < NS; ++i) {
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], 256);
@@ -359,7 +402,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->drain_b, 1);
         if constexpr (kDecay) {
-            for (int i = 0; i < SM::NVW; ++i) { mbar_init(&bars->vw_full[i], 32); mbar_init(&bars->vw_empty[i], 1); }
+            for (int i = 0; i < SM::NVW; ++i) { mbar_init(&bars->vw_full[i], 128); mbar_init(&bars->vw_empty[i], 1); }
         }
         bars->abort_flag = 0;
         fence_mbar_init();
@@ -617,53 +660,6 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&bars->drain_b, 0) && globaltimer_ns() - t0 < 1000000000ull) {}
         }
-    } else if (warp == 2) {
-        if constexpr (kDecay) {
-            // ============================================================ weighted V (decay instance)
-            // Every V chunk in ring order: the copy lambda^(rows-1-c) v_c (c the key in the block,
-            // zero past the block's end) that the state MMA reads, then the chunk's second V
-            // release, which in this instance is this warp's (the state MMA reads the copy).
-            // A chunk whose state MMA does not run passes through the ring unwritten. A line of
-            // the swizzled chunk is one key's 64 columns, so lines are scaled whole; the 32
-            // lanes take 512 contiguous bytes (4 lines) per step.
-            bool ok = true;
-            Cursor c;
-            c.init(p);
-            while (ok && c.valid) {
-                const float l2 = log2f(__ldg(p.decay + c.h));
-                for (int j = 0; j < c.Rb; ++j) {
-                    const uint32_t kc = c.kc0 + j, st = kc % NV, sw = kc % SM::NVW;
-                    if (!warp_all(wait_bar(&bars->v_full[st], (kc / NV) & 1, ab)) ||
-                        !warp_all(wait_bar(&bars->vw_empty[sw], ((kc / SM::NVW) & 1) ^ 1, ab))) {
-                        ok = false;
-                        break;
-                    }
-                    if (c.add_state || kStateOut) {
-                        const uint8_t* src = smem + OFF_V + st * V_BYTES;
-                        uint8_t* dst = smem + SM::OFF_VW + sw * V_BYTES;
-                        // packed bf16 products: the weight is rounded to bf16 and so is each product
-#pragma unroll 4
-                        for (int it = 0; it < KC / 4; ++it) {
-                            const int line = 4 * it + (lane >> 3);                 // key KC*j + line
-                            const int t = KC * j + line;
-                            const __nv_bfloat162 w2 =
-                                __float2bfloat162_rn(t < c.rows ? decay_pow(l2, c.rows - 1 - t) : 0.f);
-                            const uint32_t off = line * 128 + (lane & 7) * 16;
-                            uint4 u = *reinterpret_cast<const uint4*>(src + off);
-                            __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-                            for (int x = 0; x < 4; ++x) e[x] = __hmul2(e[x], w2);
-                            *reinterpret_cast<uint4*>(dst + off) = u;
-                        }
-                        fence_proxy_async_smem();
-                    }
-                    mbar_arrive(&bars->vw_full[sw]);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->v_empty[st]);      // done reading the V chunk
-                }
-                c.next_block(p);
-            }
-        }
     } else if (warp >= 4 && warp < 12) {
         // ================================================================ scores -> P
         const int hk = warp >= 8 ? 1 : 0;                // keys 0-63 or 64-127 of the chunk
@@ -879,6 +875,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         }
     } else if (warp >= 16) {
         // ================================================================ O epilogue
+        // (decay instance: also the weighted V copy of every chunk, one block ahead)
         const int quad = warp & 3;
         const int m = quad * 32 + lane;                  // TMEM lane: query row of the sub-unit
         const int wt = threadIdx.x - 512;                // 0..127
@@ -886,7 +883,19 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         bool ok = true;
         Cursor c;
         c.init(p);
+        Cursor cw;                                       // decay: the block whose V chunks are weighted next
+        if constexpr (kDecay) {
+            cw.init(p);
+            ok = weight_block<kStateOut, SM>(cw, p, bars, smem, quad, lane, ab);
+            if (cw.valid) cw.next_block(p);
+        }
         while (ok && c.valid) {
+            if constexpr (kDecay) {
+                if (cw.valid) {
+                    if (!weight_block<kStateOut, SM>(cw, p, bars, smem, quad, lane, ab)) break;
+                    cw.next_block(p);
+                }
+            }
             // each sub-unit in the order the issuer finishes them
             for (int r = 0; ok && r < c.Rb; ++r) {
                 const uint32_t slot = c.oslot(r);
