@@ -9,6 +9,7 @@ current stream), runs the whole problem on the GPU, and checks sampled
   bf16 prefill T = 32768, H = 64, d = 128, B = 256          heads 0, 21, 42, 63
   bf16 prefill T = 1048576, H = 64, d = 128, B = 256        heads 0, 63
   bf16 varlen, 16 sequences U[1024, 65536], H = 64, B = 256  heads 5, 58, every sequence
+  the same varlen workload with a decay rate per head          heads 0, 63, every sequence, final states
   decode, 256 sequences x 64 heads, states from a 4096-token prefill, 1000 steps,
                                                              8 (sequence, head) pairs, every step
 
@@ -99,6 +100,42 @@ def test_bf16_varlen_sampled_heads():
     cu = wl.cu_seqlens(w.seq_lens, device=DEV)
     q, k, v, o = _prefill_like_bench(w, cu)
     _check_heads(q, k, v, o, [5, 58], cu_host=np.asarray(cu.cpu().numpy(), dtype=np.int32), what=w.name)
+
+
+def test_bf16_varlen_decay_sampled_heads():
+    """The varlen workload through la_prefill_decay with the decay recipe's per-head rates, and the
+    final state of every sequence: heads 0 and 63 (fastest and slowest decay) against the oracle's
+    decay recurrence. O within 1e-2, states within the tensor-core path's 5e-3 (the state MMAs read
+    bf16-rounded weighted V)."""
+    w = wl.BF16_VARLEN
+    T, H, d, B = w.total_tokens, w.heads, w.d, w.B
+    nseq = len(w.seq_lens)
+    cu = wl.cu_seqlens(w.seq_lens, device=DEV)
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, w.seed, device=DEV)
+    decay = wl.decay_rates(H, device=DEV)
+    o = torch.full_like(q, float("nan"))
+    st = torch.full((nseq, H, d, d), float("nan"), dtype=torch.float32, device=DEV)
+    ws_bytes = la.la_prefill_decay_workspace_size(T, nseq, H, d, B, la.LA_BF16)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=DEV)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
+    s = la.la_prefill_decay(_p(q), _p(k), _p(v), _p(o), _p(cu), nseq, T, H, d, B, la.LA_BF16, None, _p(decay),
+                            _p(st), _p(ws), ws_bytes, stream)
+    assert s == 0, la.STATUS.get(s, s)
+    torch.cuda.synchronize(DEV)
+    assert la.device_status() == 0
+    del ws
+    heads = [0, 63]
+    cu_host = np.asarray(cu.cpu().numpy(), dtype=np.int32)
+    ref_o, ref_st = oracle.decay_recurrent(*(_heads_f64(x, heads) for x in (q, k, v)),
+                                           decay.cpu().double().numpy()[heads], cu_seqlens=cu_host,
+                                           return_state=True)
+    out = _heads_f64(o, heads)
+    assert np.isfinite(out).all()
+    r = _rel(out, ref_o)
+    assert r <= TOL, f"decay varlen O: {r:.3e}"
+    got_st = st[:, heads].cpu().double().numpy()
+    r = _rel(got_st, ref_st)
+    assert r <= 5e-3, f"decay varlen final states: {r:.3e}"
 
 
 def test_decode_workload_sampled_pairs():
