@@ -128,8 +128,9 @@ constexpr uint32_t IDESC_C = idesc_bf16(UM, DV, false, true);    // Q (K-major) 
 struct Bars {
     uint64_t q_full[NQ], q_empty[NQ];
     uint64_t k_full[NK_MAX], k_empty[NK_MAX]; // k_empty: two arrivals, the chunk's scores and its state MMA
-    uint64_t v_full[NV_MAX], v_empty[NV_MAX]; // v_empty: two arrivals, the chunk's PVs and its state MMA (decay
-                                          // instance: the weighting warp, which reads it for the state MMA)
+    uint64_t v_full[NV_MAX], v_empty[NV_MAX]; // v_empty: the chunk's PVs and its state MMA (decay instance:
+                                          // 1 + 128 arrivals, the PVs and the epilogue group that reads it
+                                          // for the weighted copy)
     uint64_t vw_full[NV_MAX], vw_empty[NV_MAX]; // decay instance: weighted V chunk written / read by its state MMA
     uint64_t s_full[NS], p_full[NS], s_free[NS];
     uint64_t o_full[3], o_empty[3];
