@@ -555,7 +555,10 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         const uint32_t kc = dc.kc0 + dc.j;
                         bool ready = kDecay ? mbar_test_wait(&bars->vw_full[kc % SM::NVW], (kc / SM::NVW) & 1)
                                             : mbar_test_wait(&bars->v_full[kc % NV], (kc / NV) & 1);
-                        if (ready && dc.add_state && dc.j == 0 && kvr_blk != dc.n) {
+                        // the state MMAs of a block wait for the copy-out group to have read the
+                        // prefix (and, with decay, rescaled it) whenever they run: in the
+                        // state-output instance also on a sequence's last block
+                        if (ready && (dc.add_state || kStateOut) && dc.j == 0 && kvr_blk != dc.n) {
                             if (mbar_test_wait(&bars->kv_read[dc.n & 3], (dc.n >> 2) & 1)) kvr_blk = dc.n;
                             else ready = false;
                         }

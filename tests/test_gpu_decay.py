@@ -302,3 +302,52 @@ def test_decay_full_size_sampled_heads():
         assert_close(f64(o[:, h:h + 1]), ref_o, 1e-2, f"head {h} (lambda {lam[h]:.4f})")
         # tensor-core path (64 heads x 2 halves >= 64 work items): the state bound of that path
         assert_close(st[:, h:h + 1].cpu().double().numpy(), ref_st, 5e-3, f"final state of head {h}")
+
+
+def test_decay_withheld_prefix_ends_in_timeout_not_hang():
+    """The decay instance of the on-chip-state kernel under the same fault hook as the plain one
+    (work item 3 never hands over its second block's prefix): every bounded wait of the instance,
+    the weighted-V ring's included, gives up, the launch ends with LA_ERR_TIMEOUT and the next
+    call is right."""
+    import time
+    T, H, B = 4096, 4, 256
+    q, k, v = wl.qkv(T, H, 128, torch.bfloat16, seed=5152, device=DEV)
+    decay = torch.tensor(RATES[4], dtype=torch.float32, device=DEV)
+    assert la.la_debug_set_fault(3, 200_000_000) == 0
+    assert la.la_debug_set_path(1) == 0
+    try:
+        t0 = time.time()
+        la.prefill_decay(q, k, v, decay, B=B)
+        st = la.device_status()
+        elapsed = time.time() - t0
+    finally:
+        la.la_debug_set_fault(-1, 0)
+    try:
+        assert st == 6, f"expected LA_ERR_TIMEOUT, got {la.STATUS.get(st, st)}"
+        assert elapsed < 30, f"timed-out launch took {elapsed:.1f}s"
+        o = la.prefill_decay(q, k, v, decay, B=B)
+        status_ok()
+    finally:
+        la.la_debug_set_path(0)
+    ref = oracle.decay_recurrent(f64(q), f64(k), f64(v), decay.cpu().double().numpy())
+    assert_close(f64(o), ref, 1e-2, "run after a timeout")
+
+
+@pytest.mark.parametrize("B", [128, 256])
+def test_prefill_decay_onchip_state_repeated(B):
+    """Many blocks per work item, the final state on: repeated calls must all match the oracle.
+    Guards the hand-off between the copy-out group's read (and decay rescale) of the last block's
+    prefix and that block's state MMAs, which once raced in about one call in fifteen."""
+    lengths, H = [129, 255, 2048], 12
+    T = sum(lengths)
+    q, k, v = wl.qkv(T, H, 128, torch.bfloat16, seed=T + H, device=DEV)
+    cu = wl.cu_seqlens(lengths, device=DEV)
+    decay = wl.decay_rates(H, device=DEV)
+    init = wl.state_init(len(lengths), H, 128, seed=11, device=DEV)
+    ref_o, ref_st = oracle.decay_recurrent(f64(q), f64(k), f64(v), decay.cpu().double().numpy(), cu.cpu().numpy(),
+                                           init=init.cpu().double().numpy(), return_state=True)
+    for rep in range(12):
+        o, st = la.prefill_decay(q, k, v, decay, cu, B=B, init_state=init, return_state=True)
+        status_ok()
+        assert_close(f64(o), ref_o, 1e-2, f"O, call {rep}")
+        assert_close(st.cpu().double().numpy(), ref_st, 5e-3, f"final state, call {rep}")

@@ -505,3 +505,21 @@ def test_prefill_with_state(lengths, H, B, dtype, with_init):
         status_ok()
         assert_close(st2.cpu().double().numpy(), ref_s, 1e-5, "final state, in place")
         assert torch.equal(o2, o)
+
+
+@pytest.mark.parametrize("B", [128, 256])
+def test_prefill_with_state_repeated(B):
+    """The state-output instance of the on-chip-state kernel over many blocks, repeated: every call
+    matches the oracle (the last block's state MMAs wait for the prefix to have been read)."""
+    lengths, H = [129, 255, 2048], 12
+    T = sum(lengths)
+    q, k, v = inputs(T, H, 128, torch.bfloat16, seed=T + H)
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, 128, seed=11, device=DEV)
+    ref_o, ref_s = oracle.recurrent(f64(q), f64(k), f64(v), cu.cpu().numpy(), init=init.cpu().double().numpy(),
+                                    return_state=True)
+    for rep in range(12):
+        o, st = la.prefill_with_state(q, k, v, cu, B=B, init_state=init)
+        status_ok()
+        assert_close(f64(o), ref_o, 1e-2, f"O, call {rep}")
+        assert_close(st.cpu().double().numpy(), ref_s, 1e-5, f"final state, call {rep}")
