@@ -27,10 +27,11 @@ __all__ = [
     "la_prefill_backward_workspace_size", "la_prefill_backward",
     "la_prefill_with_state_workspace_size", "la_prefill_with_state",
     "la_decode_step", "la_prefill_decay_workspace_size", "la_prefill_decay", "la_state_decay_workspace_size",
-    "la_state_decay", "la_decode_step_decay", "la_feature_map", "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
+    "la_state_decay", "la_decode_step_decay", "la_feature_map", "la_state_exclusive_prefix_decay",
+    "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
     "la_launch_count",
     "prefill", "prefill_with_state", "prefill_backward", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status",
-    "prefill_decay", "state_decay", "decode_step_decay", "feature_map",
+    "prefill_decay", "state_decay", "decode_step_decay", "feature_map", "state_exclusive_prefix_decay",
     "uses_tensor_cores",
 ]
 
@@ -104,6 +105,8 @@ def load_library():
         lib.la_state_decay.restype = i32
         lib.la_decode_step_decay.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp]
         lib.la_decode_step_decay.restype = i32
+        lib.la_state_exclusive_prefix_decay.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+        lib.la_state_exclusive_prefix_decay.restype = i32
         lib.la_feature_map.argtypes = [vp, vp, i64, i32, ctypes.c_float, vp]
         lib.la_feature_map.restype = i32
         lib.la_get_device_status.argtypes = [vp]
@@ -208,6 +211,12 @@ def la_state_decay(k, v, cu_seqlens, num_seqs, total_tokens, heads, d, dtype, in
 
 def la_decode_step_decay(q, k, v, state, o, batch, heads, d, dtype, decay, stream) -> int:
     return int(load_library().la_decode_step_decay(q, k, v, state, o, batch, heads, d, dtype, decay, stream))
+
+
+def la_state_exclusive_prefix_decay(gathered, seg_lens, world, rank, num_seqs, heads, d, decay, init, out,
+                                    stream) -> int:
+    return int(load_library().la_state_exclusive_prefix_decay(gathered, seg_lens, world, rank, num_seqs, heads, d,
+                                                               decay, init, out, stream))
 
 
 def la_feature_map(x, y, n, dtype, alpha, stream) -> int:
@@ -540,6 +549,30 @@ def decode_step_decay(q, k, v, state, decay, out=None, stream=None):
     status = la_decode_step_decay(_p(q), _p(k), _p(v), _p(state), _p(out), batch, H, d, code, _p(decay),
                                   _stream_handle(stream, q.device))
     _raise(status, "la_decode_step_decay")
+    return out
+
+
+def state_exclusive_prefix_decay(gathered, seg_lens, rank, decay, init=None, out=None, stream=None):
+    """Rank `rank`'s starting state with per-head decay for fp32 gathered [world, num_seqs, H, d, d] segment
+    states and int32 seg_lens [world, num_seqs] (see la_state_exclusive_prefix_decay)."""
+    _need(gathered, "gathered")
+    if gathered.dtype != torch.float32 or gathered.dim() != 5 or gathered.shape[-1] != gathered.shape[-2]:
+        raise LightningError("gathered must be fp32 [world, num_seqs, H, d, d]", 1)
+    world, nseq, H, d = gathered.shape[0], gathered.shape[1], gathered.shape[2], gathered.shape[3]
+    _need(seg_lens, "seg_lens", gathered.device)
+    if seg_lens.dtype != torch.int32 or tuple(seg_lens.shape) != (world, nseq):
+        raise LightningError("seg_lens must be int32 [world, num_seqs]", 1)
+    _decay_rates(decay, H, gathered.device)
+    if out is None:
+        out = torch.empty(gathered.shape[1:], dtype=torch.float32, device=gathered.device)
+    _need(out, "out", gathered.device)
+    if init is not None:
+        _need(init, "init", gathered.device)
+        if init.dtype != torch.float32 or init.shape != out.shape:
+            raise LightningError("init must be fp32 [num_seqs, H, d, d]", 1)
+    status = la_state_exclusive_prefix_decay(_p(gathered), _p(seg_lens), world, rank, nseq, H, d, _p(decay), _p(init),
+                                             _p(out), _stream_handle(stream, gathered.device))
+    _raise(status, "la_state_exclusive_prefix_decay")
     return out
 
 

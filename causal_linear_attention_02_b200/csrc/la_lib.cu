@@ -637,6 +637,36 @@ la_status la_decode_step(const void* q, const void* k, const void* v, float* sta
     return decode_d(d, dtype, q, k, v, state, o, pairs, nullptr, heads, reinterpret_cast<cudaStream_t>(stream));
 }
 
+la_status la_state_exclusive_prefix_decay(const float* gathered, const int32_t* seg_lens, int world, int rank,
+                                          int num_seqs, int heads, int d, const float* decay, const float* init,
+                                          float* out, void* stream) {
+    if (world < 1 || rank < 0 || rank > world || num_seqs < 0 || heads < 1) return LA_ERR_INVALID_ARGUMENT;
+    if (!supported_d(d)) return LA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return LA_OK;
+    if (!gathered || !out || !decay || (rank > 0 && !seg_lens)) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(gathered, 16) || !aligned(out, 16) || (init && !aligned(init, 16)) || !aligned(decay, 4) ||
+        (seg_lens && !aligned(seg_lens, 4)))
+        return LA_ERR_MISALIGNED;
+    const int64_t per_state = (int64_t)d * d;
+    const int64_t per_rank = (int64_t)num_seqs * heads * per_state;
+    const size_t bytes = (size_t)per_rank * 4;
+    if (overlaps(out, bytes, gathered, bytes * (size_t)world)) return LA_ERR_INVALID_ARGUMENT;
+    if (init && init != out && overlaps(out, bytes, init, bytes)) return LA_ERR_INVALID_ARGUMENT;
+    if (overlaps(out, bytes, decay, (size_t)heads * 4) ||
+        (seg_lens && overlaps(out, bytes, seg_lens, (size_t)world * num_seqs * 4)))
+        return LA_ERR_INVALID_ARGUMENT;
+    const int sms = num_sms();
+    if (sms <= 0) return LA_ERR_CUDA;
+    const int64_t per_rank4 = per_rank / 4;
+    const int64_t want = (per_rank4 + 255) / 256;
+    const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)sms * 8);
+    la::state_prefix_decay_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const float4*>(gathered), seg_lens, rank, num_seqs, heads, per_state / 4, per_rank4, decay,
+        reinterpret_cast<const float4*>(init), reinterpret_cast<float4*>(out));
+    note_launch();
+    return cuda_check();
+}
+
 la_status la_state_exclusive_prefix(const float* gathered, int world, int rank, int64_t n, int d, const float* init,
                                     float* out, void* stream) {
     if (world < 1 || rank < 0 || rank > world || n < 0) return LA_ERR_INVALID_ARGUMENT;

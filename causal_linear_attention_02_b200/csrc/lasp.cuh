@@ -12,6 +12,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "decay.cuh"
 
 namespace la {
 
@@ -27,6 +28,45 @@ state_prefix_kernel(const float4* __restrict__ gathered, int rank, int64_t per_r
             acc.y += x.y;
             acc.z += x.z;
             acc.w += x.w;
+        }
+        out[i] = acc;
+    }
+}
+
+// With a decay rate per head on the state (decay.cuh), rank r's starting state
+// is P_r = lambda_h^(n_{r-1}) P_{r-1} + S_{r-1}, P_0 = S0, where S_{r'} is rank
+// r''s segment state (itself decayed to the segment's end) and n_{r'} the
+// length of rank r''s segment of the sequence. seg_lens: [world][nseq] int32.
+// A bad rate (LA_ERR_BAD_DECAY) or a negative length (LA_ERR_BAD_SEQLENS)
+// leaves that state unwritten.
+__global__ void __launch_bounds__(256)
+state_prefix_decay_kernel(const float4* __restrict__ gathered, const int32_t* __restrict__ seg_lens, int rank,
+                          int nseq, int H, int64_t per_state4, int64_t per_rank4, const float* decay,
+                          const float4* init, float4* out) {
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < per_rank4; i += step) {
+        const int64_t pair = i / per_state4;              // (sequence, head)
+        const int s = (int)(pair / H), h = (int)(pair % H);
+        float l2;
+        if (!load_decay(decay, h, l2)) continue;
+        float4 acc = init ? init[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        bool ok = true;
+        for (int r = 0; r < rank; ++r) {
+            const int n = seg_lens[(int64_t)r * nseq + s];
+            if (n < 0) {
+                ok = false;
+                break;
+            }
+            const float w = decay_pow(l2, n);
+            const float4 x = __ldcs(gathered + (int64_t)r * per_rank4 + i);
+            acc.x = fmaf(w, acc.x, x.x);
+            acc.y = fmaf(w, acc.y, x.y);
+            acc.z = fmaf(w, acc.z, x.z);
+            acc.w = fmaf(w, acc.w, x.w);
+        }
+        if (!ok) {
+            record_status(LA_ERR_BAD_SEQLENS);
+            continue;
         }
         out[i] = acc;
     }

@@ -238,6 +238,28 @@ la_status la_decode_step(const void* q, const void* k, const void* v, float* sta
  * runs on CUDA cores in fp32.
  */
 
+/*
+ * The exclusive prefix of LASP+ sequence parallelism with decay: rank `rank`'s
+ * starting state when every rank holds one contiguous segment of the same
+ * sequences, ranks in sequence order.
+ *   P_0 = S0 (init, or zero),  P_r = lambda_h^(n_{r-1}) P_{r-1} + S_{r-1}
+ *   gathered  in   fp32 [world][num_seqs][heads][d][d]: rank r's segment states
+ *                  from a zero start (la_state_decay of its segments)
+ *   seg_lens  in   int32 [world][num_seqs]: length of rank r's segment of each
+ *                  sequence (>= 0); may be NULL when rank == 0
+ *   decay     in   fp32 [heads], rates in [0, 1]
+ *   init      in   fp32 [num_seqs][heads][d][d] or NULL; may be `out` itself
+ *   out       out  fp32 [num_seqs][heads][d][d]; rank == world gives the state
+ *                  after the last segment
+ * All device pointers; gathered, init and out 16-byte aligned, seg_lens and
+ * decay 4-byte aligned. Errors as la_state_exclusive_prefix; on the device a bad
+ * rate (LA_ERR_BAD_DECAY) or a negative length (LA_ERR_BAD_SEQLENS) leaves the
+ * affected states unwritten.
+ */
+la_status la_state_exclusive_prefix_decay(const float* gathered, const int32_t* seg_lens, int world, int rank,
+                                          int num_seqs, int heads, int d, const float* decay, const float* init,
+                                          float* out, void* stream);
+
 /* Workspace for la_prefill_decay; 0 for an unsupported shape. */
 size_t la_prefill_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
                                        la_dtype dtype);

@@ -160,6 +160,20 @@ def test_decay_argument_errors(lib):
     assert dec(s=2 * P) == 1
     assert dec(b=0) == 0
 
+    def pre_decay(**kw):
+        a = dict(g=P, lens=2 * P, world=2, rank=1, nseq=3, H=2, d=64, decay=3 * P, init=None, out=4 * P)
+        a.update(kw)
+        return la.la_state_exclusive_prefix_decay(a["g"], a["lens"], a["world"], a["rank"], a["nseq"], a["H"], a["d"],
+                                                  a["decay"], a["init"], a["out"], None)
+    assert pre_decay(rank=3) == 1                       # rank above world
+    assert pre_decay(H=0) == 1
+    assert pre_decay(d=20) == 2
+    assert pre_decay(decay=None) == 1
+    assert pre_decay(lens=None) == 1                    # rank > 0 needs the segment lengths
+    assert pre_decay(lens=2 * P + 2) == 3
+    assert pre_decay(out=P) == 1                        # out inside the gathered states
+    assert pre_decay(nseq=0) == 0
+
     def fm(**kw):
         a = dict(x=P, y=2 * P, n=100, dt=la.LA_BF16, alpha=0.3)
         a.update(kw)

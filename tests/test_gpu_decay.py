@@ -351,3 +351,55 @@ def test_prefill_decay_onchip_state_repeated(B):
         status_ok()
         assert_close(f64(o), ref_o, 1e-2, f"O, call {rep}")
         assert_close(st.cpu().double().numpy(), ref_st, 5e-3, f"final state, call {rep}")
+
+
+@pytest.mark.parametrize("W,B,H", [(2, 256, 32), (3, 128, 4), (4, 256, 4)])
+def test_lasp_decay_segments_on_one_gpu(W, B, H):
+    """LASP+ with decay composed from the library calls, the ranks emulated one after another on
+    one GPU (the all-gathers are stacks): segment states (la_state_decay), the decayed exclusive
+    prefix (la_state_exclusive_prefix_decay) and each segment's decay prefill from it equal the
+    whole sequences' output and final state. H = 32 puts the segment prefills on the tensor-core
+    path, H = 4 on CUDA cores."""
+    lengths, d = [1500, 777], 128
+    T = sum(lengths)
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, seed=80 + W, device=DEV)
+    init = wl.state_init(len(lengths), H, d, seed=9, device=DEV)
+    decay = wl.decay_rates(H, device=DEV)
+    rng = np.random.default_rng(W)
+    cuts = [[0, *np.sort(rng.choice(np.arange(1, L), size=W - 1, replace=False)).tolist(), L] for L in lengths]
+    starts = np.cumsum([0] + lengths[:-1])
+    rows = [np.concatenate([np.arange(s0 + c[r], s0 + c[r + 1]) for s0, c in zip(starts, cuts)]) for r in range(W)]
+    segs = []
+    for r in range(W):
+        idx = torch.from_numpy(rows[r]).to(DEV)
+        cu = wl.cu_seqlens([c[r + 1] - c[r] for c in cuts], device=DEV)
+        segs.append((q[idx].contiguous(), k[idx].contiguous(), v[idx].contiguous(), cu))
+    gathered = torch.stack([la.state_decay(kr, vr, decay, cu) for _, kr, vr, cu in segs])
+    seg_lens = torch.tensor([[c[r + 1] - c[r] for c in cuts] for r in range(W)], dtype=torch.int32, device=DEV)
+    o = torch.empty_like(q)
+    for r, (qr, kr, vr, cu) in enumerate(segs):
+        start = la.state_exclusive_prefix_decay(gathered, seg_lens, r, decay, init)
+        o[torch.from_numpy(rows[r]).to(DEV)] = la.prefill_decay(qr, kr, vr, decay, cu, B=B, init_state=start)
+    final = la.state_exclusive_prefix_decay(gathered, seg_lens, W, decay, init)
+    status_ok()
+    cu_all = wl.cu_seqlens(lengths).numpy()
+    ref, ref_state = oracle.decay_recurrent(f64(q), f64(k), f64(v), decay.cpu().double().numpy(), cu_all,
+                                            init=init.cpu().double().numpy(), return_state=True)
+    assert_close(f64(o), ref, 1e-2, "LASP+ output with decay")
+    assert_close(final.cpu().double().numpy(), ref_state, 1e-4, "LASP+ final state with decay")
+
+
+def test_state_exclusive_prefix_decay_arguments():
+    """Bad rates and negative lengths are reported on the device and leave the state unwritten."""
+    W, nseq, H, d = 2, 1, 2, 16
+    gathered = torch.randn((W, nseq, H, d, d), device=DEV)
+    seg_lens = torch.tensor([[3], [-1]], dtype=torch.int32, device=DEV)
+    decay = torch.tensor([0.5, 0.9], device=DEV)
+    out = torch.full((nseq, H, d, d), 7.0, device=DEV)
+    la.state_exclusive_prefix_decay(gathered, seg_lens, 2, decay, out=out)
+    assert la.device_status() == 7                      # LA_ERR_BAD_SEQLENS
+    assert torch.all(out == 7.0)
+    la.state_exclusive_prefix_decay(gathered, seg_lens, 1, torch.tensor([0.5, 2.0], device=DEV), out=out)
+    assert la.device_status() == 8                      # LA_ERR_BAD_DECAY: head 1 unwritten
+    assert torch.all(out[:, 1] == 7.0)
+    assert torch.allclose(out[:, 0], gathered[0, :, 0])

@@ -1,6 +1,6 @@
 """Sequence parallelism (LASP+) over several ranks: the driver's collective
 plumbing on CPU (gloo, one process per rank), checked against the oracle on
-the whole sequences.
+the whole sequences, with and without a decay rate per head.
 
 The three compute steps of ``lasp_prefill`` (segment state, exclusive prefix,
 prefill from a state) are passed in as oracle-backed ops here, so the test
@@ -23,19 +23,33 @@ import workloads as wl
 
 
 class OracleOps:
-    """fp64 CPU stand-ins for the library's three LASP+ steps."""
+    """fp64 CPU stand-ins for the library's three LASP+ steps (decay: the per-head rates, or None)."""
 
     @staticmethod
-    def segment_state(k, v, cu):
+    def segment_state(k, v, cu, decay=None):
+        if decay is not None:
+            return torch.from_numpy(oracle.decay_state(k.numpy(), v.numpy(), decay.numpy(), cu.numpy()))
         return torch.from_numpy(oracle.state(k.numpy(), v.numpy(), cu.numpy()))
 
     @staticmethod
-    def exclusive_prefix(gathered, rank, init):
-        s = gathered[:rank].sum(0)
-        return s if init is None else s + init
+    def exclusive_prefix(gathered, rank, init, seg_lens=None, decay=None):
+        if decay is None:
+            s = gathered[:rank].sum(0)
+            return s if init is None else s + init
+        # the state before rank `rank`'s segment: run the earlier segments' states forward, each
+        # discounted by lambda to the power of its segment's length before the next is added
+        lam = decay.double().numpy()[None, :, None, None]              # [1, H, 1, 1]
+        acc = np.zeros(gathered.shape[1:]) if init is None else init.double().numpy().copy()
+        for r in range(rank):
+            n = seg_lens[r].numpy().astype(np.float64)[:, None, None, None]   # [nseq, 1, 1, 1]
+            acc = lam ** n * acc + gathered[r].double().numpy()
+        return torch.from_numpy(acc)
 
     @staticmethod
-    def prefill(q, k, v, cu, B, init, out):
+    def prefill(q, k, v, cu, B, init, out, decay=None):
+        if decay is not None:
+            return torch.from_numpy(oracle.decay_blocked(q.numpy(), k.numpy(), v.numpy(), decay.numpy(), B,
+                                                         cu.numpy(), init=init.numpy()))
         return torch.from_numpy(oracle.blocked(q.numpy(), k.numpy(), v.numpy(), B, cu.numpy(), init=init.numpy()))
 
 
@@ -61,7 +75,7 @@ def _segment(arr, lengths, cuts, r):
     return np.concatenate(parts, axis=0)
 
 
-def _worker(rank, world, port, seed, outdir):
+def _worker(rank, world, port, seed, outdir, with_decay=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
@@ -71,8 +85,9 @@ def _worker(rank, world, port, seed, outdir):
         seg_len = [c[rank + 1] - c[rank] for c in cuts]
         cu = torch.tensor(np.cumsum([0] + seg_len), dtype=torch.int32)
         qr, kr, vr = (torch.from_numpy(_segment(a, lengths, cuts, rank)) for a in (q, k, v))
+        decay = torch.from_numpy(np.array([0.7, 0.97])) if with_decay else None
         o, st = lasp_prefill(qr, kr, vr, cu, B=B, init_state=torch.from_numpy(init), return_state=True,
-                             ops=OracleOps)
+                             decay=decay, ops=OracleOps)
         np.save(os.path.join(outdir, f"o{rank}.npy"), o.numpy())
         np.save(os.path.join(outdir, f"s{rank}.npy"), st.numpy())
     finally:
@@ -85,15 +100,20 @@ def _free_port():
         return s.getsockname()[1]
 
 
+@pytest.mark.parametrize("with_decay", [False, True], ids=["plain", "decay"])
 @pytest.mark.parametrize("world", [2, 3])
-def test_lasp_prefill_matches_whole_sequences(world):
+def test_lasp_prefill_matches_whole_sequences(world, with_decay):
     seed = 40 + world
     with tempfile.TemporaryDirectory() as outdir:
-        mp.spawn(_worker, args=(world, _free_port(), seed, outdir), nprocs=world, join=True)
+        mp.spawn(_worker, args=(world, _free_port(), seed, outdir, with_decay), nprocs=world, join=True)
         lengths, H, d, B, q, k, v, init, cuts = _case(world, seed)
         cu = wl.cu_seqlens(lengths).numpy()
-        ref = oracle.recurrent(q, k, v, cu, init=init)
-        ref_state = oracle.state(k, v, cu, init=init)
+        if with_decay:
+            lam = np.array([0.7, 0.97])
+            ref, ref_state = oracle.decay_recurrent(q, k, v, lam, cu, init=init, return_state=True)
+        else:
+            ref = oracle.recurrent(q, k, v, cu, init=init)
+            ref_state = oracle.state(k, v, cu, init=init)
         for r in range(world):
             o = np.load(os.path.join(outdir, f"o{r}.npy"))
             want = _segment(ref, lengths, cuts, r)
