@@ -485,8 +485,37 @@ def pin_decay_split(impl):
     _close(st, impl.decay_state(k, v, lam, init=S0), 1e-11, "decay decode final state")
 
 
+def pin_decay_bruteforce_exact(impl):
+    """Exact rational arithmetic of the recurrence S_t = lambda S_{t-1} + k_t^T v_t, o_t = q_t S_t on
+    tiny integer inputs with rates 1/2 and 3/4 and an integer S0: every value is a dyadic rational
+    that fp64 holds exactly, so each form must match bit for bit."""
+    r = _rng(46)
+    T, H, d = 7, 2, 3
+    q, k, v = (r.integers(-3, 4, size=(T, H, d)) for _ in range(3))
+    S0 = r.integers(-2, 3, size=(2, H, d, d))
+    lam = [Fraction(1, 2), Fraction(3, 4)]
+    cu = [0, 3, 7]
+    want = np.zeros((T, H, d))
+    want_st = np.zeros((2, H, d, d))
+    for si in range(2):
+        for h in range(H):
+            S = [[Fraction(int(S0[si, h, i, j])) for j in range(d)] for i in range(d)]
+            for t in range(cu[si], cu[si + 1]):
+                S = [[lam[h] * S[i][j] + int(k[t, h, i]) * int(v[t, h, j]) for j in range(d)] for i in range(d)]
+                want[t, h] = [float(sum(int(q[t, h, i]) * S[i][j] for i in range(d))) for j in range(d)]
+            want_st[si, h] = [[float(x) for x in row] for row in S]
+    qf, kf, vf, s0 = (x.astype(np.float64) for x in (q, k, v, S0))
+    lf = np.array([0.5, 0.75])
+    assert np.array_equal(impl.decay_quadratic(qf, kf, vf, lf, cu, init=s0), want), "decay brute force (quadratic)"
+    assert np.array_equal(impl.decay_recurrent(qf, kf, vf, lf, cu, init=s0), want), "decay brute force (recurrent)"
+    for B in (1, 2, 3, 5, 8):
+        assert np.array_equal(impl.decay_blocked(qf, kf, vf, lf, B, cu, init=s0), want), \
+            f"decay brute force (blocked B={B})"
+    assert np.array_equal(impl.decay_state(kf, vf, lf, cu, init=s0), want_st), "decay brute force (state)"
+
+
 DECAY_PINS = [pin_decay_change_of_variables, pin_decay_one, pin_decay_zero, pin_decay_discounted_cumsum,
-              pin_decay_split]
+              pin_decay_split, pin_decay_bruteforce_exact]
 
 
 # --------------------------------------------------------------------------- feature map

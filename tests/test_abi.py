@@ -208,3 +208,19 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(la, "_lib", None)
     with pytest.raises(la.LightningError):
         la.load_library()
+
+
+def test_decay_conveniences_reject_host_tensors():
+    """The decay and feature-map conveniences take device tensors only; host tensors raise
+    (the library has no CPU path)."""
+    import torch
+    x = torch.zeros(8, 2, 16)
+    rates = torch.ones(2)
+    for call in (lambda: la.prefill_decay(x, x, x, rates),
+                 lambda: la.state_decay(x, x, rates),
+                 lambda: la.decode_step_decay(x, x, x, torch.zeros(8, 2, 16, 16), rates),
+                 lambda: la.feature_map(x),
+                 lambda: la.state_exclusive_prefix_decay(torch.zeros(2, 1, 2, 16, 16),
+                                                         torch.zeros(2, 1, dtype=torch.int32), 1, rates)):
+        with pytest.raises(la.LightningError):
+            call()
