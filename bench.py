@@ -157,7 +157,9 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- distributed
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU under torchrun (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_* from the
+    environment). The benchmark uses NCCL; gloo serves the host-side tests."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -167,22 +169,33 @@ def dist_setup(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
         pg = dist
     return rank, local, world, pg
 
 
+def _on_gpus(pg) -> bool:
+    return pg.get_backend() == "nccl"
+
+
 def barrier(pg, local):
     if pg is not None:
-        pg.barrier(device_ids=[local])
+        if _on_gpus(pg):
+            pg.barrier(device_ids=[local])
+        else:
+            pg.barrier()
 
 
 def max_over_ranks(pg, x: float) -> float:
+    """The largest of the ranks' values (every rank gets it): times are reported as the slowest rank's."""
     if pg is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if _on_gpus(pg) else "cpu")
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 
