@@ -13,6 +13,13 @@
  * decode step is the recurrent form S <- S + k^T v, o = q S, O(d^2) per token
  * (same page, same section, and section "与标准 Softmax Attention 的区别").
  *
+ * Beside the method itself: its final states in the same pass
+ * (la_prefill_with_state), its gradients (la_prefill_backward), the prefix of
+ * LASP+ sequence parallelism (la_state_exclusive_prefix), a variant with a
+ * decay rate per head on the state (la_prefill_decay, la_state_decay,
+ * la_decode_step_decay, la_state_exclusive_prefix_decay; not on the pages),
+ * and the feature map of one page as a separate pre-pass (la_feature_map).
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - All tensor pointers are DEVICE pointers owned by the caller. The library
@@ -37,9 +44,10 @@
  * ------
  *  Host-checkable argument errors are returned before anything is enqueued.
  *  Launch errors return LA_ERR_CUDA. Conditions only visible on the device
- *  (cu_seqlens inconsistent with total_tokens, a bounded wait that ran out)
- *  set a per-device status word that la_get_device_status reports; the
- *  affected launch then writes no output rows.
+ *  (cu_seqlens inconsistent with total_tokens, a bounded wait that ran out, a
+ *  decay rate outside [0, 1]) set a per-device status word that
+ *  la_get_device_status reports; the affected launch then writes no output
+ *  rows (the decay entry points state what they leave unwritten).
  */
 #ifndef LIGHTNING_ATTENTION_H
 #define LIGHTNING_ATTENTION_H
