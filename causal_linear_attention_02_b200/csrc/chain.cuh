@@ -752,13 +752,62 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         Cursor c;
         c.init(p);
         while (ok && c.valid) {
+            if constexpr (kDecay) {
+                // KV_b (or S0) -> bf16 operand of the inter-block product, one 32-column half at a
+                // time straight into the shared buffer, and lambda^rows KV_b back into the
+                // accumulator for this block's keys
+                if (c.b > 0) {
+                    if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
+                    ++kvc;
+                    tc_fence_after();
+                }
+                if (!warp_all(wait_bar(&bars->sb_empty, (c.n & 1) ^ 1, ab))) { ok = false; break; }
+                const bool has = c.b > 0 || p.init != nullptr;
+                const float wn = decay_pow(log2f(__ldg(p.decay + c.h)), c.rows);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a[32];
+                    if (c.b > 0) {
+                        tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                        tmem_wait_ld();
+                    } else if (p.init) {
+                        const float4* s0 = reinterpret_cast<const float4*>(
+                            p.init + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half + 32 * hh);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 x = __ldg(s0 + q);
+                            a[4 * q] = __float_as_uint(x.x);
+                            a[4 * q + 1] = __float_as_uint(x.y);
+                            a[4 * q + 2] = __float_as_uint(x.z);
+                            a[4 * q + 3] = __float_as_uint(x.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) a[q] = 0u;
+                    }
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int gg = 4 * hh + g;                      // 16-byte chunk of row m
+                        *reinterpret_cast<uint4*>(sb + (m >> 3) * 1024 + (m & 7) * 128 + ((gg ^ (m & 7)) << 4)) =
+                            make_uint4(pack_bf16x2(__uint_as_float(a[8 * g]), __uint_as_float(a[8 * g + 1])),
+                                       pack_bf16x2(__uint_as_float(a[8 * g + 2]), __uint_as_float(a[8 * g + 3])),
+                                       pack_bf16x2(__uint_as_float(a[8 * g + 4]), __uint_as_float(a[8 * g + 5])),
+                                       pack_bf16x2(__uint_as_float(a[8 * g + 6]), __uint_as_float(a[8 * g + 7])));
+                    }
+                    if (has) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__uint_as_float(a[q]) * wn);
+                        tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                    }
+                }
+                if (has) tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars->kv_read[c.n & 3]);            // the accumulator may take this block's keys
+                fence_proxy_async_smem();
+                if (!(c.w == p.suppress_item && c.b == 1)) mbar_arrive(&bars->sb_full);
+            } else {
             // KV_b -> bf16 operand of the inter-block product (row m, 64 columns)
             uint32_t pk[32];
-            float l2 = 0.f, wn = 1.f;                   // decay: log2 of the rate, lambda^rows
-            if constexpr (kDecay) {
-                l2 = log2f(__ldg(p.decay + c.h));
-                wn = decay_pow(l2, c.rows);
-            }
             if (c.b > 0) {
                 if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
                 ++kvc;
@@ -769,28 +818,13 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     uint32_t a[32];
                     tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
                     tmem_wait_ld();
-                    if constexpr (kDecay) {
-                        // the accumulator carries lambda^rows KV_b into this block's keys
-#pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__uint_as_float(a[q]) * wn);
-                        tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
-                        if (hh == 1) {
-                            tmem_wait_st();
-                            tc_fence_before();
-                            mbar_arrive(&bars->kv_read[c.n & 3]);
-                        }
-                    } else {
-                        if (hh == 1) {
-                            tc_fence_before();
-                            mbar_arrive(&bars->kv_read[c.n & 3]);    // the accumulator may take this block's keys
-                        }
-#pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+                    if (hh == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&bars->kv_read[c.n & 3]);    // the accumulator may take this block's keys
                     }
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
                 }
             } else {
                 // A work item's first block: KV_0 = S0 (zero without a carried-in state).
@@ -809,19 +843,10 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                             a[4 * q + 2] = __float_as_uint(v.z);
                             a[4 * q + 3] = __float_as_uint(v.w);
                         }
-                        if constexpr (kDecay) {   // seeded as lambda^rows S0
+                        tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
 #pragma unroll
-                            for (int q = 0; q < 16; ++q)
-                                pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(__uint_as_float(a[q]) * wn);
-                            tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
-                        } else {
-                            tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);
-#pragma unroll
-                            for (int q = 0; q < 16; ++q)
-                                pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
-                        }
+                        for (int q = 0; q < 16; ++q)
+                            pk[16 * hh + q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
                     }
                     tmem_wait_st();
                 } else {
@@ -838,6 +863,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
             fence_proxy_async_smem();
             if (!(c.w == p.suppress_item && c.b == 1)) mbar_arrive(&bars->sb_full);
+            }
             if (wt == 0) LA_CTRACE(c.n, TR_SB);
             if (kStateOut && !c.add_state) {
                 // the work item's last block: its state MMAs complete the final state
@@ -858,7 +884,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 // the tokens past the last full 16-key step, on CUDA cores
                 for (int t = c.tok0 + (c.rows & ~15); t < c.tok0 + c.rows; ++t) {
                     float ki = __bfloat162float(p.k[((int64_t)t * p.H + c.h) * D + m]);
-                    if constexpr (kDecay) ki *= decay_pow(l2, c.tok0 + c.rows - 1 - t);
+                    if constexpr (kDecay) ki *= decay_pow(log2f(__ldg(p.decay + c.h)), c.tok0 + c.rows - 1 - t);
                     const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + c.h) * D + DV * c.half);
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
