@@ -31,6 +31,9 @@ are pinned by reduction to the pinned no-decay functions through an exact
 change of variables (q_t -> lambda^(t+1) q_t, k_s -> lambda^-(s+1) k_s), by
 lambda = 1 and lambda = 0 closed forms, by a discounted cumulative sum computed
 with scipy's IIR filter, and by the splitting of a sequence at any token.
+``decay_backward`` (the gradients of the decay variant) is pinned by central
+differences through the pinned ``decay_quadratic`` and by reduction to
+``backward`` at lambda = 1.
 ``feature_map`` (phi(x) = ELU(x) + alpha x, page "MiniMax-M2.5语言模型：Linear
 Attention架构解析与实践", section 2.2) is pinned by torch's ELU and by values
 worked by hand.
@@ -81,6 +84,7 @@ def _load():
             lib.oracle_decay_blocked.argtypes = [dp, dp, dp, dp, ip, i, i, i, i, dp, dp, dp]
             lib.oracle_decay_state.argtypes = [dp, dp, ip, i, i, i, dp, dp, dp]
             lib.oracle_decay_decode_step.argtypes = [dp, dp, dp, dp, dp, i, i, i, dp]
+            lib.oracle_decay_backward.argtypes = [dp, dp, dp, dp, ip, i, i, i, dp, dp, dp, dp, dp, dp]
             lib.oracle_feature_map.argtypes = [dp, dp, ctypes.c_int64, ctypes.c_double]
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -293,6 +297,24 @@ def decay_decode_step(q, k, v, state_in, decay):
     o = np.zeros_like(q)
     _load().oracle_decay_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(st), _ptr(o), batch, H, d, _ptr(lam))
     return o, st
+
+
+def decay_backward(q, k, v, dout, decay, cu_seqlens=None, init=None):
+    """Gradients (dq, dk, dv, dinit) of L = sum_t dout_t . O_t for the decay variant's O."""
+    q, k, v = _check_qkv(q, k, v)
+    dout = _f64(dout)
+    if dout.shape != q.shape:
+        raise ValueError("dout must have the shape of q")
+    T, H, d = q.shape
+    cu, cup = _cu(cu_seqlens, T)
+    nseq = cu.size - 1
+    init = _init(init, nseq, H, d)
+    lam = _lam(decay, H)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    dinit = np.zeros((nseq, H, d, d))
+    _load().oracle_decay_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), cup, nseq, H, d, _ptr(init), _ptr(lam),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dinit))
+    return dq, dk, dv, dinit
 
 
 def feature_map(x, alpha=0.3):

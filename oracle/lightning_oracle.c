@@ -34,7 +34,8 @@
  *                       forward only, so this is the calculus of the forward
  *                       definition above, written out);
  *   oracle_decay_*    - the same forms with a per-head decay on the state (an
- *                       extension the pages do not give; defined further down);
+ *                       extension the pages do not give; defined further down),
+ *                       and their gradients;
  *   oracle_feature_map- the feature map phi one page gives, elementwise.
  *
  * Layout (all row-major, innermost index fastest):
@@ -444,6 +445,69 @@ void oracle_decay_decode_step(const double* q, const double* k, const double* v,
         for (int j = 0; j < d; ++j) op[j] = 0.0;
         for (int i = 0; i < d; ++i)
             for (int j = 0; j < d; ++j) op[j] += qp[i] * S[(int64_t)i * d + j];
+    }
+}
+
+/*
+ * Gradients of L = sum_t dO_t . O_t for the decay variant, per (sequence, head):
+ *   dq_t = dO_t S_t^T                         with S_t = lambda S_{t-1} + k_t^T v_t (forward)
+ *   R_s  = lambda R_{s+1} + q_s^T dO_s        (reverse, R past the end = 0)
+ *   dk_s = v_s R_s^T,   dv_s = k_s R_s,   dS0 = lambda R_start
+ * (R_s = sum_{t >= s} lambda^(t-s) q_t^T dO_t; S0 enters O_t with lambda^(t-start+1)).
+ */
+void oracle_decay_backward(const double* q, const double* k, const double* v, const double* dout,
+                           const int32_t* cu_seqlens, int nseq, int H, int d, const double* init,
+                           const double* lam, double* dq, double* dk, double* dv, double* dinit)
+{
+    int64_t npairs = (int64_t)nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t p = 0; p < npairs; ++p) {
+        int s = (int)(p / H), h = (int)(p % H);
+        int64_t start = cu_seqlens[s], end = cu_seqlens[s + 1];
+        double* S = (double*)calloc((size_t)d * d, sizeof(double));
+        if (init) memcpy(S, state_ptr(init, s, h, H, d), sizeof(double) * d * d);
+        for (int64_t t = start; t < end; ++t) {
+            const double* kt = k + at3(t, h, 0, H, d);
+            const double* vt = v + at3(t, h, 0, H, d);
+            const double* gt = dout + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j)
+                    S[(int64_t)i * d + j] = lam[h] * S[(int64_t)i * d + j] + kt[i] * vt[j];
+            double* dqt = dq + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += gt[j] * S[(int64_t)i * d + j];
+                dqt[i] = acc;
+            }
+        }
+        double* R = S;                                   /* reused: reverse state */
+        memset(R, 0, sizeof(double) * d * d);
+        for (int64_t t = end - 1; t >= start; --t) {
+            const double* qt = q + at3(t, h, 0, H, d);
+            const double* kt = k + at3(t, h, 0, H, d);
+            const double* vt = v + at3(t, h, 0, H, d);
+            const double* gt = dout + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i)
+                for (int j = 0; j < d; ++j)
+                    R[(int64_t)i * d + j] = lam[h] * R[(int64_t)i * d + j] + qt[i] * gt[j];
+            double* dkt = dk + at3(t, h, 0, H, d);
+            double* dvt = dv + at3(t, h, 0, H, d);
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += R[(int64_t)i * d + j] * vt[j];
+                dkt[i] = acc;
+            }
+            for (int j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i) acc += kt[i] * R[(int64_t)i * d + j];
+                dvt[j] = acc;
+            }
+        }
+        if (dinit) {
+            double* g0 = (double*)state_ptr(dinit, s, h, H, d);
+            for (int64_t x = 0; x < (int64_t)d * d; ++x) g0[x] = lam[h] * R[x];
+        }
+        free(S);
     }
 }
 

@@ -537,3 +537,57 @@ def pin_feature_map(impl):
 
 
 FEATURE_PINS = [pin_feature_map]
+
+
+# --------------------------------------------------------------------------- decay backward
+def pin_decay_backward_finite_differences(impl):
+    """Every gradient of the decay variant equals the central difference of L through the pinned
+    ``decay_quadratic``; O is linear in each of q, k, v and S0 taken alone, so a step of 1 gives
+    the derivative exactly, up to rounding."""
+    r = _rng(47)
+    cu = [0, 5, 9]
+    T, H, d = 9, 2, 3
+    q, k, v, do = (r.standard_normal((T, H, d)) for _ in range(4))
+    init = r.standard_normal((2, H, d, d))
+    lam = np.array([0.6, 0.9])
+    dq, dk, dv, dinit = impl.decay_backward(q, k, v, do, lam, cu, init)
+    args = {"q": q, "k": k, "v": v, "init": init}
+
+    def loss(a):
+        return float((do * impl.decay_quadratic(a["q"], a["k"], a["v"], lam, cu, init=a["init"])).sum())
+
+    for name, grad in (("q", dq), ("k", dk), ("v", dv), ("init", dinit)):
+        x = args[name]
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            plus, minus = dict(args), dict(args)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += 1.0
+            xm[idx] -= 1.0
+            plus[name], minus[name] = xp, xm
+            fd[idx] = 0.5 * (loss(plus) - loss(minus))
+        _close(grad, fd, 1e-10, f"decay dL/d{name}")
+
+
+def pin_decay_backward_one_and_zero(impl):
+    """lambda = 1 is the backward without decay; lambda = 0 leaves O_t = (q_t . k_t) v_t, whose
+    gradients are dq_t = (dO_t . v_t) k_t, dk_t = (dO_t . v_t) q_t, dv_t = (q_t . k_t) dO_t, dS0 = 0."""
+    r = _rng(48)
+    cu = [0, 4, 11]
+    T, H, d = 11, 2, 3
+    q, k, v, do = (r.standard_normal((T, H, d)) for _ in range(4))
+    init = r.standard_normal((2, H, d, d))
+    got = impl.decay_backward(q, k, v, do, np.ones(H), cu, init)
+    want = impl.backward(q, k, v, do, cu, init)
+    for name, a, b in zip(("dq", "dk", "dv", "dS0"), got, want):
+        _close(a, b, 1e-12, f"lambda = 1: {name}")
+    dq, dk, dv, dinit = impl.decay_backward(q, k, v, do, np.zeros(H), cu, init)
+    gv = np.einsum("thj,thj->th", do, v)[:, :, None]
+    qk = np.einsum("thi,thi->th", q, k)[:, :, None]
+    _close(dq, gv * k, 1e-14, "lambda = 0: dq")
+    _close(dk, gv * q, 1e-14, "lambda = 0: dk")
+    _close(dv, qk * do, 1e-14, "lambda = 0: dv")
+    assert np.array_equal(dinit, np.zeros_like(dinit)), "lambda = 0: dS0"
+
+
+DECAY_BACKWARD_PINS = [pin_decay_backward_finite_differences, pin_decay_backward_one_and_zero]

@@ -368,3 +368,56 @@ def test_feature_map_pin_is_sharp(bug):
     except AssertionError:
         caught = True
     assert caught == (bug is not None)
+
+
+class DecayBackwardTwin(DecayTwin):
+    """numpy restatement of the decay variant's gradients with an optional planted bug (its
+    forward and plain backward are the clean twin's)."""
+
+    def __init__(self, bug=None):
+        super().__init__(None)
+        self.gbug = bug
+
+    def decay_backward(self, q, k, v, dout, decay, cu_seqlens=None, init=None):
+        q, k, v, g = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
+        T, H, d = q.shape
+        cu = self._cu(T, cu_seqlens)
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+        dinit = np.zeros((len(cu) - 1, H, d, d))
+        for s in range(len(cu) - 1):
+            a, b = cu[s], cu[s + 1]
+            for h in range(H):
+                lam = decay[h]
+                S = self._init(init, s, h, d)
+                for t in range(a, b):
+                    S = (S if self.gbug == "gbwd_forward_undecayed" else lam * S) + np.outer(k[t, h], v[t, h])
+                    dq[t, h] = S @ g[t, h]
+                R = np.zeros((d, d))
+                for t in range(b - 1, a - 1, -1):
+                    R = (R if self.gbug == "gbwd_reverse_undecayed" else lam * R) + np.outer(q[t, h], g[t, h])
+                    dk[t, h] = R @ v[t, h]
+                    dv[t, h] = R.T @ k[t, h]
+                dinit[s, h] = R if self.gbug == "gbwd_dinit_undecayed" else lam * R
+        return dq, dk, dv, dinit
+
+
+DECAY_BACKWARD_BUGS = ["gbwd_forward_undecayed", "gbwd_reverse_undecayed", "gbwd_dinit_undecayed"]
+
+
+def _failing_decay_backward_pins(impl):
+    failed = []
+    for pin in pins.DECAY_BACKWARD_PINS:
+        try:
+            pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+def test_clean_decay_backward_twin_passes():
+    assert _failing_decay_backward_pins(DecayBackwardTwin()) == []
+
+
+@pytest.mark.parametrize("bug", DECAY_BACKWARD_BUGS)
+def test_planted_decay_backward_bug_is_caught(bug):
+    assert _failing_decay_backward_pins(DecayBackwardTwin(bug)), f"no pin catches {bug!r}"

@@ -20,6 +20,11 @@ def test_oracle_decay_and_feature_pin(pin):
     pin(oracle)
 
 
+@pytest.mark.parametrize("pin", pins.DECAY_BACKWARD_PINS, ids=lambda p: p.__name__)
+def test_oracle_decay_backward_pin(pin):
+    pin(oracle)
+
+
 def test_oracle_validates_arguments():
     import numpy as np
     q = np.zeros((4, 1, 2))
