@@ -28,10 +28,12 @@ __all__ = [
     "la_prefill_with_state_workspace_size", "la_prefill_with_state",
     "la_decode_step", "la_prefill_decay_workspace_size", "la_prefill_decay", "la_state_decay_workspace_size",
     "la_state_decay", "la_decode_step_decay", "la_feature_map", "la_state_exclusive_prefix_decay",
+    "la_prefill_backward_decay_workspace_size", "la_prefill_backward_decay",
     "la_get_device_status", "la_set_kernel_timer", "la_debug_set_fault", "la_debug_set_trace", "la_debug_set_path", "la_status_string", "la_version",
     "la_launch_count",
     "prefill", "prefill_with_state", "prefill_backward", "state_from_prefill", "state_exclusive_prefix", "decode_step", "device_status",
     "prefill_decay", "state_decay", "decode_step_decay", "feature_map", "state_exclusive_prefix_decay",
+    "prefill_backward_decay",
     "uses_tensor_cores",
 ]
 
@@ -107,6 +109,11 @@ def load_library():
         lib.la_decode_step_decay.restype = i32
         lib.la_state_exclusive_prefix_decay.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         lib.la_state_exclusive_prefix_decay.restype = i32
+        lib.la_prefill_backward_decay_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32]
+        lib.la_prefill_backward_decay_workspace_size.restype = sz
+        lib.la_prefill_backward_decay.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, vp, vp, vp, vp,
+                                                  vp, vp, vp, sz, vp]
+        lib.la_prefill_backward_decay.restype = i32
         lib.la_feature_map.argtypes = [vp, vp, i64, i32, ctypes.c_float, vp]
         lib.la_feature_map.restype = i32
         lib.la_get_device_status.argtypes = [vp]
@@ -217,6 +224,17 @@ def la_state_exclusive_prefix_decay(gathered, seg_lens, world, rank, num_seqs, h
                                     stream) -> int:
     return int(load_library().la_state_exclusive_prefix_decay(gathered, seg_lens, world, rank, num_seqs, heads, d,
                                                                decay, init, out, stream))
+
+
+def la_prefill_backward_decay_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) -> int:
+    return int(load_library().la_prefill_backward_decay_workspace_size(total_tokens, num_seqs, heads, d, B, dtype))
+
+
+def la_prefill_backward_decay(q, k, v, dout, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state,
+                              decay, dq, dk, dv, dinit_state, workspace, workspace_bytes, stream) -> int:
+    return int(load_library().la_prefill_backward_decay(q, k, v, dout, cu_seqlens, num_seqs, total_tokens, heads, d,
+                                                        B, dtype, init_state, decay, dq, dk, dv, dinit_state,
+                                                        workspace, workspace_bytes, stream))
 
 
 def la_feature_map(x, y, n, dtype, alpha, stream) -> int:
@@ -574,6 +592,37 @@ def state_exclusive_prefix_decay(gathered, seg_lens, rank, decay, init=None, out
                                              _p(out), _stream_handle(stream, gathered.device))
     _raise(status, "la_state_exclusive_prefix_decay")
     return out
+
+
+def prefill_backward_decay(q, k, v, dout, decay, cu_seqlens=None, B: int = 256, init_state=None,
+                           need_init_grad=False, workspace=None, stream=None):
+    """(dq, dk, dv, dinit) of L = sum_t dout_t . O_t for O = prefill_decay(q, k, v, decay, ...) (see
+    la_prefill_backward_decay); dinit is None unless need_init_grad."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _need(t, n, q.device)
+    if q.dim() != 3 or any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, dout)):
+        raise LightningError("q, k, v, dout must share one [T, H, d] shape and dtype", 1)
+    T, H, d = q.shape
+    _decay_rates(decay, H, q.device)
+    nseq = 1
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", q.device)
+        nseq = cu_seqlens.numel() - 1
+    if init_state is not None:
+        _need(init_state, "init_state", q.device)
+    code = _dtype_code(q.dtype)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dinit = torch.empty((nseq, H, d, d), dtype=torch.float32, device=q.device) if need_init_grad else None
+    ws_bytes = la_prefill_backward_decay_workspace_size(T, nseq, H, d, B, code)
+    if ws_bytes == 0:
+        raise LightningError(f"unsupported prefill shape T={T} H={H} d={d} B={B}", 2)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    status = la_prefill_backward_decay(_p(q), _p(k), _p(v), _p(dout), _p(cu_seqlens), nseq, T, H, d, B, code,
+                                       _p(init_state), _p(decay), _p(dq), _p(dk), _p(dv), _p(dinit), _p(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
+    _raise(status, "la_prefill_backward_decay")
+    return dq, dk, dv, dinit
 
 
 def feature_map(x, alpha: float = 0.3, out=None, stream=None):

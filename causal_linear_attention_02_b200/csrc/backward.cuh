@@ -52,4 +52,17 @@ transpose_states_kernel(const float* __restrict__ in, float* __restrict__ out, i
     }
 }
 
+// states[i] *= lambda_h for every (sequence, head) state of [nseq][H][d][d]
+// (the decay variant's dS0 = lambda R_start); float4 groups, grid-stride.
+__global__ void __launch_bounds__(256)
+scale_states_kernel(float4* states, const float* decay, int H, int64_t per_state4, int64_t total4) {
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total4; i += step) {
+        const float lam = decay[(i / per_state4) % H];
+        float4 x = states[i];
+        x.x *= lam; x.y *= lam; x.z *= lam; x.w *= lam;
+        states[i] = x;
+    }
+}
+
 }  // namespace la

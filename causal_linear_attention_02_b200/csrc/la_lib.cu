@@ -414,7 +414,8 @@ struct BackwardLayout {
     size_t tensor = 0, off_rk = 0, off_rq = 0, off_rdo = 0, off_rv = 0, off_rout = 0, off_s0t = 0, off_pws = 0,
            pws = 0, off_sws = 0, sws = 0, total = 0;
 };
-BackwardLayout backward_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt) {
+Layout simt_layout(int64_t T, int nseq, int H, int d, int B);
+BackwardLayout backward_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt, bool decay = false) {
     BackwardLayout L;
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     L.tensor = (size_t)T * H * d * esize(dt);
@@ -425,9 +426,13 @@ BackwardLayout backward_layout(int64_t T, int nseq, int H, int d, int B, la_dtyp
     L.off_rv = off; off = up(off + L.tensor);
     L.off_rout = off; off = up(off + L.tensor);
     L.off_s0t = off; off = up(off + (size_t)nseq * H * d * d * 4);
-    L.pws = prefill_layout(T, nseq, H, d, B, dt).total;
+    if (decay)   // the workspaces of la_prefill_decay and la_state_decay
+        L.pws = T > 0 && prefill_path(dt, d, B, nseq, H) == Path::chain ? prefill_layout(T, nseq, H, d, B, dt).total
+                                                                        : simt_layout(T, nseq, H, d, B).total;
+    else
+        L.pws = prefill_layout(T, nseq, H, d, B, dt).total;
     L.off_pws = off; off = up(off + L.pws);
-    L.sws = state_layout(T, nseq, H, d, dt).total;
+    L.sws = decay ? simt_state_layout(T, nseq, H, d).total : state_layout(T, nseq, H, d, dt).total;
     L.off_sws = off; off = up(off + L.sws);
     L.total = off;
     return L;
@@ -745,10 +750,45 @@ size_t la_prefill_backward_workspace_size(int64_t total_tokens, int num_seqs, in
     return backward_layout(total_tokens, num_seqs, heads, d, B, dtype).total;
 }
 
+static la_status prefill_backward_impl(const void* q, const void* k, const void* v, const void* dout,
+                                const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d,
+                                int B, la_dtype dtype, const float* init_state, const float* decay, void* dq,
+                                void* dk, void* dv, float* dinit_state, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 la_status la_prefill_backward(const void* q, const void* k, const void* v, const void* dout,
                               const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d, int B,
                               la_dtype dtype, const float* init_state, void* dq, void* dk, void* dv,
                               float* dinit_state, void* workspace, size_t workspace_bytes, void* stream) {
+    return prefill_backward_impl(q, k, v, dout, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state,
+                                 nullptr, dq, dk, dv, dinit_state, workspace, workspace_bytes, stream);
+}
+
+size_t la_prefill_backward_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                                la_dtype dtype) {
+    if (la_prefill_decay_workspace_size(total_tokens, num_seqs, heads, d, B, dtype) == 0) return 0;
+    return backward_layout(total_tokens, num_seqs, heads, d, B, dtype, true).total;
+}
+
+la_status la_prefill_backward_decay(const void* q, const void* k, const void* v, const void* dout,
+                                    const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d,
+                                    int B, la_dtype dtype, const float* init_state, const float* decay, void* dq,
+                                    void* dk, void* dv, float* dinit_state, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    if (!decay) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(decay, 4)) return LA_ERR_MISALIGNED;
+    return prefill_backward_impl(q, k, v, dout, cu_seqlens, num_seqs, total_tokens, heads, d, B, dtype, init_state,
+                                 decay, dq, dk, dv, dinit_state, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+// The backward pass without (decay = nullptr) or with a decay rate per head.
+static la_status prefill_backward_impl(const void* q, const void* k, const void* v, const void* dout,
+                                const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d,
+                                int B, la_dtype dtype, const float* init_state, const float* decay, void* dq,
+                                void* dk, void* dv, float* dinit_state, void* workspace, size_t workspace_bytes,
+                                void* stream) {
     la_status s = check_tokens(total_tokens, num_seqs, heads, d, dtype, cu_seqlens);
     if (s != LA_OK) return s;
     if (!supported_B(B)) return LA_ERR_UNSUPPORTED;
@@ -775,7 +815,10 @@ la_status la_prefill_backward(const void* q, const void* k, const void* v, const
         if (dinit_state && cudaMemsetAsync(dinit_state, 0, sb, st) != cudaSuccess) return LA_ERR_CUDA;
         return LA_OK;
     }
-    const BackwardLayout L = backward_layout(T, num_seqs, heads, d, B, dtype);
+    const BackwardLayout L = backward_layout(T, num_seqs, heads, d, B, dtype, decay != nullptr);
+    if (decay && (overlaps(decay, (size_t)heads * 4, dq, tb) || overlaps(decay, (size_t)heads * 4, dk, tb) ||
+                  overlaps(decay, (size_t)heads * 4, dv, tb)))
+        return LA_ERR_INVALID_ARGUMENT;
     if (!workspace) return LA_ERR_INVALID_ARGUMENT;
     if (!aligned(workspace, 256)) return LA_ERR_MISALIGNED;
     if (workspace_bytes < L.total) return LA_ERR_WORKSPACE_TOO_SMALL;
@@ -794,29 +837,43 @@ la_status la_prefill_backward(const void* q, const void* k, const void* v, const
         note_launch();
         if ((s = cuda_check()) != LA_OK) return s;
     }
-    if ((s = la_prefill(dout, v, k, dq, cu_seqlens, num_seqs, T, heads, d, B, dtype, init_state ? s0t : nullptr, pws,
-                        L.pws, stream)) != LA_OK)
-        return s;
+    auto fwd = [&](const void* a, const void* b, const void* c, void* out, const float* init) {
+        return decay ? la_prefill_decay(a, b, c, out, cu_seqlens, num_seqs, T, heads, d, B, dtype, init, decay, nullptr,
+                                        pws, L.pws, stream)
+                     : la_prefill(a, b, c, out, cu_seqlens, num_seqs, T, heads, d, B, dtype, init, pws, L.pws, stream);
+    };
+    if ((s = fwd(dout, v, k, dq, init_state ? s0t : nullptr)) != LA_OK) return s;
     // dV and dK: forward prefills over the reversed sequences, reversed back
     if ((s = launch_reverse(k, rk, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
         (s = launch_reverse(q, rq, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
         (s = launch_reverse(dout, rdo, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
         (s = launch_reverse(v, rv, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK)
         return s;
-    if ((s = la_prefill(rk, rq, rdo, rout, cu_seqlens, num_seqs, T, heads, d, B, dtype, nullptr, pws, L.pws, stream)) !=
-            LA_OK ||
+    if ((s = fwd(rk, rq, rdo, rout, nullptr)) != LA_OK ||
         (s = launch_reverse(rout, dv, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK)
         return s;
-    if ((s = la_prefill(rv, rdo, rq, rout, cu_seqlens, num_seqs, T, heads, d, B, dtype, nullptr, pws, L.pws, stream)) !=
-            LA_OK ||
+    if ((s = fwd(rv, rdo, rq, rout, nullptr)) != LA_OK ||
         (s = launch_reverse(rout, dk, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK)
         return s;
-    // dS0 = state of (Q, dO)
-    if (dinit_state)
+    if (!dinit_state) return LA_OK;
+    if (!decay)   // dS0 = state of (Q, dO)
         return la_state_from_prefill(q, dout, cu_seqlens, num_seqs, T, heads, d, dtype, nullptr, dinit_state,
                                      ws + L.off_sws, L.sws, stream);
-    return LA_OK;
+    // decay: dS0 = lambda R_start, R_start = the decayed state of the reversed (Q, dO)
+    if ((s = la_state_decay(rq, rdo, cu_seqlens, num_seqs, T, heads, d, dtype, nullptr, decay, dinit_state,
+                            ws + L.off_sws, L.sws, stream)) != LA_OK)
+        return s;
+    const int sms = num_sms();
+    if (sms <= 0) return LA_ERR_CUDA;
+    const int64_t per_state4 = (int64_t)d * d / 4, total4 = (int64_t)num_seqs * heads * per_state4;
+    const unsigned grid = (unsigned)std::min<int64_t>((total4 + 255) / 256, (int64_t)sms * 8);
+    la::scale_states_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<float4*>(dinit_state), decay, heads, per_state4,
+                                                 total4);
+    note_launch();
+    return cuda_check();
 }
+
+extern "C" {
 
 // ---------------------------------------------------------------- decay variant
 size_t la_prefill_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B, la_dtype dtype) {

@@ -291,6 +291,23 @@ la_status la_prefill_decay(const void* q, const void* k, const void* v, void* o,
                            const float* init_state, const float* decay, float* state_out, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Workspace for la_prefill_backward_decay; 0 for an unsupported shape. */
+size_t la_prefill_backward_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
+                                                la_dtype dtype);
+
+/*
+ * Gradients of L = sum_t dout_t . O_t for O = la_prefill_decay(...): arguments, layouts and errors
+ * as la_prefill_backward, plus `decay` as above. With R_s = sum_{t >= s} lambda^(t-s) q_t^T dO_t:
+ *   dq_t = dO_t S_t^T   (the decay prefill of (dO, V, K) from S0^T),
+ *   dk_s = R_s v_s, dv_s = R_s^T k_s   (decay prefills over the reversed sequences, reversed back),
+ *   dS0  = lambda R_start   (the decayed state of the reversed (Q, dO), times lambda).
+ */
+la_status la_prefill_backward_decay(const void* q, const void* k, const void* v, const void* dout,
+                                    const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d,
+                                    int B, la_dtype dtype, const float* init_state, const float* decay, void* dq,
+                                    void* dk, void* dv, float* dinit_state, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
 /* Workspace for la_state_decay; 0 for an unsupported shape. */
 size_t la_state_decay_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, la_dtype dtype);
 

@@ -403,3 +403,27 @@ def test_state_exclusive_prefix_decay_arguments():
     assert la.device_status() == 8                      # LA_ERR_BAD_DECAY: head 1 unwritten
     assert torch.all(out[:, 1] == 7.0)
     assert torch.allclose(out[:, 0], gathered[0, :, 0])
+
+
+@pytest.mark.parametrize("dtype,d,B,H,lengths", [
+    (torch.bfloat16, 128, 256, 32, [700, 0, 300]),      # tensor-core decay prefills
+    (torch.bfloat16, 128, 128, 4, [500, 1]),             # CUDA-core decay prefills (few work items)
+    (torch.float32, 64, 64, 2, [333, 129]),
+], ids=["bf16-onchip", "bf16-cudacores", "fp32"])
+@pytest.mark.parametrize("with_init", [False, True], ids=["zero-S0", "S0"])
+def test_prefill_backward_decay(dtype, d, B, H, lengths, with_init):
+    """Gradients of the decay variant against the oracle's (dq, dk, dv within the O bound of the
+    dtype, dS0 from a CUDA-core state pass within 1e-4)."""
+    T = sum(lengths)
+    q, k, v = wl.qkv(T, H, d, dtype, seed=90 + d, device=DEV)
+    do = wl.normal_scaled((T, H, d), d, dtype, 91, device=DEV)
+    cu = wl.cu_seqlens(lengths, device=DEV)
+    decay = wl.decay_rates(H, device=DEV)
+    init = wl.state_init(len(lengths), H, d, seed=12, device=DEV) if with_init else None
+    dq, dk, dv, dinit = la.prefill_backward_decay(q, k, v, do, decay, cu, B=B, init_state=init, need_init_grad=True)
+    status_ok()
+    ref = oracle.decay_backward(f64(q), f64(k), f64(v), f64(do), decay.cpu().double().numpy(), cu.cpu().numpy(),
+                                init=None if init is None else init.cpu().double().numpy())
+    for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
+        assert_close(f64(got), want, TOL[dtype], name)
+    assert_close(dinit.cpu().double().numpy(), ref[3], 1e-4, "dS0")
