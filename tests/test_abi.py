@@ -174,6 +174,22 @@ def test_decay_argument_errors(lib):
     assert pre_decay(out=P) == 1                        # out inside the gathered states
     assert pre_decay(nseq=0) == 0
 
+    def bwd(**kw):
+        a = dict(q=P, k=2 * P, v=3 * P, do=4 * P, cu=None, nseq=1, T=64, H=2, d=64, B=64, dt=la.LA_FP32, init=None,
+                 decay=9 * P, dq=5 * P, dk=6 * P, dv=7 * P, dinit=None, ws=8 * P, wsb=BIG)
+        a.update(kw)
+        return la.la_prefill_backward_decay(a["q"], a["k"], a["v"], a["do"], a["cu"], a["nseq"], a["T"], a["H"],
+                                            a["d"], a["B"], a["dt"], a["init"], a["decay"], a["dq"], a["dk"], a["dv"],
+                                            a["dinit"], a["ws"], a["wsb"], None)
+    assert bwd(decay=None) == 1
+    assert bwd(decay=9 * P + 2) == 3
+    assert bwd(decay=5 * P) == 1                        # rates inside dq
+    assert bwd(dq=P) == 1                               # dq aliases q
+    assert bwd(B=96) == 2
+    assert bwd(wsb=16) == 4
+    assert la.la_prefill_backward_decay_workspace_size(4096, 2, 4, 64, 64, la.LA_FP32) > 0
+    assert la.la_prefill_backward_decay_workspace_size(4096, 2, 4, 64, 48, la.LA_FP32) == 0
+
     def fm(**kw):
         a = dict(x=P, y=2 * P, n=100, dt=la.LA_BF16, alpha=0.3)
         a.update(kw)
