@@ -62,6 +62,9 @@ KERNEL_SOURCES = {
     "prefill_chain_kernel_decay": ("chain.cuh", "pipe.cuh", "sm100.cuh", "common.cuh", "decay.cuh"),
     "prefill_fused_kernel": ("fused.cuh", "pipe.cuh", "sm100.cuh", "common.cuh"),
     "decode_step_kernel": ("decode.cuh", "common.cuh"),
+    # the same kernel on the million-token and varlen workloads (traffic per launch differs)
+    "prefill_chain_kernel_1m": ("chain.cuh", "pipe.cuh", "sm100.cuh", "common.cuh"),
+    "prefill_chain_kernel_varlen": ("chain.cuh", "pipe.cuh", "sm100.cuh", "common.cuh"),
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
@@ -95,7 +98,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
-    def __init__(self, device, period_s=0.002):
+    def __init__(self, device, period_s=0.0005):
         self.device = device
         self.period = period_s
         self.samples = []
@@ -153,7 +156,7 @@ class ClockSampler:
         loaded = [x for x in sm if self.smax and x > 0.5 * self.smax] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": self.smax, "reasons": reasons,
                 "samples": len(sm), "sm_mhz_min": min(sm), "power_w_max": max(x[2] for x in self.samples),
-                "source": "NVML, every 2 ms during the timed region"}
+                "source": f"NVML, every {self.period * 1e3:g} ms during the timed region"}
 
 
 # ---------------------------------------------------------------------------- distributed
@@ -294,10 +297,23 @@ def run_cuda(args):
     if not args.no_decode:
         dec = run_decode(la, dev, stream, args, pk, pg, local)
 
-    # ---- decay variant on the same inputs (CUDA-core path), per-head rates of the decay recipe
+    # ---- decay variant on the same inputs (the decay instance of the tensor-core kernel), per-head
+    # rates of the decay recipe
     dcy = None
     if not args.no_decay:
         dcy = run_decay(la, dev, stream, args, pk, pg, local, q, k, v, o, w)
+
+    # ---- backward pass on the 32k workload
+    bwd = None
+    if not args.no_backward:
+        bwd = run_backward(la, dev, stream, args, pk, pg, local, q, k, v, w)
+
+    # ---- the million-token and the varlen workloads (prefill, same kernel)
+    big = {}
+    if not args.no_big:
+        for key, wk in (("long", wl.BF16_1M), ("varlen", wl.BF16_VARLEN)):
+            big[key] = run_prefill_workload(la, dev, stream, args, pk, pg, local, wk, key)
+            torch.cuda.empty_cache()
 
     # ---- end to end through host buffers, every step: H2D of q, k, v from pinned host memory,
     # la_prefill, D2H of o. Two device buffer sets and three streams, so that step i+1's upload
@@ -376,6 +392,9 @@ def run_cuda(args):
                          "algorithmic_bytes": alg_bytes},
             "decode": dec,
             "decay": dcy,
+            "backward": bwd,
+            "long": big.get("long"),
+            "varlen": big.get("varlen"),
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
@@ -392,7 +411,7 @@ def run_decode(la, dev, stream, args, pk, pg, local):
     import ctypes
     w = wl.DECODE
     Bt, H, d = w.decode_batch, w.heads, w.d
-    n_steps = min(w.decode_steps, max(args.steps * 10, 50))
+    n_steps = w.decode_steps                     # the workload's 1000 steps, every run
     T0 = Bt * w.prefill_len
     k0 = wl.normal_scaled((T0, H, d), d, torch.bfloat16, w.seed * 1000 + 1, device=dev)
     v0 = wl.normal_scaled((T0, H, d), d, torch.bfloat16, w.seed * 1000 + 2, device=dev)
@@ -515,6 +534,104 @@ def run_decay(la, dev, stream, args, pk, pg, local, q, k, v, o, w):
                          "algorithmic_bytes": alg_bytes}}
 
 
+def _timed_calls(la, dev, stream, pg, local, call, n, warmup):
+    """n timed calls after `warmup` untimed ones: (ms per call from events around all
+    calls, mean main-kernel ms from la_set_kernel_timer, launches per call)."""
+    import ctypes
+    for _ in range(warmup):
+        call()
+    timers = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in timers:
+        a.record(); b.record()
+    torch.cuda.synchronize(dev)
+    barrier(pg, local)
+    launches0 = la.la_launch_count()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for i in range(n):
+        la.la_set_kernel_timer(ctypes.c_void_p(timers[i][0].cuda_event), ctypes.c_void_p(timers[i][1].cuda_event))
+        call()
+    a1.record(stream)
+    launches = la.la_launch_count() - launches0
+    torch.cuda.synchronize(dev)
+    barrier(pg, local)
+    ms = max_over_ranks(pg, a0.elapsed_time(a1)) / n
+    kms = max_over_ranks(pg, statistics.mean(a.elapsed_time(b) for a, b in timers))
+    if la.device_status() != 0:
+        raise RuntimeError("device status after a timed sub-measurement")
+    return ms, kms, launches / n
+
+
+def run_prefill_workload(la, dev, stream, args, pk, pg, local, w, key):
+    """la_prefill on another workload of the same shape family: the million-token sequence
+    (Q, K, V, O of 16 GiB each) or the 16-sequence varlen pack (int32 cu_seqlens, state reset
+    at every sequence start). Same kernel, roofline and FLOP count as the main line."""
+    import ctypes
+    T, H, d, B = w.total_tokens, w.heads, w.d, w.B
+    nseq = len(w.seq_lens)
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, w.seed, device=dev)
+    o = torch.empty_like(q)
+    cu = wl.cu_seqlens(w.seq_lens, device=dev) if nseq > 1 else None
+    ws_bytes = la.la_prefill_workspace_size(T, nseq, H, d, B, la.LA_BF16)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+    def call():
+        s = la.la_prefill(P(q), P(k), P(v), P(o), P(cu), nseq, T, H, d, B, la.LA_BF16, None, P(ws), ws_bytes, sh)
+        if s != 0:
+            raise RuntimeError(f"la_prefill ({key}) failed: {la.STATUS.get(s, s)}")
+
+    n = 5 if T > 300000 else 10
+    ms, kms, launches = _timed_calls(la, dev, stream, pg, local, call, n, max(3, args.warmup))
+    del q, k, v, o, ws
+    alg_bytes = 8 * d * T * H
+    gbs = alg_bytes / (kms / 1e3) / 1e9
+    tflops = flops_per_token_head(B, d) * T * H / (ms / 1e3) / 1e12
+    return {"workload": w.name, "tokens": T, "sequences": nseq, "seed": w.seed, "steps": n,
+            "ms_per_step": ms, "kernel_ms": kms, "tokens_per_s": T / (ms / 1e3), "tflops": tflops,
+            "tc_peak_frac": tflops / pk["bf16_tflops"], "launches_per_step": launches,
+            "l2": "no flush: inputs far larger than the 126 MB L2",
+            "roofline": {"bound": "hbm", "kernel": "prefill_chain_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                         "traffic": captured_traffic("prefill_chain_kernel_" + ("1m" if key == "long" else key)),
+                         "algorithmic_bytes": alg_bytes}}
+
+
+def run_backward(la, dev, stream, args, pk, pg, local, q, k, v, w):
+    """la_prefill_backward on the 32k workload (dO iid like the inputs): dq, dk, dv.
+    Its launches run back to back, so the roofline uses the whole call's time:
+    algorithmic bytes = read Q, K, V, dO + write dQ, dK, dV (bf16) = 14 d bytes per
+    token-head; counted FLOPs = three forward products (dq, dk, dv), 3 (4 B d + 4 d^2)."""
+    import ctypes
+    T, H, d, B = w.total_tokens, w.heads, w.d, w.B
+    do = wl.normal_scaled((T, H, d), d, torch.bfloat16, w.seed * 1000 + 3, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws_bytes = la.la_prefill_backward_workspace_size(T, 1, H, d, B, la.LA_BF16)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    def call():
+        s = la.la_prefill_backward(P(q), P(k), P(v), P(do), None, 1, T, H, d, B, la.LA_BF16, None, P(dq), P(dk), P(dv),
+                                   None, P(ws), ws_bytes, sh)
+        if s != 0:
+            raise RuntimeError(f"la_prefill_backward failed: {la.STATUS.get(s, s)}")
+
+    n = 10
+    ms, _, launches = _timed_calls(la, dev, stream, pg, local, call, n, max(3, args.warmup))
+    del do, dq, dk, dv, ws
+    alg_bytes = 14 * d * T * H
+    gbs = alg_bytes / (ms / 1e3) / 1e9
+    tflops = 3 * flops_per_token_head(B, d) * T * H / (ms / 1e3) / 1e12
+    return {"workload": f"backward of the {w.name} prefill (dq, dk, dv)", "steps": n, "ms_per_step": ms,
+            "tokens_per_s": T / (ms / 1e3), "tflops": tflops, "tc_peak_frac": tflops / pk["bf16_tflops"],
+            "launches_per_step": launches,
+            "roofline": {"bound": "hbm", "kernel": f"la_prefill_backward (whole call, {launches:g} launches)",
+                         "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                         "traffic": None, "algorithmic_bytes": alg_bytes}}
+
+
 # ---------------------------------------------------------------------------- reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -565,6 +682,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-decay", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-big", action="store_true", help="skip the million-token and varlen sub-measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -825,6 +825,11 @@ static la_status prefill_backward_impl(const void* q, const void* k, const void*
     if (overlaps(workspace, L.total, dq, tb) || overlaps(workspace, L.total, dk, tb) ||
         overlaps(workspace, L.total, dv, tb) || (dinit_state && overlaps(workspace, L.total, dinit_state, sb)))
         return LA_ERR_INVALID_ARGUMENT;
+    // the rates are read by every pass: none of the workspace's copies may land on them,
+    // and the final dS0 scaling reads them while it writes dinit_state
+    if (decay && (overlaps(workspace, L.total, decay, (size_t)heads * 4) ||
+                  (dinit_state && overlaps(decay, (size_t)heads * 4, dinit_state, sb))))
+        return LA_ERR_INVALID_ARGUMENT;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     void *rk = ws + L.off_rk, *rq = ws + L.off_rq, *rdo = ws + L.off_rdo, *rv = ws + L.off_rv, *rout = ws + L.off_rout;
     float* s0t = reinterpret_cast<float*>(ws + L.off_s0t);

@@ -15,7 +15,11 @@
 // device address once, with cudaGetSymbolAddress, and caches it; that first
 // call should therefore happen before any stream capture. Every later call on
 // the device reuses the cached address. Nothing here calls cudaMalloc,
-// cudaFree or any allocating routine.
+// cudaFree or any allocating routine. Two limits follow from the cache: the
+// scratch is the current device's copy, so the caller's stream must belong to
+// the current device; and the cached address does not survive a
+// cudaDeviceReset of that device, after which this entry point may not be
+// called on it again.
 //
 // All calls on a device share the one array, which keeps whatever the last
 // call left in it: la_prefill rebuilds every part of its workspace that must

@@ -34,6 +34,18 @@ from . import (prefill, prefill_decay, state_decay, state_exclusive_prefix, stat
 __all__ = ["LibraryOps", "lasp_prefill"]
 
 
+def _all_gather(out: torch.Tensor, x: torch.Tensor, group) -> None:
+    """out[r] = rank r's x. NCCL (and any backend on host tensors) gathers in place;
+    a gloo group with device tensors gathers host copies (gloo moves host memory only),
+    which is how ranks that share one GPU, or a CPU-only cluster, run this driver."""
+    if x.is_cuda and dist.get_backend(group) == "gloo":
+        host = torch.empty(out.shape, dtype=out.dtype)
+        dist.all_gather(list(host.unbind(0)), x.cpu(), group=group)
+        out.copy_(host)
+    else:
+        dist.all_gather(list(out.unbind(0)), x, group=group)
+
+
 class LibraryOps:
     """The three compute steps, on the library's CUDA kernels (decay: the rates, or None)."""
 
@@ -77,7 +89,7 @@ def lasp_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: 
     else:
         local = ops.segment_state(k, v, cu_seqlens, decay)
     gathered = torch.empty((world,) + tuple(local.shape), dtype=local.dtype, device=local.device)
-    dist.all_gather(list(gathered.unbind(0)), local.contiguous(), group=group)
+    _all_gather(gathered, local.contiguous(), group)
     if decay is None:
         start = ops.exclusive_prefix(gathered, rank, init_state)
         o = ops.prefill(q, k, v, cu_seqlens, B, start, out)
@@ -88,7 +100,7 @@ def lasp_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: 
     else:
         lens = (cu_seqlens[1:] - cu_seqlens[:-1]).to(torch.int32).contiguous()
     seg_lens = torch.empty((world, lens.numel()), dtype=torch.int32, device=lens.device)
-    dist.all_gather(list(seg_lens.unbind(0)), lens, group=group)
+    _all_gather(seg_lens, lens, group)
     start = ops.exclusive_prefix(gathered, rank, init_state, seg_lens, decay)
     o = ops.prefill(q, k, v, cu_seqlens, B, start, out, decay)
     return (o, ops.exclusive_prefix(gathered, world, init_state, seg_lens, decay)) if return_state else o

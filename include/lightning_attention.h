@@ -116,7 +116,10 @@ la_status la_prefill(const void* q, const void* k, const void* v, void* o,
  * nothing: the first call on each device (with that device current) looks up
  * the array's device address once, so make that first call before any stream
  * capture. All calls on a device share the array; calls that overlap on the
- * GPU race and give undefined results.
+ * GPU race and give undefined results. The scratch used is the copy of the
+ * device current on the calling thread, so `stream` must belong to that
+ * device. The looked-up address is kept for the life of the process: after a
+ * cudaDeviceReset of a device, this entry point may not be called on it again.
  */
 #define LA_NOALLOC_SCRATCH_BYTES (64u << 20)
 la_status la_prefill_noalloc(const void* q, const void* k, const void* v, void* o,
@@ -301,6 +304,9 @@ size_t la_prefill_backward_decay_workspace_size(int64_t total_tokens, int num_se
  *   dq_t = dO_t S_t^T   (the decay prefill of (dO, V, K) from S0^T),
  *   dk_s = R_s v_s, dv_s = R_s^T k_s   (decay prefills over the reversed sequences, reversed back),
  *   dS0  = lambda R_start   (the decayed state of the reversed (Q, dO), times lambda).
+ * The rates are constants of this pass: no gradient with respect to lambda is
+ * computed or returned. `decay` may not overlap the workspace or dinit_state
+ * (LA_ERR_INVALID_ARGUMENT).
  */
 la_status la_prefill_backward_decay(const void* q, const void* k, const void* v, const void* dout,
                                     const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens, int heads, int d,

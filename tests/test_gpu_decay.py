@@ -427,3 +427,56 @@ def test_prefill_backward_decay(dtype, d, B, H, lengths, with_init):
     for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
         assert_close(f64(got), want, TOL[dtype], name)
     assert_close(dinit.cpu().double().numpy(), ref[3], 1e-4, "dS0")
+
+
+def _bits_equal_bf16(o, ref):
+    ref_b = torch.from_numpy(np.ascontiguousarray(ref)).to(torch.bfloat16)
+    return int((o.cpu().view(torch.int16) != ref_b.view(torch.int16)).sum().item())
+
+
+@pytest.mark.parametrize("B,T", [(256, 600), (128, 300)])
+def test_prefill_decay_tc_integer_exact_rate_one(B, T):
+    """Rate 1 on every head through the decay instance of the on-chip-state tensor-core kernel
+    (forced), {-1,0,1} inputs over several blocks: every power of the rate is exactly 1, so
+    the decay masks, weighted V and scaled Q rows change nothing, and the output must equal
+    the method without decay bit for bit (scores, P, prefixes and O are integers that bf16
+    and fp32 hold exactly)."""
+    H, d = 2, 128
+    q, k, v = wl.integer_qkv(T, H, d, torch.bfloat16, seed=B + T + 1, device=DEV)
+    for n in range(B, T, B):
+        assert np.abs(oracle.state(f64(k)[:n], f64(v)[:n])).max() <= 256, "precondition: bf16-exact prefix"
+    force = la.la_debug_set_path(1)
+    assert force == 0
+    try:
+        o = la.prefill_decay(q, k, v, torch.ones(H, dtype=torch.float32, device=DEV), B=B)
+    finally:
+        la.la_debug_set_path(0)
+    status_ok()
+    mism = _bits_equal_bf16(o, oracle.recurrent(f64(q), f64(k), f64(v)))
+    assert mism == 0, f"{mism} outputs differ from the exact result"
+
+
+@pytest.mark.parametrize("T", [8, 5])
+def test_prefill_decay_tc_integer_exact_dyadic(T):
+    """Dyadic rates 1/2 and 1/4 on the decay instance of the tensor-core kernel (forced), one
+    short block with {-1,0,1} inputs and an integer carried-in state: every power of the rate
+    is a power of two, every product (decay mask times score, rate times query row, weighted
+    value) is exact in bf16, and every sum spans fewer than 24 bits, so the output must equal
+    the exact result rounded to bf16 bit for bit. (Over longer sequences the powers 2^-n span
+    more bits than fp32 holds, so exactness stops there; those lengths are held to the
+    tolerance by the tests above.)"""
+    H, d, B = 2, 128, 256
+    rates = torch.tensor([0.5, 0.25], dtype=torch.float32, device=DEV)
+    q, k, v = wl.integer_qkv(T, H, d, torch.bfloat16, seed=700 + T, device=DEV)
+    g = torch.Generator().manual_seed(800 + T)
+    s0 = (torch.randint(0, 3, (1, H, d, d), generator=g) - 1).float().to(DEV)
+    assert la.la_debug_set_path(1) == 0
+    try:
+        o = la.prefill_decay(q, k, v, rates, B=B, init_state=s0)
+    finally:
+        la.la_debug_set_path(0)
+    status_ok()
+    ref = oracle.decay_recurrent(f64(q), f64(k), f64(v), rates.cpu().double().numpy(),
+                                 init=s0.cpu().double().numpy())
+    mism = _bits_equal_bf16(o, ref)
+    assert mism == 0, f"{mism} of {ref.size} outputs differ from the exact result"

@@ -129,6 +129,23 @@ def test_prefill_tc_integer_exact(B, T, tc_path):
     assert mism == 0, f"{mism} of {ref.numel()} outputs differ from the exact result"
 
 
+def test_prefill_fp32_integer_exact():
+    """The small fp32 workload's shape (T = 1024, H = 2, d = 64, B = 64: the CUDA-core
+    three-kernel path) with {-1,0,1} inputs: every score, block state, prefix entry and
+    output is an integer far below 2^24, exact in fp32, so the output must equal the
+    oracle's bit for bit."""
+    w = wl.FP32_SMALL
+    T, H, d, B = w.total_tokens, w.heads, w.d, w.B
+    q, k, v = wl.integer_qkv(T, H, d, torch.float32, seed=91, device=DEV)
+    o = la.prefill(q, k, v, B=B)
+    status_ok()
+    ref = oracle.recurrent(f64(q), f64(k), f64(v))
+    assert np.abs(ref).max() < 2 ** 24 and np.abs(oracle.state(f64(k), f64(v))).max() < 2 ** 24
+    got = o.cpu().double().numpy()
+    mism = int((got != ref).sum())
+    assert mism == 0, f"{mism} of {ref.size} fp32 outputs differ from the exact result"
+
+
 @pytest.mark.parametrize("B", [128, 256])
 def test_prefill_tc_varlen(B, tc_path):
     lengths = [1, 255, 256, 0, 257, 700, 64, 513, 128]

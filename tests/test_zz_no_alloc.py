@@ -3,9 +3,10 @@
 Such callers (allocator-free runtimes, fixed memory budgets, hooks running
 inside another library's memory manager) get the same prefill with the
 scratch taken from a static device array built into the library. These checks
-call it through the C ABI and compare it with the workspace entry point,
-la_prefill, on two calls in a row (the second call reuses the scratch the
-first one left behind), within the bf16 tolerance of the parity tests.
+call it through the C ABI and compare it with the fp64 oracle and with the
+workspace entry point, la_prefill, on two calls in a row (the second call
+reuses the scratch the first one left behind), within the tolerances of the
+parity tests.
 This file sorts last so that a failure here cannot hide another test's.
 """
 import ctypes
@@ -15,6 +16,7 @@ import pytest
 import torch
 
 import causal_linear_attention_02_b200 as la
+import oracle
 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -59,11 +61,21 @@ def test_noalloc_matches_workspace_prefill_twice(dtype, d, B):
         assert torch.isfinite(o.float()).all()
         r = _rel(o, ref)
         assert r <= tol, f"no-alloc vs workspace prefill: {r:.3e} > {tol:.0e}"
+        f = lambda t: t.float().cpu().double().numpy()
+        exact = oracle.recurrent(f(q), f(k), f(v), cu_seqlens=cu.cpu().numpy())
+        e = float(np.abs(f(o) - exact).max() / np.abs(exact).max())
+        assert e <= tol, f"no-alloc vs oracle: {e:.3e} > {tol:.0e}"
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    T, H, d, B = 1 << 16, 64, 128, 64            # fp32 keeps one state per block: ~8.6 GB of scratch
+    # fp32 at B = 64 keeps two d x d states per (block, head): 8192 tokens x 8 heads need
+    # about 132 MB of scratch, twice the static array
+    T, H, d, B = 8192, 8, 128, 64
     assert la.la_prefill_workspace_size(T, 1, H, d, B, la.LA_FP32) > la.LA_NOALLOC_SCRATCH_BYTES
-    P = 1 << 20                                  # never dereferenced: rejected on the host
-    status = la.la_prefill_noalloc(P, 2 * P, 3 * P, 4 * P, None, 1, T, H, d, B, la.LA_FP32, None, None)
-    assert status == 4                           # LA_ERR_WORKSPACE_TOO_SMALL
+    q, k, v = wl.qkv(T, H, d, torch.float32, 23, device=DEV)
+    o = torch.full_like(q, float("nan"))
+    stream = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
+    status = la.la_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), None, 1, T, H, d, B, la.LA_FP32, None, stream)
+    assert status == 4                           # LA_ERR_WORKSPACE_TOO_SMALL, before anything is enqueued
+    torch.cuda.synchronize(DEV)
+    assert torch.isnan(o).all()                  # nothing was written
