@@ -308,6 +308,12 @@ def run_cuda(args):
     if not args.no_backward:
         bwd = run_backward(la, dev, stream, args, pk, pg, local, q, k, v, w)
 
+    # ---- a serving batch: prompts and one-token continuations in one launch
+    mix = None
+    if not args.no_mixed:
+        mix = run_mixed(la, dev, stream, args, pk, pg, local)
+        torch.cuda.empty_cache()
+
     # ---- the million-token and the varlen workloads (prefill, same kernel)
     big = {}
     if not args.no_big:
@@ -393,6 +399,7 @@ def run_cuda(args):
             "decode": dec,
             "decay": dcy,
             "backward": bwd,
+            "mixed": mix,
             "long": big.get("long"),
             "varlen": big.get("varlen"),
             "e2e": e2e,
@@ -632,6 +639,63 @@ def run_backward(la, dev, stream, args, pk, pg, local, q, k, v, w):
                          "traffic": None, "algorithmic_bytes": alg_bytes}}
 
 
+def run_mixed(la, dev, stream, args, pk, pg, local):
+    """A serving batch in one launch (la_prefill_with_state): 4 prompts (lengths iid
+    U[1024, 5120], seed 6) and 2000 one-token continuations, each sequence with its own
+    carried-in fp32 state, H = 64, d = 128, B = 256. Beside it the same work in two calls:
+    la_prefill_with_state of the prompts, then la_decode_step of the continuations (whose
+    states are one contiguous batch). Algorithmic bytes: 8 d per token-head of Q, K, V, O,
+    plus the fp32 states, read (S0) and written (final state), 8 d^2 per (sequence, head)."""
+    import ctypes
+    H, d, B = 64, 128, 256
+    prompts = wl.varlen_lengths(4, 1024, 5120, seed=6)
+    n_cont = 2000
+    lengths = prompts + [1] * n_cont
+    T, nseq, Tp = sum(lengths), len(lengths), sum(prompts)
+    q, k, v = wl.qkv(T, H, d, torch.bfloat16, 6, device=dev)
+    o = torch.empty_like(q)
+    init = wl.state_init(nseq, H, d, seed=6, device=dev, scale=0.2)
+    st = torch.empty_like(init)
+    cu = wl.cu_seqlens(lengths, device=dev)
+    cu_p = wl.cu_seqlens(prompts, device=dev)
+    ws_bytes = max(la.la_prefill_with_state_workspace_size(T, nseq, H, d, B, la.LA_BF16),
+                   la.la_prefill_with_state_workspace_size(Tp, len(prompts), H, d, B, la.LA_BF16))
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    state_c = init[len(prompts):].clone()                    # the continuations' states, updated in place
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    def mixed():
+        s = la.la_prefill_with_state(P(q), P(k), P(v), P(o), P(cu), nseq, T, H, d, B, la.LA_BF16, P(init), P(st),
+                                     P(ws), ws_bytes, sh)
+        if s != 0:
+            raise RuntimeError(f"la_prefill_with_state (mixed batch) failed: {la.STATUS.get(s, s)}")
+
+    def split():
+        s = la.la_prefill_with_state(P(q), P(k), P(v), P(o), P(cu_p), len(prompts), Tp, H, d, B, la.LA_BF16,
+                                     P(init), P(st), P(ws), ws_bytes, sh)
+        if s != 0:
+            raise RuntimeError(f"la_prefill_with_state (prompts) failed: {la.STATUS.get(s, s)}")
+        s = la.la_decode_step(P(q[Tp:]), P(k[Tp:]), P(v[Tp:]), P(state_c), P(o[Tp:]), n_cont, H, d, la.LA_BF16, sh)
+        if s != 0:
+            raise RuntimeError(f"la_decode_step (continuations) failed: {la.STATUS.get(s, s)}")
+
+    n = 10
+    ms, kms, launches = _timed_calls(la, dev, stream, pg, local, mixed, n, max(3, args.warmup))
+    ms_split, _, launches_split = _timed_calls(la, dev, stream, pg, local, split, n, max(3, args.warmup))
+    del q, k, v, o, init, st, ws, state_c
+    alg_bytes = 8 * d * T * H + 8 * d * d * nseq * H
+    gbs = alg_bytes / (ms / 1e3) / 1e9
+    return {"workload": f"serving batch: prompts {prompts} + {n_cont} one-token continuations, H={H} d={d} B={B}, "
+                        "each sequence with its own fp32 state", "steps": n,
+            "ms_per_step": ms, "kernel_ms": kms, "launches_per_step": launches,
+            "split_ms_per_step": ms_split, "split_launches_per_step": launches_split,
+            "one_launch_over_split": ms / ms_split, "tokens_per_s": T / (ms / 1e3),
+            "roofline": {"bound": "hbm", "kernel": "prefill_chain_kernel (state-output instance)", "achieved": gbs,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes": alg_bytes}}
+
+
 # ---------------------------------------------------------------------------- reference arm
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -683,6 +747,7 @@ def main():
     ap.add_argument("--no-decay", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-mixed", action="store_true")
     ap.add_argument("--no-big", action="store_true", help="skip the million-token and varlen sub-measurements")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -50,7 +50,10 @@ struct Control {
     int32_t ok;          // 1 when cu_seqlens passed the device-side checks
     int32_t nslots;      // published-state slots used (single-pass prefill)
     int32_t abort;       // set by any CTA of the single-pass prefill whose bounded wait expired
-    int32_t pad[60];
+    int32_t nmulti;      // sequences of two or more tokens; the processing order lists them first
+    int32_t nsingle;     // one-token sequences, listed next (0 unless the order is sorted)
+    int32_t ticket;      // next one-token (sequence, head) of the prefill with final states
+    int32_t pad[57];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 

@@ -360,8 +360,7 @@ la_status launch_chain(const void* q, const void* k, const void* v, void* o, con
         const int64_t per_seq4 = (int64_t)heads * d * d / 4;
         const int sms = num_sms();
         if (sms <= 0) return LA_ERR_CUDA;
-        const int64_t want = ((int64_t)num_seqs * per_seq4 + 255) / 256;
-        la::empty_states_kernel<<<(unsigned)std::min<int64_t>(want, (int64_t)sms * 4), 256, 0, st>>>(
+        la::empty_states_kernel<<<(unsigned)std::min<int64_t>(num_seqs, (int64_t)sms * 8), 256, 0, st>>>(
             seqs, num_seqs, per_seq4, reinterpret_cast<const float4*>(init_state), reinterpret_cast<float4*>(state_out),
             ctrl);
         note_launch();
@@ -381,6 +380,7 @@ la_status launch_chain(const void* q, const void* k, const void* v, void* o, con
     prm.state_out = state_out;
     prm.k = static_cast<const __nv_bfloat16*>(k);
     prm.v = static_cast<const __nv_bfloat16*>(v);
+    prm.q = static_cast<const __nv_bfloat16*>(q);
     prm.H = heads;
     prm.B = B;
     prm.log2B = B == 256 ? 8 : 7;

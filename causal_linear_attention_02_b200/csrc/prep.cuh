@@ -144,9 +144,9 @@ __global__ void __launch_bounds__(1024) seq_table_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ order,
                                                          Control* __restrict__ ctrl) {
     __shared__ int32_t lens[kSortMax];
-    __shared__ int bad;
+    __shared__ int bad, nmulti, nsingle;
     const int tid = threadIdx.x;
-    if (tid == 0) bad = 0;
+    if (tid == 0) { bad = 0; nmulti = 0; nsingle = 0; }
     __syncthreads();
     if (cu != nullptr) {
         for (int s = tid; s < nseq; s += blockDim.x)
@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(1024) seq_table_kernel(const int32_t* __restri
         seqs[s] = e;
         if (sort) lens[s] = e.len;
         else order[s] = s;
+        if (e.len >= 2) atomicAdd(&nmulti, 1);
+        else if (e.len == 1) atomicAdd(&nsingle, 1);
     }
     __syncthreads();
     if (sort) {
@@ -190,6 +192,11 @@ __global__ void __launch_bounds__(1024) seq_table_kernel(const int32_t* __restri
         ctrl->ok = 1;
         ctrl->nslots = 0;
         ctrl->abort = 0;
+        // longest first puts the sequences of two or more tokens first and the one-token
+        // sequences right after them; unsorted, every sequence stays in the first group
+        ctrl->nmulti = sort ? nmulti : nseq;
+        ctrl->nsingle = sort ? nsingle : 0;
+        ctrl->ticket = 0;
     }
 }
 
@@ -250,17 +257,20 @@ __global__ void __launch_bounds__(256) chain_scan_kernel(const float* __restrict
 }
 
 // Final states of the empty sequences for la_prefill_with_state (the prefill
-// kernel visits only sequences with tokens): S0, or zero without one. One
-// 16-byte group per thread and iteration over [nseq][H][d][d]. Nothing when
-// the call's checks failed (ctrl->ok = 0).
+// kernel visits only sequences with tokens): S0, or zero without one. A CTA
+// takes one sequence at a time and copies its [H][d][d] state in 16-byte
+// groups; sequences with tokens cost one length read. Nothing when the call's
+// checks failed (ctrl->ok = 0).
 __global__ void __launch_bounds__(256)
 empty_states_kernel(const SeqEntry* seqs, int nseq, int64_t per_seq4, const float4* init, float4* out,
                     const Control* ctrl) {
     if (!ctrl->ok) return;
-    const int64_t total = (int64_t)nseq * per_seq4;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        if (seqs[i / per_seq4].len > 0) continue;
-        out[i] = init ? init[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    // a CTA per empty sequence at a time; sequences with tokens are skipped whole
+    for (int s = blockIdx.x; s < nseq; s += gridDim.x) {
+        if (seqs[s].len > 0) continue;
+        const int64_t base = (int64_t)s * per_seq4;
+        for (int64_t i = threadIdx.x; i < per_seq4; i += blockDim.x)
+            out[base + i] = init ? init[base + i] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 

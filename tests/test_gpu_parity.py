@@ -524,6 +524,57 @@ def test_prefill_with_state(lengths, H, B, dtype, with_init):
         assert torch.equal(o2, o)
 
 
+def _mixed_batch(seed, n_cont=500):
+    """A serving batch: four prompts of 257 to 3001 tokens, n_cont one-token continuations and two
+    empty sequences, shuffled together (the lengths in a seeded random order)."""
+    rng = np.random.default_rng(seed)
+    lengths = [3001, 1000, 1500, 257] + [1] * n_cont + [0, 0]
+    return [int(x) for x in rng.permutation(lengths)]
+
+
+@pytest.mark.parametrize("decay", [False, True], ids=["plain", "decay"])
+@pytest.mark.parametrize("in_place", [False, True], ids=["out", "in-place"])
+def test_prefill_with_state_mixed_batch(decay, in_place):
+    """One launch for a mixed batch on the on-chip-state kernel's state-output instance: the
+    prompts as chain work items, the one-token continuations as decode steps from their own
+    carried-in states (taken by the CTAs once their chain items are done). O of every token
+    and the final states of heads 0 and 31 against the oracle."""
+    lengths, H, d, B = _mixed_batch(5 + decay + 2 * in_place), 32, 128, 256
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, torch.bfloat16, seed=140 + decay)
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, d, seed=12, device=DEV, scale=0.2)
+    init64 = init[:, [0, H - 1]].cpu().double().numpy()
+    singles = [s for s, n in enumerate(lengths) if n == 1]
+    s0 = init[torch.tensor(singles, device=DEV)].cpu().double().numpy()   # before an in-place update
+    rates = wl.decay_rates(H, device=DEV) if decay else None
+    st = init if in_place else None
+    if decay:
+        o, st = la.prefill_decay(q, k, v, rates, cu, B=B, init_state=init, return_state=True,
+                                 state_out=st)
+    else:
+        o, st = la.prefill_with_state(q, k, v, cu, B=B, init_state=init, state_out=st)
+    status_ok()
+    cu_h = cu.cpu().numpy()
+    heads = [0, H - 1]
+    sel = lambda t: f64(t[:, heads])
+    if decay:
+        ref_o, ref_s = oracle.decay_recurrent(sel(q), sel(k), sel(v), rates.cpu().double().numpy()[heads], cu_h,
+                                              init=init64, return_state=True)
+    else:
+        ref_o, ref_s = oracle.recurrent(sel(q), sel(k), sel(v), cu_h, init=init64, return_state=True)
+    assert_close(sel(o), ref_o, 1e-2, "O of the sampled heads")
+    assert_close(st[:, heads].cpu().double().numpy(), ref_s, 5e-3 if decay else 1e-5, "final states")
+    # every head: the one-token rows against the decode step from their own state
+    rows = cu_h[singles]
+    q1, k1, v1 = (f64(x[rows]) for x in (q, k, v))
+    if decay:
+        ref1, _ = oracle.decay_decode_step(q1, k1, v1, s0, rates.cpu().double().numpy())
+    else:
+        ref1, _ = oracle.decode_step(q1, k1, v1, s0)
+    assert_close(f64(o[rows]), ref1, 1e-2, "O of the one-token sequences, every head")
+
+
 @pytest.mark.parametrize("B", [128, 256])
 def test_prefill_with_state_repeated(B):
     """The state-output instance of the on-chip-state kernel over many blocks, repeated: every call
