@@ -140,8 +140,29 @@ struct Bars {
     uint64_t drain, drain_b;
     uint32_t tmem_base;
     int abort_flag;
+    uint32_t peer_blocks;     // blocks whose Q and K loads the other CTA of the cluster has issued
 };
 static_assert(sizeof(Bars) <= 512, "barrier block");
+
+// The two CTAs of a cluster walk the two value halves of the same work items (items 2c + k G
+// and 2c + 1 + k G, G the even grid size), so they read the same Q and K tiles. A producer
+// issues block n's Q and K loads only while the other is at most kPeerLag blocks behind,
+// which keeps the second read of every tile in L2 over any number of blocks.
+constexpr uint32_t kPeerLag = 2;
+__device__ __forceinline__ uint32_t cluster_rank_of_cta() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Relaxed store to the same shared-memory variable of the other CTA of the pair.
+__device__ __forceinline__ void st_peer_u32(const void* local, uint32_t value) {
+    uint32_t a;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(cluster_rank_of_cta() ^ 1u));
+    asm volatile("st.shared::cluster.u32 [%0], %1;" :: "r"(a), "r"(value) : "memory");
+}
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 struct Params {
     __nv_bfloat16* out;
@@ -203,13 +224,16 @@ struct Blk { int w, seq, h, tok_s, len, b, tok0, rows, Rb, more; };
 // The block after `c` (the first block of the next work item with tokens,
 // from w + step on, after the last block of one); with `first`, the CTA's first
 // block. Out of line: every role's cursor shares this one copy.
-__device__ __noinline__ Blk next_blk(Blk c, bool first, int step, int nitems, const int32_t* order,
-                                     const SeqEntry* seqs, int H, int log2B) {
+// `nseq` counts the sequences walked; with `multi_only` (the prefill with final states)
+// the one-token sequences, listed after the others, are left to singles_phase.
+__device__ __noinline__ Blk next_blk(Blk c, bool first, int step, int nseq, bool multi_only, const Control* ctrl,
+                                     const int32_t* order, const SeqEntry* seqs, int H, int log2B) {
     const int bs = 1 << log2B;
     int nb = (c.len + bs - 1) >> log2B;
     if (!first && c.b + 1 < nb) {
         ++c.b;
     } else {
+        const int nitems = 2 * (multi_only ? ctrl->nmulti : nseq) * H;   // 2 nseq H < 2^31
         int w = first ? c.w : c.w + step;
         c.len = 0;
         for (; w < nitems; w += step) {
@@ -250,7 +274,6 @@ struct Cursor {
     int j, r;                            // its chunk and sub-unit
     uint32_t i;
     bool valid;
-    int nitems;                          // work items: 2 per (sequence, head) of the sequences walked
 
     __device__ __forceinline__ void set_item() {
         if (Rb == 2) {
@@ -262,7 +285,7 @@ struct Cursor {
         }
     }
     __device__ __forceinline__ void take(const Params& p, bool first) {
-        bk = next_blk(bk, first, gridDim.x, nitems, p.order, p.seqs, p.H, p.log2B);   // 2 nseq H < 2^31
+        bk = next_blk(bk, first, gridDim.x, p.nseq, p.state_out != nullptr, p.ctrl, p.order, p.seqs, p.H, p.log2B);
         valid = bk.len > 0;
         w = bk.w;
         seq = bk.seq;
@@ -279,8 +302,6 @@ struct Cursor {
     __device__ __forceinline__ void init(const Params& p) {
         n = q0 = kc0 = o0 = 0;
         i = 0;
-        // with final states, one-token sequences are left to the decode phase (singles_phase)
-        nitems = 2 * (p.state_out ? p.ctrl->nmulti : p.nseq) * p.H;
         bk.w = blockIdx.x;
         bk.len = 0;
         bk.b = 0;
@@ -575,7 +596,7 @@ __device__ __noinline__ void singles_phase(const Params& p, uint8_t* smem, const
 // product each rounded to bf16: relative 2^-8 per term). Rates are checked
 // before the launch (a bad rate leaves the launch with no work).
 template <bool kStateOut, bool kDecay>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
     using SM = Smem<kDecay>;
@@ -610,6 +631,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             for (int i = 0; i < SM::NVW; ++i) { mbar_init(&bars->vw_full[i], 128); mbar_init(&bars->vw_empty[i], 1); }
         }
         bars->abort_flag = 0;
+        bars->peer_blocks = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -620,7 +642,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         prefetch_tmap(&tmQ); prefetch_tmap(&tmK); prefetch_tmap(&tmV);
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_barrier();            // both CTAs' barriers and progress words exist before any remote store
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
@@ -639,9 +661,12 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             bool ok = true;
             uint32_t idle = 0;
             uint64_t t_idle = 0;
+            uint32_t published = 0;                          // blocks whose Q and K loads are all issued
+            const volatile uint32_t* peer = &bars->peer_blocks;
             while (cq.valid || ck.valid || cv.valid) {
                 bool prog = false;
-                if (cq.valid) {
+                const uint32_t lead = *peer + kPeerLag;      // highest block this CTA may load Q / K for
+                if (cq.valid && cq.n <= lead) {
                     const uint32_t qc = cq.q0 + rq;
                     if (mbar_test_wait(&bars->q_empty[qc % NQ], ((qc / NQ) & 1) ^ 1)) {
                         const int t = cq.tok0 + UM * rq;
@@ -655,7 +680,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         prog = true;
                     }
                 }
-                if (ck.valid) {
+                if (ck.valid && ck.n <= lead) {
                     const uint32_t kc = ck.kc0 + rk;
                     if (mbar_test_wait(&bars->k_empty[kc % NK], ((kc / NK) & 1) ^ 1)) {
                         const int t = ck.tok0 + KC * rk;
@@ -682,6 +707,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         prog = true;
                     }
                 }
+                // a cursor's block count stops at its total once the stream is done
+                if (min(cq.n, ck.n) != published) {
+                    published = min(cq.n, ck.n);
+                    st_peer_u32(&bars->peer_blocks, published);
+                }
                 if (prog) {
                     idle = 0;
                 } else if ((++idle & 63u) == 0) {
@@ -691,6 +721,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     else if (now - t_idle > ab.limit_ns) { ab.raise(); ok = false; break; }
                 }
             }
+            // let the other CTA run on freely from here (this CTA issues no more loads)
+            st_peer_u32(&bars->peer_blocks, 0x7fffffffu);
             // On abort, wait (bounded) for this producer's copies still in flight
             // into shared memory: only the latest load of each stage can be pending.
             if (!ok) {
@@ -1173,6 +1205,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     if constexpr (kStateOut) {
         if (p.ctrl->ok && !ab.raised()) singles_phase<kDecay>(p, smem, ab);
     }
+    cluster_barrier();            // no remote store reaches a CTA that has ended
 }
 
 }  // namespace chain

@@ -344,6 +344,32 @@ la_status launch_decay_check(const float* decay, int heads, uint8_t* ws, cudaStr
     return cuda_check();
 }
 
+// 2-CTA clusters of the on-chip-state kernel that fit on the device at once (cached per
+// device): the grid stays within them, so no cluster waits for another to finish.
+int chain_max_clusters() {
+    static std::mutex mu;
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int n = 0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(la::chain::NTHREADS, 1, 1);
+        cfg.dynamicSmemBytes = la::chain::Smem<true>::BYTES;   // the larger of the instances
+        cfg.gridDim = dim3(2 * 74, 1, 1);
+        if (cudaFuncSetAttribute(la::chain::prefill_chain_kernel<true, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cfg.dynamicSmemBytes) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, la::chain::prefill_chain_kernel<true, true>, &cfg) != cudaSuccess ||
+            n <= 0) {
+            cudaGetLastError();
+            n = num_sms() / 2;
+        }
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 la_status launch_chain(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens, int num_seqs,
                        int64_t total_tokens, int heads, int d, int B, const float* init_state, float* state_out,
                        uint8_t* ws, const Layout& L, cudaStream_t st, const float* decay = nullptr) {
@@ -388,10 +414,11 @@ la_status launch_chain(const void* q, const void* k, const void* v, void* o, con
     prm.wait_ns = t_wait_ns ? t_wait_ns : kWaitNs;
     prm.suppress_item = t_suppress_tile;
     prm.decay = decay;
+    // items come in (value half 0, value half 1) pairs: an even grid of 2-CTA clusters
     const int64_t items = 2 * (int64_t)num_seqs * heads;
-    const int sms = num_sms();
-    if (sms <= 0) return LA_ERR_CUDA;
-    const unsigned grid = (unsigned)(items < sms ? items : sms);
+    const int clusters = chain_max_clusters();
+    if (clusters <= 0) return LA_ERR_CUDA;
+    const unsigned grid = (unsigned)(items < 2 * (int64_t)clusters ? items : 2 * (int64_t)clusters);
     const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
     prm.trace = (t_trace && t_trace_bytes >= per_block) ? t_trace : nullptr;
     prm.trace_blocks = prm.trace ? (int)std::min<size_t>(t_trace_bytes / per_block, 1 << 30) : 0;

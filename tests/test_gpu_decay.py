@@ -92,9 +92,19 @@ def test_prefill_decay(dtype, d, B, lengths, H, with_init, path):
                                            return_state=True)
     assert_close(f64(o), ref_o, TOL[dtype], "decay prefill O")
     assert_close(st.cpu().double().numpy(), ref_st, STATE_TOL[path], "decay prefill final state")
-    # the state output is optional and changes nothing else
+    # the state output is optional and changes nothing else, except that on the on-chip-state
+    # kernel a one-token sequence with a state output is a decode step (fp32 on CUDA cores)
+    # rather than a block of the tensor-core pipeline: equal up to rounding there
     o2 = la.prefill_decay(q, k, v, decay, cu, B=B, init_state=init)
-    assert torch.equal(o2, o)
+    cu_h = cu.cpu().numpy()
+    one = np.zeros(T, dtype=bool)
+    for s_, n in enumerate(lengths):
+        if n == 1:
+            one[cu_h[s_]] = True
+    multi = torch.from_numpy(~one).to(DEV)
+    assert torch.equal(o2[multi], o[multi])
+    if one.any():
+        assert_close(f64(o2[~multi]), ref_o[one], TOL[dtype], "one-token rows without the state output")
 
 
 @pytest.mark.parametrize("lengths,H,B", [
