@@ -12,8 +12,8 @@
 // have it, and finds its exclusive prefix by walking back over its
 // predecessors' published inclusive prefixes or aggregates.
 //
-// One persistent CTA per SM, tiles t = (block g, head h), g-major, taken
-// round-robin (t = blockIdx.x, blockIdx.x + gridDim.x, ...). A tile is B
+// One persistent CTA per SM, tiles t = (block g, head h), g-major, taken by
+// atomic ticket in that order (see kTileRing). A tile is B
 // query rows processed as R = B/128 sub-units of 128 rows, last sub-unit
 // first (it streams every key chunk of the block and so computes U_b on the
 // way). Roles (512 threads, 128 registers each):
@@ -72,7 +72,8 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_KV = OFF_Q + NQ * Q_BYTES;
 constexpr uint32_t OFF_PRE = OFF_KV + NKV * 2 * KV_BYTES;
 constexpr uint32_t OFF_BAR = OFF_PRE + PRE_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 1024 + 1024;   // barriers and tile ring + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_U = 384, TM_COLS = 512;
 
@@ -82,6 +83,14 @@ constexpr uint32_t IDESC_QP = idesc_bf16(128, 128, false, true);
 constexpr uint32_t IDESC_KV = idesc_bf16(128, 128, true, true);
 
 constexpr int NTHREADS = 512;
+// Tiles are taken by atomic ticket in tile order (block-major, head fastest), so every
+// predecessor of a tile (same head, earlier block: a smaller ticket) belongs to a CTA that
+// was already running when this one drew it. Forward progress then never depends on CTAs
+// that are not resident (another stream's kernel may hold SMs). The producer draws each
+// tile when it first needs it, at most two ahead of the one it loads, and hands the
+// sequence to the other roles through a small ring; roles lag the producer by a few
+// tiles at most, far less than the ring holds.
+constexpr uint32_t kTileRing = 32;
 
 struct Bars {
     uint64_t q_full[NQ], q_empty[NQ];
@@ -98,8 +107,11 @@ struct Bars {
     uint64_t slot_ok;                     // publisher -> P group: this tile's ring slot may be written
     uint32_t tmem_base;
     int abort_flag;
+    int32_t tile_ring[kTileRing];         // the CTA's k-th tile at [k % kTileRing], drawn by the producer
+    int32_t tile_tag[kTileRing];          // k of the entry (a stale entry is an error, never used)
+    uint32_t drawn;                       // tiles drawn so far
 };
-static_assert(sizeof(Bars) <= 512, "barrier block");
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 struct Params {
     __nv_bfloat16* out;
@@ -225,6 +237,35 @@ __device__ __forceinline__ bool spin_flag(const int* flag, const Abort& ab) {
     }
 }
 
+// The CTA's k-th tile from the ring (ntiles when the tickets have run out). Blocking
+// (bounded) until the producer has drawn it; a ring entry of another k means a role fell
+// further behind than the ring holds: the launch gives up (LA_ERR_TIMEOUT) rather than
+// use it.
+__device__ __noinline__ bool ring_tile(Bars* bars, uint32_t k, int64_t ntiles, const Abort ab, int64_t& t) {
+    const volatile uint32_t* drawn = &bars->drawn;
+    if (*drawn <= k) {
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t it = 1; *drawn <= k; ++it) {
+            if ((it & 31u) == 0) {
+                if (ab.raised()) { *ab.cta = 1; return false; }
+                if (globaltimer_ns() - t0 > ab.limit_ns) { ab.raise(); return false; }
+            }
+        }
+    }
+    const volatile int32_t* ring = bars->tile_ring;
+    const volatile int32_t* tag = bars->tile_tag;
+    const int32_t v = ring[k % kTileRing];
+    if ((uint32_t)tag[k % kTileRing] != k) { ab.raise(); return false; }
+    t = v < ntiles ? (int64_t)v : ntiles;
+    return true;
+}
+// Non-blocking: -1 while the producer has not drawn tile k yet.
+__device__ __forceinline__ int64_t ring_peek(Bars* bars, uint32_t k, int64_t ntiles) {
+    if (*reinterpret_cast<const volatile uint32_t*>(&bars->drawn) <= k) return -1;
+    const int32_t v = reinterpret_cast<const volatile int32_t*>(bars->tile_ring)[k % kTileRing];
+    return v < ntiles ? (int64_t)v : ntiles;
+}
+
 // Ring-slot reuse: block b writes slot b % W, last used by block b - W, which
 // the look-backs of blocks b-W+1 .. b-W+L may read. With W = L + 2 the newest
 // of those is two blocks back, so the check (made by the publisher lane) never
@@ -262,6 +303,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars->incl_pub, 1);
         mbar_init(&bars->slot_ok, 1);
         bars->abort_flag = 0;
+        bars->drawn = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -318,20 +360,41 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     if (!load_chunk(y, j, keep)) return false;   // read again by the tile itself
                 return true;
             };
-            if (!load_lookahead(blockIdx.x)) ok = false;
-            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+            // draws the CTA's tiles 0..k (tile tickets, see kTileRing) and returns tile k
+            Control* ctrl_w = const_cast<Control*>(p.ctrl);
+            volatile uint32_t* drawn = &bars->drawn;
+            volatile int32_t* ring = bars->tile_ring;
+            volatile int32_t* tag = bars->tile_tag;
+            auto tile_k = [&](uint32_t k) -> int64_t {
+                while (*drawn <= k) {
+                    const uint32_t n = *drawn;
+                    const int v = atomicAdd(&ctrl_w->ticket, 1);
+                    ring[n % kTileRing] = v;
+                    tag[n % kTileRing] = (int32_t)n;
+                    __threadfence_block();
+                    *drawn = n + 1;
+                }
+                const int32_t v = ring[k % kTileRing];
+                return v < ntiles ? (int64_t)v : ntiles;
+            };
+            if (!load_lookahead(tile_k(0))) ok = false;
+            for (uint32_t k = 0; ok; ++k) {
+                const int64_t t = tile_k(k);
+                if (t >= ntiles) break;
                 const Tile x = tile_of(t, p);
-                if (t + gridDim.x < ntiles) {          // the next tile's Q into L2 a tile ahead
-                    const Tile y = tile_of(t + gridDim.x, p);
+                const int64_t t1 = tile_k(k + 1);
+                if (t1 < ntiles) {                     // the next tile's Q into L2 a tile ahead
+                    const Tile y = tile_of(t1, p);
                     for (int r = R - 1; r >= 0; --r) {
                         if (sub_rows(y, r) <= 0) continue;
                         tma_prefetch_l2_3d(&tmQ, 0, y.h, y.e.tok0 + UM * r);
                         tma_prefetch_l2_3d(&tmQ, 64, y.h, y.e.tok0 + UM * r);
                     }
                 }
-                if (LA_FUSED_KV_PREFETCH && t + 2 * (int64_t)gridDim.x < ntiles) {
+                const int64_t t2 = LA_FUSED_KV_PREFETCH ? tile_k(k + 2) : ntiles;
+                if (t2 < ntiles) {
                     // K / V of the tile after next into L2, ahead of its look-ahead loads
-                    const Tile y = tile_of(t + 2 * (int64_t)gridDim.x, p);
+                    const Tile y = tile_of(t2, p);
                     if (owns_state(y)) {
                         for (int j = 0; j < R * (UM / KC); ++j) {
                             const int tk = y.e.tok0 + KC * j;
@@ -342,7 +405,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         }
                     }
                 }
-                if (!load_lookahead(t + gridDim.x)) { ok = false; break; }
+                if (!load_lookahead(t1)) { ok = false; break; }
                 for (int r = R - 1; ok && r >= 0; --r) {
                     if (sub_rows(x, r) <= 0) continue;
                     const uint32_t qs = q_it % NQ;
@@ -407,10 +470,12 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 ++u_it;
                 return true;
             };
-            if (!lookahead_state(blockIdx.x)) ok = false;
-            for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+            int64_t tnext = ntiles;
+            if (!ring_tile(bars, 0, ntiles, ab, tnext) || !lookahead_state(tnext)) ok = false;
+            for (uint32_t k = 0; ok && tnext < ntiles; ++k) {
+                const int64_t t = tnext;
                 const Tile x = tile_of(t, p);
-                if (!lookahead_state(t + gridDim.x)) { ok = false; break; }
+                if (!ring_tile(bars, k + 1, ntiles, ab, tnext) || !lookahead_state(tnext)) { ok = false; break; }
                 uint32_t sub_q[2], sub_o[2];
                 int nsub = 0;
                 for (int r = R - 1; ok && r >= 0; --r) {
@@ -533,9 +598,13 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             ++u_it;
             return true;
         };
-        if (!store_aggregate(blockIdx.x)) ok = false;
-        for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+        int64_t tnext = ntiles;
+        ok = warp_all(ring_tile(bars, 0, ntiles, ab, tnext));
+        if (ok && !store_aggregate(tnext)) ok = false;
+        for (uint32_t k = 0; ok && tnext < ntiles; ++k) {
+            const int64_t t = tnext;
             const Tile x = tile_of(t, p);
+            if (!warp_all(ring_tile(bars, k + 1, ntiles, ab, tnext))) { ok = false; break; }
             for (int r = R - 1; ok && r >= 0; --r) {
                 if (sub_rows(x, r) <= 0) continue;
                 const int nkc = sub_chunks(x, r);
@@ -635,10 +704,10 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         bulk_commit();
                     }
                 }
-                if (r == R - 1 && ok && !store_aggregate(t + gridDim.x)) ok = false;
+                if (r == R - 1 && ok && !store_aggregate(tnext)) ok = false;
             }
             if (!ok) break;
-            if (sub_rows(x, R - 1) <= 0 && !store_aggregate(t + gridDim.x)) { ok = false; break; }
+            if (sub_rows(x, R - 1) <= 0 && !store_aggregate(tnext)) { ok = false; break; }
             // the staging buffer is free for the next prefix once these stores have read it
             if (wt == 0) {
                 bulk_wait_read0();
@@ -674,7 +743,10 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
             }
         };
-        for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+        for (uint32_t k = 0; ok; ++k) {
+            int64_t t = ntiles;
+            if (!warp_all(ring_tile(bars, k, ntiles, ab, t))) { ok = false; break; }
+            if (t >= ntiles) break;
             const Tile x = tile_of(t, p);
             const bool own = owns_state(x);
             float4 acc[16];
@@ -804,19 +876,26 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         //   lb / agg / incl: for each completed item the worker group's mbarrier
         //         arrive released its accesses at CTA scope; the release store below
         //         makes them visible at gpu scope together with the flag.
-        int64_t t_lb = blockIdx.x, t_ag = blockIdx.x, t_in = blockIdx.x, t_sl = blockIdx.x;
+        // Each stream is an index into the CTA's tile sequence; -1: not drawn yet (asked again).
+        uint32_t k_lb = 0, k_ag = 0, k_in = 0, k_sl = 0;
+        int64_t t_lb = -1, t_ag = -1, t_in = -1, t_sl = -1;
         uint32_t n_lb = 0, n_ag = 0, n_in = 0, n_sl = 0;
-        auto next_own = [&](int64_t t) {
-            while (t < ntiles && !owns_state(tile_of(t, p))) t += gridDim.x;
-            return t;
+        auto own_at = [&](uint32_t& k) -> int64_t {    // the first tile at index >= k with a state of its own
+            for (;;) {
+                const int64_t t = ring_peek(bars, k, ntiles);
+                if (t < 0 || t >= ntiles || owns_state(tile_of(t, p))) return t;
+                ++k;
+            }
         };
-        t_ag = next_own(t_ag);
-        t_in = next_own(t_in);
-        t_sl = next_own(t_sl);
         uint64_t t0 = globaltimer_ns();
-        while (t_lb < ntiles || t_ag < ntiles || t_in < ntiles) {
+        for (;;) {
+            if (t_lb < 0) t_lb = ring_peek(bars, k_lb, ntiles);
+            if (t_ag < 0) t_ag = own_at(k_ag);
+            if (t_in < 0) t_in = own_at(k_in);
+            if (t_sl < 0) t_sl = own_at(k_sl);
+            if (t_lb >= ntiles && t_ag >= ntiles && t_in >= ntiles) break;
             bool any = false;
-            if (t_sl < ntiles && n_sl <= n_ag) {
+            if (t_sl >= 0 && t_sl < ntiles && n_sl <= n_ag) {
                 const Tile x = tile_of(t_sl, p);
                 const int blk = x.e.blk;
                 int free = 1;
@@ -824,26 +903,26 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     free &= ld_acquire(p.lb_done + (int64_t)(x.g - (blk - c)) * p.H + x.h);
                 if (free) {
                     mbar_arrive(&bars->slot_ok);
-                    ++n_sl; t_sl = next_own(t_sl + gridDim.x); any = true;
+                    ++n_sl; ++k_sl; t_sl = -1; any = true;
                 }
             }
-            if (t_lb < ntiles && mbar_test_wait(&bars->lbd_st, n_lb & 1)) {
+            if (t_lb >= 0 && t_lb < ntiles && mbar_test_wait(&bars->lbd_st, n_lb & 1)) {
                 const Tile x = tile_of(t_lb, p);
                 st_release(p.lb_done + (int64_t)x.g * p.H + x.h, 1);
                 LA_TRACE(t_lb, TR_LB_END);
                 mbar_arrive(&bars->lbd_pub);
-                ++n_lb; t_lb += gridDim.x; any = true;
+                ++n_lb; ++k_lb; t_lb = -1; any = true;
             }
-            if (t_ag < ntiles && mbar_test_wait(&bars->agg_st[n_ag & 1], (n_ag >> 1) & 1)) {
+            if (t_ag >= 0 && t_ag < ntiles && mbar_test_wait(&bars->agg_st[n_ag & 1], (n_ag >> 1) & 1)) {
                 const Tile x = tile_of(t_ag, p);
                 LA_TRACE(t_ag, TR_PUB_AGG);
                 if (t_ag != p.suppress_tile) {
                     st_release(p.agg_flag + (int64_t)x.g * p.H + x.h, 1);
                     LA_TRACE(t_ag, TR_AGG);
                 }
-                ++n_ag; t_ag = next_own(t_ag + gridDim.x); any = true;
+                ++n_ag; ++k_ag; t_ag = -1; any = true;
             }
-            if (t_in < ntiles && mbar_test_wait(&bars->incl_st, n_in & 1)) {
+            if (t_in >= 0 && t_in < ntiles && mbar_test_wait(&bars->incl_st, n_in & 1)) {
                 const Tile x = tile_of(t_in, p);
                 LA_TRACE(t_in, TR_PUB_INCL);
                 if (t_in != p.suppress_tile) {
@@ -851,7 +930,7 @@ prefill_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     LA_TRACE(t_in, TR_INCL);
                 }
                 mbar_arrive(&bars->incl_pub);
-                ++n_in; t_in = next_own(t_in + gridDim.x); any = true;
+                ++n_in; ++k_in; t_in = -1; any = true;
             }
             if (any) {
                 t0 = globaltimer_ns();

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(1024) seq_blocks_kernel(const int32_t* __restr
         ctrl->ok = 1;
         ctrl->nslots = carry_s;
         ctrl->abort = 0;
+        ctrl->ticket = 0;       // the single-pass prefill's tile tickets
     }
 }
 

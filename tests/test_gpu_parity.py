@@ -146,6 +146,33 @@ def test_prefill_fp32_integer_exact():
     assert mism == 0, f"{mism} of {ref.size} fp32 outputs differ from the exact result"
 
 
+def test_lookback_finishes_beside_another_kernel():
+    """The block-parallel kernel (forced) while another stream's matmul loop holds SMs for about
+    a second, with the device wait limit cut to 300 ms: its CTAs take tiles by ticket, so a tile's
+    predecessors always belong to CTAs that are already running, and the call ends with LA_OK and
+    the oracle's result (it never waits on a CTA that is not resident)."""
+    T, H, d, B = 12000, 2, 128, 256               # 47 blocks x 2 heads = 94 tiles
+    q, k, v = inputs(T, H, d, torch.bfloat16, seed=77)
+    ref = oracle.recurrent(f64(q), f64(k), f64(v))
+    a = torch.randn(8192, 8192, device=DEV, dtype=torch.bfloat16)
+    side = torch.cuda.Stream(DEV)
+    torch.cuda.synchronize(DEV)
+    assert la.la_debug_set_fault(-1, 300_000_000) == 0
+    force_path(2)
+    try:
+        with torch.cuda.stream(side):
+            for _ in range(1200):                 # about a second of 8192^3 bf16 products
+                c = a @ a
+        o = la.prefill(q, k, v, B=B)              # the current stream, beside them
+        torch.cuda.synchronize(DEV)
+    finally:
+        la.la_debug_set_fault(-1, 0)
+        force_path(0)
+    del c
+    status_ok()
+    assert_close(f64(o), ref, 1e-2, "block-parallel prefill beside another kernel")
+
+
 @pytest.mark.parametrize("B", [128, 256])
 def test_prefill_tc_varlen(B, tc_path):
     lengths = [1, 255, 256, 0, 257, 700, 64, 513, 128]
