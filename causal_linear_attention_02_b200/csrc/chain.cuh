@@ -219,19 +219,23 @@ enum TraceEvent {
 // token tok_s and length len) and, within it, block b with its first token,
 // rows, sub-units Rb and whether its K^T V is needed by a later block (more).
 // len = 0: no block left.
-struct Blk { int w, seq, h, tok_s, len, b, tok0, rows, Rb, more; };
+// first: the item's first block in walking order (block 0, or the last block when
+// walking backwards).
+struct Blk { int w, seq, h, tok_s, len, b, tok0, rows, Rb, more, first; };
 
 // The block after `c` (the first block of the next work item with tokens,
 // from w + step on, after the last block of one); with `first`, the CTA's first
 // block. Out of line: every role's cursor shares this one copy.
 // `nseq` counts the sequences walked; with `multi_only` (the prefill with final states)
-// the one-token sequences, listed after the others, are left to singles_phase.
-__device__ __noinline__ Blk next_blk(Blk c, bool first, int step, int nseq, bool multi_only, const Control* ctrl,
-                                     const int32_t* order, const SeqEntry* seqs, int H, int log2B) {
+// the one-token sequences, listed after the others, are left to singles_phase. With
+// `rev` (the anti-causal instance) an item's blocks are walked from the last to the first.
+__device__ __noinline__ Blk next_blk(Blk c, bool first, int step, int nseq, bool multi_only, bool rev,
+                                     const Control* ctrl, const int32_t* order, const SeqEntry* seqs, int H,
+                                     int log2B) {
     const int bs = 1 << log2B;
     int nb = (c.len + bs - 1) >> log2B;
-    if (!first && c.b + 1 < nb) {
-        ++c.b;
+    if (!first && (rev ? c.b > 0 : c.b + 1 < nb)) {
+        c.b += rev ? -1 : 1;
     } else {
         const int nitems = 2 * (multi_only ? ctrl->nmulti : nseq) * H;   // 2 nseq H < 2^31
         int w = first ? c.w : c.w + step;
@@ -249,13 +253,14 @@ __device__ __noinline__ Blk next_blk(Blk c, bool first, int step, int nseq, bool
             }
         }
         c.w = w;
-        c.b = 0;
         nb = (c.len + bs - 1) >> log2B;
+        c.b = rev && nb > 0 ? nb - 1 : 0;
     }
     c.tok0 = c.tok_s + (c.b << log2B);
     c.rows = min(bs, c.len - (c.b << log2B));
     c.Rb = (c.rows + UM - 1) / UM;
-    c.more = c.b + 1 < nb;
+    c.more = rev ? c.b > 0 : c.b + 1 < nb;
+    c.first = rev ? c.b == nb - 1 : c.b == 0;
     return c;
 }
 
@@ -265,7 +270,9 @@ __device__ __noinline__ Blk next_blk(Blk c, bool first, int step, int nseq, bool
 // and i (items). A block has Rb = ceil(rows / 128) sub-units and as many
 // 128-key chunks; its items are (0,0), (0,1), (1,1) when Rb = 2 and (0,0)
 // when Rb = 1.
-struct Cursor {
+// kRev (the anti-causal instance): blocks walked backwards, items (0,0), (1,0), (1,1).
+template <bool kRev>
+struct CursorT {
     Blk bk;
     int w, seq, h, half, tok0, rows, Rb, b;
     bool add_state;                      // the block's K^T V is needed (not the last block)
@@ -277,15 +284,16 @@ struct Cursor {
 
     __device__ __forceinline__ void set_item() {
         if (Rb == 2) {
-            j = k == 2 ? 1 : 0;
-            r = k == 0 ? 0 : 1;
+            j = kRev ? (k == 0 ? 0 : 1) : (k == 2 ? 1 : 0);
+            r = kRev ? (k == 2 ? 1 : 0) : (k == 0 ? 0 : 1);
         } else {
             j = 0;
             r = 0;
         }
     }
     __device__ __forceinline__ void take(const Params& p, bool first) {
-        bk = next_blk(bk, first, gridDim.x, p.nseq, p.state_out != nullptr, p.ctrl, p.order, p.seqs, p.H, p.log2B);
+        bk = next_blk(bk, first, gridDim.x, p.nseq, p.state_out != nullptr, kRev, p.ctrl, p.order, p.seqs, p.H,
+                      p.log2B);
         valid = bk.len > 0;
         w = bk.w;
         seq = bk.seq;
@@ -323,11 +331,11 @@ struct Cursor {
         }
         next_block(p);
     }
-    // item properties
-    __device__ __forceinline__ bool first_of_chunk() const { return k != 1; }     // (0,0), (1,1)
-    __device__ __forceinline__ bool last_of_chunk() const { return k != 0 || Rb == 1; }   // (0,1), (1,1)
-    __device__ __forceinline__ bool first_of_sub() const { return j == 0; }       // (0,0), (0,1)
-    __device__ __forceinline__ bool last_of_sub() const { return k != 1 || Rb == 1; }     // (0,0), (1,1)
+    // item properties (forward: (0,0), (0,1), (1,1); anti-causal: (0,0), (1,0), (1,1))
+    __device__ __forceinline__ bool first_of_chunk() const { return k != (kRev ? 2 : 1); }
+    __device__ __forceinline__ bool last_of_chunk() const { return k != (kRev ? 1 : 0) || Rb == 1; }
+    __device__ __forceinline__ bool first_of_sub() const { return kRev ? k != 1 : j == 0; }
+    __device__ __forceinline__ bool last_of_sub() const { return k != (kRev ? 0 : 1) || Rb == 1; }
     __device__ __forceinline__ bool last_of_block() const { return k == (Rb == 2 ? 2 : 0); }
     // O slot of sub-unit rr: the sub-unit that finishes last alternates between
     // slots 1 and 2 from block to block; sub-unit 0 of a two-sub-unit block
@@ -335,6 +343,7 @@ struct Cursor {
     __device__ __forceinline__ uint32_t oslot(int rr) const { return rr == Rb - 1 ? 1 + (n & 1) : 0; }
     __device__ __forceinline__ uint32_t ouse(int rr) const { return rr == Rb - 1 ? (n >> 1) : o0; }
 };
+using Cursor = CursorT<false>;
 
 // Decay instance: the weighted copy lambda^(rows-1-c) v_c (c the key in the block, zero past the
 // block's end) of every V chunk of the cursor's block, the B operand of its state MMAs, written by
@@ -595,11 +604,19 @@ __device__ __noinline__ void singles_phase(const Params& p, uint8_t* smem, const
 // The weighted V and the scaled Q rows are packed bf16 products (weight and
 // product each rounded to bf16: relative 2^-8 per term). Rates are checked
 // before the launch (a bad rate leaves the launch with no work).
-template <bool kStateOut, bool kDecay>
+// kRev: the anti-causal instance (no state output, no decay), O_t = q_t S0 + sum_{s >= t,
+// same sequence} (q_t . k_s) v_s: blocks walked from each sequence's end, the mask keeping
+// keys at or after the query row, and the running state the suffix of the blocks walked.
+// If the first block walked (the sequence's last) is ragged, its state is added on CUDA
+// cores by the copy-out group at the next block (the rows past the sequence end belong to
+// the next sequence, so no MMA may take them); its own state MMAs are skipped.
+template <bool kStateOut, bool kDecay, bool kRev = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
+    static_assert(!kRev || (!kStateOut && !kDecay), "the anti-causal instance has neither state output nor decay");
     using SM = Smem<kDecay>;
+    using Cursor = CursorT<kRev>;
     constexpr int NK = SM::NK, NV = SM::NV;
     constexpr uint32_t OFF_Q = SM::OFF_Q, OFF_K = SM::OFF_K, OFF_V = SM::OFF_V, OFF_SB = SM::OFF_SB,
                        OFF_BAR = SM::OFF_BAR;
@@ -794,12 +811,15 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         // the state MMAs of a block wait for the copy-out group to have read the
                         // prefix (and, with decay, rescaled it) whenever they run: in the
                         // state-output instance also on a sequence's last block
-                        if (ready && (dc.add_state || kStateOut) && dc.j == 0 && kvr_blk != dc.n) {
+                        // the anti-causal instance's ragged first block: state added on CUDA cores
+                        const bool run = (dc.add_state || kStateOut) &&
+                                         !(kRev && dc.bk.first && dc.rows < (1 << p.log2B));
+                        if (ready && run && dc.j == 0 && kvr_blk != dc.n) {
                             if (mbar_test_wait(&bars->kv_read[dc.n & 3], (dc.n >> 2) & 1)) kvr_blk = dc.n;
                             else ready = false;
                         }
                         if (ready) {
-                            if (dc.add_state || kStateOut) {
+                            if (run) {
                                 tc_fence_after();
                                 const uint64_t a = dkt + (((kc % NK) * K_BYTES) >> 4),
                                                b = kDecay ? dvs + (((kc % SM::NVW) * V_BYTES) >> 4)
@@ -812,7 +832,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                                 for (int s = 0; s < KC / 16; ++s)
                                     if (s < nsteps)
                                         mma_ss(tmem + TM_KV, a + ((s * 2048) >> 4), b + ((s * 2048) >> 4), IDESC_KV,
-                                               (dc.b > 0 || dc.j > 0 || s > 0 || p.init != nullptr));
+                                               (!dc.bk.first || dc.j > 0 || s > 0 || p.init != nullptr));
                                 if (dc.j == dc.Rb - 1) {
                                     tc_commit(&bars->kv_ready);
                                     LA_CTRACE(dc.n, TR_KVR);
@@ -939,6 +959,15 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         f = c0 <= lim ? f * lam : f;
                         pk[16 * hh + q] = pack_bf16x2(x0, x1);
                     }
+                } else if constexpr (kRev) {
+                    // keys at or after the query row (col >= lim) and inside the sequence (col < hi)
+                    const int hi = c.rows - KC * c.j - 64 * hk;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int c0 = 32 * hh + 2 * q;
+                        pk[16 * hh + q] = pack_bf16x2(c0 >= lim && c0 < hi ? __uint_as_float(a[2 * q]) : 0.f,
+                                                      c0 + 1 >= lim && c0 + 1 < hi ? __uint_as_float(a[2 * q + 1]) : 0.f);
+                    }
                 } else {
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
@@ -1044,7 +1073,53 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             } else {
             // KV_b -> bf16 operand of the inter-block product (row m, 64 columns)
             uint32_t pk[32];
-            if (c.b > 0) {
+            // anti-causal: the block walked after a ragged first block (the sequence's last)
+            // takes that block's state on CUDA cores instead of from its (skipped) MMAs
+            const int nbk = (c.bk.len + (1 << p.log2B) - 1) >> p.log2B;
+            if (kRev && !c.bk.first && c.b == nbk - 2 && (c.bk.len & ((1 << p.log2B) - 1)) != 0) {
+                float x[DV];
+                if (p.init) {                              // S0, seeded at the first block
+                    tc_fence_after();
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t a[32];
+                        tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) x[32 * hh + q] = __uint_as_float(a[q]);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < DV; ++q) x[q] = 0.f;
+                }
+                for (int t = c.bk.tok_s + ((nbk - 1) << p.log2B); t < c.bk.tok_s + c.bk.len; ++t) {
+                    const float ki = __bfloat162float(p.k[((int64_t)t * p.H + c.h) * D + m]);
+                    const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + c.h) * D + DV * c.half);
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const uint4 u = __ldg(vr + g);
+                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            x[8 * g + 2 * e] = fmaf(ki, __uint_as_float(w4[e] << 16), x[8 * g + 2 * e]);
+                            x[8 * g + 2 * e + 1] = fmaf(ki, __uint_as_float(w4[e] & 0xffff0000u), x[8 * g + 2 * e + 1]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a[32];
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(x[32 * hh + q]);
+                    tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);   // the later blocks' MMAs add onto it
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        pk[16 * hh + q] = pack_bf16x2(x[32 * hh + 2 * q], x[32 * hh + 2 * q + 1]);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars->kv_read[c.n & 3]);            // the accumulator may take this block's keys
+            } else if (!c.bk.first) {
                 if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
                 ++kvc;
                 if (wt == 0) LA_CTRACE(c.n, TR_XR);

@@ -370,9 +370,11 @@ int chain_max_clusters() {
     return cached[dev];
 }
 
+// rev: the anti-causal instance (O_t = q_t S0 + sum_{s >= t} (q_t . k_s) v_s; no state output,
+// no decay), which the backward pass uses for dk and dv.
 la_status launch_chain(const void* q, const void* k, const void* v, void* o, const int32_t* cu_seqlens, int num_seqs,
                        int64_t total_tokens, int heads, int d, int B, const float* init_state, float* state_out,
-                       uint8_t* ws, const Layout& L, cudaStream_t st, const float* decay = nullptr) {
+                       uint8_t* ws, const Layout& L, cudaStream_t st, const float* decay = nullptr, bool rev = false) {
     la_status s;
     const Control* ctrl = reinterpret_cast<const Control*>(ws);
     la::SeqEntry* seqs = reinterpret_cast<la::SeqEntry*>(ws + L.off_seqs);
@@ -422,7 +424,9 @@ la_status launch_chain(const void* q, const void* k, const void* v, void* o, con
     const size_t per_block = (size_t)grid * la::chain::kTraceEvents * sizeof(uint64_t);
     prm.trace = (t_trace && t_trace_bytes >= per_block) ? t_trace : nullptr;
     prm.trace_blocks = prm.trace ? (int)std::min<size_t>(t_trace_bytes / per_block, 1 << 30) : 0;
-    auto kernel = decay ? (state_out ? la::chain::prefill_chain_kernel<true, true>
+    if (rev && (decay || state_out)) return LA_ERR_UNSUPPORTED;
+    auto kernel = rev ? la::chain::prefill_chain_kernel<false, false, true>
+                : decay ? (state_out ? la::chain::prefill_chain_kernel<true, true>
                                      : la::chain::prefill_chain_kernel<false, true>)
                         : (state_out ? la::chain::prefill_chain_kernel<true, false>
                                      : la::chain::prefill_chain_kernel<false, false>);
@@ -442,10 +446,16 @@ struct BackwardLayout {
            pws = 0, off_sws = 0, sws = 0, total = 0;
 };
 Layout simt_layout(int64_t T, int nseq, int H, int d, int B);
+// dk and dv by the anti-causal instance of the on-chip-state kernel (no sequence
+// reversals) wherever the forward prefill takes that kernel, without decay.
+bool backward_in_place_order(la_dtype dt, int d, int B, int nseq, int H, bool decay) {
+    return !decay && prefill_path(dt, d, B, nseq, H) == Path::chain;
+}
 BackwardLayout backward_layout(int64_t T, int nseq, int H, int d, int B, la_dtype dt, bool decay = false) {
     BackwardLayout L;
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-    L.tensor = (size_t)T * H * d * esize(dt);
+    // the reversed copies are needed only when dk and dv come from prefills of reversed sequences
+    L.tensor = backward_in_place_order(dt, d, B, nseq, H, decay) ? 0 : (size_t)T * H * d * esize(dt);
     size_t off = 0;
     L.off_rk = off; off = up(off + L.tensor);
     L.off_rq = off; off = up(off + L.tensor);
@@ -875,6 +885,17 @@ static la_status prefill_backward_impl(const void* q, const void* k, const void*
                      : la_prefill(a, b, c, out, cu_seqlens, num_seqs, T, heads, d, B, dtype, init, pws, L.pws, stream);
     };
     if ((s = fwd(dout, v, k, dq, init_state ? s0t : nullptr)) != LA_OK) return s;
+    if (backward_in_place_order(dtype, d, B, num_seqs, heads, decay != nullptr)) {
+        // dV_s = sum_{t >= s} (k_s . q_t) dO_t and dK_s = sum_{t >= s} (v_s . dO_t) q_t: the
+        // anti-causal prefills of (K, Q, dO) and (V, dO, Q), in the tensors' own order
+        const Layout PL = prefill_layout(T, num_seqs, heads, d, B, dtype);
+        uint8_t* pw = static_cast<uint8_t*>(pws);
+        if ((s = launch_chain(k, q, dout, dv, cu_seqlens, num_seqs, T, heads, d, B, nullptr, nullptr, pw, PL, st,
+                              nullptr, true)) != LA_OK ||
+            (s = launch_chain(v, dout, q, dk, cu_seqlens, num_seqs, T, heads, d, B, nullptr, nullptr, pw, PL, st,
+                              nullptr, true)) != LA_OK)
+            return s;
+    } else {
     // dV and dK: forward prefills over the reversed sequences, reversed back
     if ((s = launch_reverse(k, rk, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
         (s = launch_reverse(q, rq, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK ||
@@ -887,6 +908,7 @@ static la_status prefill_backward_impl(const void* q, const void* k, const void*
     if ((s = fwd(rv, rdo, rq, rout, nullptr)) != LA_OK ||
         (s = launch_reverse(rout, dk, cu_seqlens, num_seqs, T, heads, d, dtype, st)) != LA_OK)
         return s;
+    }
     if (!dinit_state) return LA_OK;
     if (!decay)   // dS0 = state of (Q, dO)
         return la_state_from_prefill(q, dout, cu_seqlens, num_seqs, T, heads, d, dtype, nullptr, dinit_state,

@@ -477,6 +477,27 @@ def test_prefill_backward(dtype, d, B, with_init, tc_path):
     assert_close(dinit.cpu().double().numpy(), ref[3], 1e-5, "dS0")
 
 
+def test_prefill_backward_default_path_many_heads():
+    """32 heads: the automatic path is the on-chip-state kernel, so dk and dv come from its
+    anti-causal instance (blocks walked from each sequence's end, ragged last blocks with 188,
+    16 and 0 extra rows, a one-token sequence) with no sequence reversal; against the oracle."""
+    lengths, H, d, B = [700, 1, 1296, 256, 40], 32, 128, 256
+    T = sum(lengths)
+    q, k, v = inputs(T, H, d, torch.bfloat16, seed=83)
+    dout = wl.normal_scaled((T, H, d), d, torch.bfloat16, 84, device=DEV)
+    cu = cu_of(lengths)
+    init = wl.state_init(len(lengths), H, d, seed=9, device=DEV)
+    dq, dk, dv, dinit = la.prefill_backward(q, k, v, dout, cu, B=B, init_state=init, need_init_grad=True)
+    status_ok()
+    heads = [0, 17, 31]
+    sel = lambda t: f64(t[:, heads])
+    ref = oracle.backward(sel(q), sel(k), sel(v), sel(dout), cu.cpu().numpy(),
+                          init=init[:, heads].cpu().double().numpy())
+    for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
+        assert_close(sel(got), want, TOL[torch.bfloat16], name)
+    assert_close(dinit[:, heads].cpu().double().numpy(), ref[3], 1e-5, "dS0")
+
+
 @pytest.mark.gpu
 def test_prefill_backward_arguments():
     T, H, d, B = 300, 2, 128, 256
