@@ -7,10 +7,25 @@ tokens, H = 64 heads, d = 128, B = 256, Q, K, V iid N(0,1) * d^-1/2 in bf16
 (inputs 1.6 GB > L2, so nothing is flushed between steps). Rank 0 prints one
 JSON line with tokens/s (whole job), TFLOP/s counted as 4*B*d + 4*d^2 per
 token per head, the roofline of the main kernel (timed live with CUDA events
-on its stream via la_set_kernel_timer), the decode step of the batched decode
-workload (256 sequences x 64 heads, 128x128 fp32 states) as a sub-measurement,
-an end-to-end number through host buffers, SM clocks sampled during the timed
-region and the fp64 CPU oracle timed on a bounded sample on the host cores.
+on its stream via la_set_kernel_timer), an end-to-end number through host
+buffers, SM clocks sampled during the timed region and the fp64 CPU oracle
+timed on a bounded sample on the host cores. Sub-measurements of the same line,
+each timed with CUDA events on its own stream after warm-up calls:
+
+  decode    the batched decode workload (256 sequences x 64 heads, 128x128
+            fp32 states, 1000 steps), GB/s against HBM; decode.decay the same
+            with a decay rate per head
+  decay     the prefill with a decay rate per head on the 32k inputs
+  long      the million-token prefill (T = 1,048,576, H = 64), roofline and
+            DRAM traffic of its launch
+  varlen    the packed prefill of 16 sequences of U[1024, 65536] tokens
+  backward  la_prefill_backward on the 32k inputs (dq, dk, dv, dS0)
+  mixed     one la_prefill_with_state launch over 4 prompts and 2000
+            one-token continuations, beside the split form (prompts through
+            la_prefill_with_state, the continuations through la_decode_step)
+
+--no-decode, --no-decay, --no-big (long, varlen), --no-backward, --no-mixed and
+--no-cpu-baseline leave a sub-measurement out.
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own
 independent prefill of the same size (weak scaling, no collective on the data
@@ -98,7 +113,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
-    def __init__(self, device, period_s=0.0005):
+    def __init__(self, device, period_s=0.002):
         self.device = device
         self.period = period_s
         self.samples = []
@@ -446,11 +461,12 @@ def run_decode(la, dev, stream, args, pk, pg, local):
     torch.cuda.synchronize(dev)
     barrier(pg, local)
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for i in range(n_steps):
-        step(i, timers[i])
-    a1.record(stream)
-    torch.cuda.synchronize(dev)
+    with ClockSampler(dev, period_s=0.002) as clocks:
+        a0.record(stream)
+        for i in range(n_steps):
+            step(i, timers[i])
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
     barrier(pg, local)
     ms = max_over_ranks(pg, a0.elapsed_time(a1)) / n_steps
     kms = max_over_ranks(pg, statistics.mean(a.elapsed_time(b) for a, b in timers))
@@ -479,7 +495,7 @@ def run_decode(la, dev, stream, args, pk, pg, local):
     dgbs = (state_bytes + io_bytes) / (dkms / 1e3) / 1e9
     return {"workload": w.name, "steps": n_steps, "ms_per_step": ms, "kernel_ms": kms,
             "value": gbs, "unit": "GB/s", "hbm_frac": gbs / pk["hbm_gbs"],
-            "tokens_per_s": Bt / (ms / 1e3),
+            "tokens_per_s": Bt / (ms / 1e3), "clocks": clocks.summary(),
             "decay": {"kernel_ms": dkms, "value": dgbs, "unit": "GB/s", "hbm_frac": dgbs / pk["hbm_gbs"]},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": captured_traffic("decode_step_kernel"),
@@ -516,12 +532,13 @@ def run_decay(la, dev, stream, args, pk, pg, local, q, k, v, o, w):
     barrier(pg, local)
     launches0 = la.la_launch_count()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for i in range(n):
-        step(timers[i])
-    a1.record(stream)
-    launches = la.la_launch_count() - launches0
-    torch.cuda.synchronize(dev)
+    with ClockSampler(dev, period_s=0.002) as clocks:
+        a0.record(stream)
+        for i in range(n):
+            step(timers[i])
+        a1.record(stream)
+        launches = la.la_launch_count() - launches0
+        torch.cuda.synchronize(dev)
     barrier(pg, local)
     ms = max_over_ranks(pg, a0.elapsed_time(a1)) / n
     kms = max_over_ranks(pg, statistics.mean(a.elapsed_time(b) for a, b in timers))
@@ -535,6 +552,7 @@ def run_decay(la, dev, stream, args, pk, pg, local, q, k, v, o, w):
             "rates": "lambda_h = exp(-2^(-8 (h+1) / H)), 0.40 .. 0.996",
             "steps": n, "ms_per_step": ms, "kernel_ms": kms, "tokens_per_s": T / (ms / 1e3),
             "tflops": tflops, "tc_peak_frac": tflops / pk["bf16_tflops"], "launches_per_step": launches / n,
+            "clocks": clocks.summary(),
             "roofline": {"bound": "hbm", "kernel": "prefill_chain_kernel (decay instance)", "achieved": gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                          "traffic": captured_traffic("prefill_chain_kernel_decay"),
@@ -543,7 +561,8 @@ def run_decay(la, dev, stream, args, pk, pg, local, q, k, v, o, w):
 
 def _timed_calls(la, dev, stream, pg, local, call, n, warmup):
     """n timed calls after `warmup` untimed ones: (ms per call from events around all
-    calls, mean main-kernel ms from la_set_kernel_timer, launches per call)."""
+    calls, mean main-kernel ms from la_set_kernel_timer, launches per call, SM clocks
+    sampled during the timed calls)."""
     import ctypes
     for _ in range(warmup):
         call()
@@ -554,19 +573,20 @@ def _timed_calls(la, dev, stream, pg, local, call, n, warmup):
     barrier(pg, local)
     launches0 = la.la_launch_count()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for i in range(n):
-        la.la_set_kernel_timer(ctypes.c_void_p(timers[i][0].cuda_event), ctypes.c_void_p(timers[i][1].cuda_event))
-        call()
-    a1.record(stream)
-    launches = la.la_launch_count() - launches0
-    torch.cuda.synchronize(dev)
+    with ClockSampler(dev, period_s=0.002) as clocks:
+        a0.record(stream)
+        for i in range(n):
+            la.la_set_kernel_timer(ctypes.c_void_p(timers[i][0].cuda_event), ctypes.c_void_p(timers[i][1].cuda_event))
+            call()
+        a1.record(stream)
+        launches = la.la_launch_count() - launches0
+        torch.cuda.synchronize(dev)
     barrier(pg, local)
     ms = max_over_ranks(pg, a0.elapsed_time(a1)) / n
     kms = max_over_ranks(pg, statistics.mean(a.elapsed_time(b) for a, b in timers))
     if la.device_status() != 0:
         raise RuntimeError("device status after a timed sub-measurement")
-    return ms, kms, launches / n
+    return ms, kms, launches / n, clocks.summary()
 
 
 def run_prefill_workload(la, dev, stream, args, pk, pg, local, w, key):
@@ -590,7 +610,7 @@ def run_prefill_workload(la, dev, stream, args, pk, pg, local, w, key):
             raise RuntimeError(f"la_prefill ({key}) failed: {la.STATUS.get(s, s)}")
 
     n = 5 if T > 300000 else 10
-    ms, kms, launches = _timed_calls(la, dev, stream, pg, local, call, n, max(3, args.warmup))
+    ms, kms, launches, clk = _timed_calls(la, dev, stream, pg, local, call, n, max(3, args.warmup))
     del q, k, v, o, ws
     alg_bytes = 8 * d * T * H
     gbs = alg_bytes / (kms / 1e3) / 1e9
@@ -598,7 +618,7 @@ def run_prefill_workload(la, dev, stream, args, pk, pg, local, w, key):
     return {"workload": w.name, "tokens": T, "sequences": nseq, "seed": w.seed, "steps": n,
             "ms_per_step": ms, "kernel_ms": kms, "tokens_per_s": T / (ms / 1e3), "tflops": tflops,
             "tc_peak_frac": tflops / pk["bf16_tflops"], "launches_per_step": launches,
-            "l2": "no flush: inputs far larger than the 126 MB L2",
+            "l2": "no flush: inputs far larger than the 126 MB L2", "clocks": clk,
             "roofline": {"bound": "hbm", "kernel": "prefill_chain_kernel", "achieved": gbs, "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                          "traffic": captured_traffic("prefill_chain_kernel_" + ("1m" if key == "long" else key)),
@@ -626,14 +646,14 @@ def run_backward(la, dev, stream, args, pk, pg, local, q, k, v, w):
             raise RuntimeError(f"la_prefill_backward failed: {la.STATUS.get(s, s)}")
 
     n = 10
-    ms, _, launches = _timed_calls(la, dev, stream, pg, local, call, n, max(3, args.warmup))
+    ms, _, launches, clk = _timed_calls(la, dev, stream, pg, local, call, n, max(3, args.warmup))
     del do, dq, dk, dv, ws
     alg_bytes = 14 * d * T * H
     gbs = alg_bytes / (ms / 1e3) / 1e9
     tflops = 3 * flops_per_token_head(B, d) * T * H / (ms / 1e3) / 1e12
     return {"workload": f"backward of the {w.name} prefill (dq, dk, dv)", "steps": n, "ms_per_step": ms,
             "tokens_per_s": T / (ms / 1e3), "tflops": tflops, "tc_peak_frac": tflops / pk["bf16_tflops"],
-            "launches_per_step": launches,
+            "launches_per_step": launches, "clocks": clk,
             "roofline": {"bound": "hbm", "kernel": f"la_prefill_backward (whole call, {launches:g} launches)",
                          "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                          "traffic": None, "algorithmic_bytes": alg_bytes}}
@@ -681,8 +701,9 @@ def run_mixed(la, dev, stream, args, pk, pg, local):
             raise RuntimeError(f"la_decode_step (continuations) failed: {la.STATUS.get(s, s)}")
 
     n = 10
-    ms, kms, launches = _timed_calls(la, dev, stream, pg, local, mixed, n, max(3, args.warmup))
-    ms_split, _, launches_split = _timed_calls(la, dev, stream, pg, local, split, n, max(3, args.warmup))
+    ms, kms, launches, clk = _timed_calls(la, dev, stream, pg, local, mixed, n, max(3, args.warmup))
+    ms_split, _, launches_split, clk_split = _timed_calls(la, dev, stream, pg, local, split, n,
+                                                          max(3, args.warmup))
     del q, k, v, o, init, st, ws, state_c
     alg_bytes = 8 * d * T * H + 8 * d * d * nseq * H
     gbs = alg_bytes / (ms / 1e3) / 1e9
@@ -691,6 +712,7 @@ def run_mixed(la, dev, stream, args, pk, pg, local):
             "ms_per_step": ms, "kernel_ms": kms, "launches_per_step": launches,
             "split_ms_per_step": ms_split, "split_launches_per_step": launches_split,
             "one_launch_over_split": ms / ms_split, "tokens_per_s": T / (ms / 1e3),
+            "clocks": clk, "split_clocks": clk_split,
             "roofline": {"bound": "hbm", "kernel": "prefill_chain_kernel (state-output instance)", "achieved": gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes": alg_bytes}}
