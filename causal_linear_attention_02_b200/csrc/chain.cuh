@@ -385,6 +385,88 @@ __device__ __forceinline__ bool weight_block(const Cursor& c, const Params& p, B
     return true;
 }
 
+// Anti-causal instance, the block walked after a sequence's ragged last block (walked first):
+// that block's rows past the sequence end belong to the next sequence, so its state MMAs were
+// skipped; its 1..B-1 tokens' k^T v (row m of the state, this CTA's 64 value columns) is added
+// here on CUDA cores to what the accumulator holds (S0, seeded at the first block, or nothing),
+// and written back for the later blocks' MMAs to add onto. Out of line: a cold path, once per
+// sequence at most. Ends with the TMEM stores complete.
+__device__ __noinline__ void rev_ragged_state(const Params& p, uint32_t tkv, int m, int tok_first, int tok_end,
+                                              int h, int half) {
+    if (p.init) tc_fence_after();
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {                     // one 32-column half at a time
+        float x[32];
+        if (p.init) {
+            uint32_t a[32];
+            tmem_ld_x32(tkv + 32 * hh, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(a[q]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) x[q] = 0.f;
+        }
+        for (int t = tok_first; t < tok_end; ++t) {
+            const float ki = __bfloat162float(p.k[((int64_t)t * p.H + h) * D + m]);
+            const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + h) * D + DV * half + 32 * hh);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const uint4 u = __ldg(vr + g);
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x[8 * g + 2 * e] = fmaf(ki, __uint_as_float(w4[e] << 16), x[8 * g + 2 * e]);
+                    x[8 * g + 2 * e + 1] = fmaf(ki, __uint_as_float(w4[e] & 0xffff0000u), x[8 * g + 2 * e + 1]);
+                }
+            }
+        }
+        uint32_t a[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(x[q]);
+        tmem_st_x32(tkv + 32 * hh, a);
+    }
+    tmem_wait_st();
+}
+
+// State-output instance, a work item's last block: row m of the final state (this CTA's 64
+// value columns) = the accumulator (zero when no MMA ever ran: `none`) plus the tokens
+// tok_first..tok_end-1 past the last full 16-key MMA step, on CUDA cores (with decay each
+// weighted by lambda^(tok_end - 1 - t)), stored to state_out. Out of line and a 32-column half
+// at a time, so it adds no register pressure to the pipeline roles.
+template <bool kDecay>
+__device__ __noinline__ void write_final_state(const Params& p, uint32_t tkv, int m, bool none, int tok_first,
+                                               int tok_end, int seq, int h, int half) {
+    float* row = p.state_out + (((int64_t)seq * p.H + h) * D + m) * D + DV * half;
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+        float x[32];
+        uint32_t a[32];
+        tmem_ld_x32(tkv + 32 * hh, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) x[q] = none ? 0.f : __uint_as_float(a[q]);
+        for (int t = tok_first; t < tok_end; ++t) {
+            float ki = __bfloat162float(p.k[((int64_t)t * p.H + h) * D + m]);
+            if constexpr (kDecay) ki *= decay_pow(log2f(__ldg(p.decay + h)), tok_end - 1 - t);
+            const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + h) * D + DV * half + 32 * hh);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const uint4 u = __ldg(vr + g);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    x[8 * g + 2 * e] += ki * __uint_as_float(w[e] << 16);
+                    x[8 * g + 2 * e + 1] += ki * __uint_as_float(w[e] & 0xffff0000u);
+                }
+            }
+        }
+        float4* dst = reinterpret_cast<float4*>(row + 32 * hh);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+    }
+}
+
 // State-output instance, after the CTA's chain work: the one-token sequences of the batch
 // (a serving batch's continuations, each with its carried-in state) are one recurrent
 // step each, the decode step's arithmetic at HBM rate instead of a chain work item:
@@ -976,8 +1058,17 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                                                       c0 + 1 <= lim ? __uint_as_float(a[2 * q + 1]) : 0.f);
                     }
                 }
+                if constexpr (kRev || kStateOut) {
+                    // these instances store each half as soon as it is packed (16 packed words
+                    // live instead of 32: no spills in their larger code)
+                    uint32_t ph[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) ph[q] = pk[16 * hh + q];
+                    tmem_st_x16(ts + 16 * hh, ph);
+                }
             }
-            tmem_st_x32(ts, pk);             // P of these 64 keys over the first 32 of their columns
+            // P of these 64 keys over the first 32 of their columns
+            if constexpr (!kRev && !kStateOut) tmem_st_x32(ts, pk);
             if constexpr (kDecay) {
                 if (c.first_of_sub()) {
                     // lambda^(r+1) q_r over the other 32 columns: head dims 64 hk .. 64 hk + 63 of
@@ -1076,54 +1167,17 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             // anti-causal: the block walked after a ragged first block (the sequence's last)
             // takes that block's state on CUDA cores instead of from its (skipped) MMAs
             const int nbk = (c.bk.len + (1 << p.log2B) - 1) >> p.log2B;
-            if (kRev && !c.bk.first && c.b == nbk - 2 && (c.bk.len & ((1 << p.log2B) - 1)) != 0) {
-                float x[DV];
-                if (p.init) {                              // S0, seeded at the first block
-                    tc_fence_after();
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t a[32];
-                        tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) x[32 * hh + q] = __uint_as_float(a[q]);
-                    }
+            const bool ragged_next = kRev && !c.bk.first && c.b == nbk - 2 && (c.bk.len & ((1 << p.log2B) - 1)) != 0;
+            if (ragged_next || !c.bk.first) {
+                if (ragged_next) {
+                    rev_ragged_state(p, tmem + lane_base + TM_KV, m, c.bk.tok_s + ((nbk - 1) << p.log2B),
+                                     c.bk.tok_s + c.bk.len, c.h, c.half);
                 } else {
-#pragma unroll
-                    for (int q = 0; q < DV; ++q) x[q] = 0.f;
+                    if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
+                    ++kvc;
+                    if (wt == 0) LA_CTRACE(c.n, TR_XR);
+                    tc_fence_after();
                 }
-                for (int t = c.bk.tok_s + ((nbk - 1) << p.log2B); t < c.bk.tok_s + c.bk.len; ++t) {
-                    const float ki = __bfloat162float(p.k[((int64_t)t * p.H + c.h) * D + m]);
-                    const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + c.h) * D + DV * c.half);
-#pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        const uint4 u = __ldg(vr + g);
-                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            x[8 * g + 2 * e] = fmaf(ki, __uint_as_float(w4[e] << 16), x[8 * g + 2 * e]);
-                            x[8 * g + 2 * e + 1] = fmaf(ki, __uint_as_float(w4[e] & 0xffff0000u), x[8 * g + 2 * e + 1]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t a[32];
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) a[q] = __float_as_uint(x[32 * hh + q]);
-                    tmem_st_x32(tmem + lane_base + TM_KV + 32 * hh, a);   // the later blocks' MMAs add onto it
-#pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        pk[16 * hh + q] = pack_bf16x2(x[32 * hh + 2 * q], x[32 * hh + 2 * q + 1]);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bars->kv_read[c.n & 3]);            // the accumulator may take this block's keys
-            } else if (!c.bk.first) {
-                if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
-                ++kvc;
-                if (wt == 0) LA_CTRACE(c.n, TR_XR);
-                tc_fence_after();
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t a[32];
@@ -1181,36 +1235,9 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 if (!warp_all(wait_bar(&bars->kv_ready, kvc & 1, ab))) { ok = false; break; }
                 ++kvc;
                 tc_fence_after();
-                float x[DV];
                 // with no carried-in state and fewer than 16 tokens no MMA ever ran
-                const bool none = p.init == nullptr && c.bk.len < 16;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t a[32];
-                    tmem_ld_x32(tmem + lane_base + TM_KV + 32 * hh, a);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) x[32 * hh + q] = none ? 0.f : __uint_as_float(a[q]);
-                }
-                // the tokens past the last full 16-key step, on CUDA cores
-                for (int t = c.tok0 + (c.rows & ~15); t < c.tok0 + c.rows; ++t) {
-                    float ki = __bfloat162float(p.k[((int64_t)t * p.H + c.h) * D + m]);
-                    if constexpr (kDecay) ki *= decay_pow(log2f(__ldg(p.decay + c.h)), c.tok0 + c.rows - 1 - t);
-                    const uint4* vr = reinterpret_cast<const uint4*>(p.v + ((int64_t)t * p.H + c.h) * D + DV * c.half);
-#pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        const uint4 u = __ldg(vr + g);
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            x[8 * g + 2 * e] += ki * __uint_as_float(w[e] << 16);
-                            x[8 * g + 2 * e + 1] += ki * __uint_as_float(w[e] & 0xffff0000u);
-                        }
-                    }
-                }
-                float4* dst = reinterpret_cast<float4*>(p.state_out + (((int64_t)c.seq * p.H + c.h) * D + m) * D + DV * c.half);
-#pragma unroll
-                for (int q = 0; q < DV / 4; ++q) dst[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+                write_final_state<kDecay>(p, tmem + lane_base + TM_KV, m, p.init == nullptr && c.bk.len < 16,
+                                          c.tok0 + (c.rows & ~15), c.tok0 + c.rows, c.seq, c.h, c.half);
             }
             c.next_block(p);
         }
