@@ -1058,17 +1058,14 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                                                       c0 + 1 <= lim ? __uint_as_float(a[2 * q + 1]) : 0.f);
                     }
                 }
-                if constexpr (kRev || kStateOut) {
-                    // these instances store each half as soon as it is packed (16 packed words
-                    // live instead of 32: no spills in their larger code)
-                    uint32_t ph[16];
+                // P of these 64 keys goes over the first 32 of their columns, each half as soon
+                // as it is packed: the store overlaps the next half's load, and 16 packed words
+                // are live instead of 32 (no spills in the larger instances)
+                uint32_t ph[16];
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) ph[q] = pk[16 * hh + q];
-                    tmem_st_x16(ts + 16 * hh, ph);
-                }
+                for (int q = 0; q < 16; ++q) ph[q] = pk[16 * hh + q];
+                tmem_st_x16(ts + 16 * hh, ph);
             }
-            // P of these 64 keys over the first 32 of their columns
-            if constexpr (!kRev && !kStateOut) tmem_st_x32(ts, pk);
             if constexpr (kDecay) {
                 if (c.first_of_sub()) {
                     // lambda^(r+1) q_r over the other 32 columns: head dims 64 hk .. 64 hk + 63 of
