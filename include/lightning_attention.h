@@ -80,8 +80,11 @@ typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
  * the on-chip-state kernel (one CTA per sequence, head and half of the value
  * columns, the running state kept in tensor memory) when num_seqs * heads * 2
  * >= 64, else the block-parallel kernel (block prefixes by a single-pass
- * decoupled look-back scan); la_debug_set_path overrides the choice. Every
- * other supported combination runs on the CUDA-core (SIMT) path.
+ * decoupled look-back scan; its CTAs take (block, head) tiles by atomic
+ * ticket, so a tile only ever waits on tiles drawn earlier by CTAs already
+ * running, and the launch finishes even while another kernel holds SMs);
+ * la_debug_set_path overrides the choice. Every other supported combination
+ * runs on the CUDA-core (SIMT) path.
  */
 
 /* Bytes of device workspace la_prefill needs for these sizes (0 if unsupported). */
@@ -151,8 +154,13 @@ la_status la_state_from_prefill(const void* k, const void* v, const int32_t* cu_
  * On the on-chip-state path (bf16, d = 128, B in {128, 256}, at least 64
  * (sequence, head, value-half) work items) this is one pass: the prefill
  * kernel's accumulator already holds the running state, and the kernel writes
- * it out after each sequence's last block. Elsewhere it is la_prefill followed
- * by la_state_from_prefill. state_out may be init_state itself (in-place
+ * it out after each sequence's last block. Sequences of one token (a serving
+ * batch's continuations) are not work items there: at the end of the same
+ * launch they are run as decode steps, S = S0 + k^T v, o = q S0 + (q . k) v,
+ * at close to the HBM rate of their states (page "MiniMax-01 Lightning
+ * Attention", section "计算优化": prefill and decode kept apart, fused into one
+ * batched launch). Elsewhere it is la_prefill followed by
+ * la_state_from_prefill. state_out may be init_state itself (in-place
  * update); it must not overlap q, k, v, o or the workspace otherwise. The
  * workspace is la_prefill_with_state_workspace_size bytes. Errors as
  * la_prefill, plus LA_ERR_INVALID_ARGUMENT for a NULL state_out.
