@@ -1,12 +1,14 @@
 // Helpers of the prefill's backward pass (the training pass; the pages give the
 // forward only). With S_t = S0 + sum_{s <= t} k_s^T v_s and L = sum_t dO_t . O_t:
 //   dQ_t = dO_t S_t^T                    -> a forward prefill of (dO, V, K) from S0^T
-//   dV_s = sum_{t >= s} (k_s . q_t) dO_t -> a forward prefill of (K, Q, dO) over the
-//   dK_s = sum_{t >= s} (dO_t . v_s) q_t    reversed sequences, reversed back; and
-//                                        -> a forward prefill of (V, dO, Q) likewise
+//   dV_s = sum_{t >= s} (k_s . q_t) dO_t -> an anti-causal prefill of (K, Q, dO)
+//   dK_s = sum_{t >= s} (dO_t . v_s) q_t -> an anti-causal prefill of (V, dO, Q)
 //   dS0  = sum_t q_t^T dO_t              -> the state of (Q, dO)
-// so the pass reuses the forward kernels. These kernels reverse the token order
-// inside every sequence and transpose the carried-in states.
+// so the pass reuses the forward kernels. The on-chip-state kernel has an
+// anti-causal instance; on the other paths (and with decay) the anti-causal
+// prefills are causal prefills over every sequence reversed, reversed back.
+// These kernels reverse the token order inside every sequence (that path) and
+// transpose the carried-in states.
 #pragma once
 
 #include "common.cuh"

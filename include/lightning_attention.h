@@ -181,18 +181,22 @@ la_status la_prefill_with_state(const void* q, const void* k, const void* v, voi
  *   dk_s = v_s R_s^T,  dv_s = k_s R_s,  R_s = sum_{t >= s, same sequence} q_t^T dout_t
  *   dinit_state = R at each sequence's first token (= sum_t q_t^T dout_t)
  * Computed with the forward kernels: dq is a prefill of (dout, v, k) from
- * init_state^T; dv and dk are prefills of (k, q, dout) and (v, dout, q) over
- * every sequence reversed, reversed back; dinit_state is la_state_from_prefill
- * of (q, dout). Rounding is that of those prefills (bf16 operands, fp32
- * accumulation; bf16 outputs for bf16 inputs).
+ * init_state^T; dv and dk are anti-causal prefills (keys at or after each
+ * query) of (k, q, dout) and (v, dout, q): on the on-chip-state path by that
+ * kernel's anti-causal instance, which walks each sequence's blocks from the
+ * last, elsewhere by causal prefills over every sequence reversed, reversed
+ * back; dinit_state is la_state_from_prefill of (q, dout). Rounding is that of
+ * those prefills (bf16 operands, fp32 accumulation; bf16 outputs for bf16
+ * inputs).
  *   q, k, v, dout     in   [total_tokens][heads][d], dtype (device)
  *   init_state        in   fp32 [num_seqs][heads][d][d] or NULL (the forward's S0)
  *   dq, dk, dv        out  [total_tokens][heads][d], dtype; no overlap with the
  *                          inputs, each other or the workspace
  *   dinit_state       out  fp32 [num_seqs][heads][d][d], or NULL (not computed)
  * Shapes, dtypes and errors as la_prefill; the workspace is
- * la_prefill_backward_workspace_size bytes (five [T][H][d] tensors plus the
- * prefill's and the state pass's workspaces), 256-byte aligned, caller-owned.
+ * la_prefill_backward_workspace_size bytes (on the reversal path five
+ * [T][H][d] tensors, plus the prefill's and the state pass's workspaces),
+ * 256-byte aligned, caller-owned.
  * Asynchronous on `stream`; allocates nothing.
  */
 size_t la_prefill_backward_workspace_size(int64_t total_tokens, int num_seqs, int heads, int d, int B,
